@@ -1,0 +1,229 @@
+"""CPU oracle of the neighbour-graph hot path (TEST INFRASTRUCTURE).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product path (the CUDA library and
+its binding) never imports, links or runs anything here, and this package
+never imports the product.
+
+The arithmetic lives in ``mlg_oracle.c`` (plain C, fp64, no contraction),
+compiled to ``liboracle.so`` beside it. This module only marshals numpy
+arrays. Each function names the passage it follows; the C file's header
+states the definitions in full:
+
+* neighbour CSR -- deepmd-kit issue "DPA4 .pt2 LAMMPS (C++ AOTI) inference
+  3-6x slower than Python (ASE)", Root cause analysis (createEdgeTensors():
+  edge index and edge vector per neighbour pair), and issue "NeighborGraph
+  attention is 4-9x slower than dense", Proposed fix (destination CSR);
+* per-centre cap -- the same issues, Reproduction (sel=181) and Measurements
+  (nsel 120 / rcut 6, nsel 40 / rcut 4);
+* attention -- NeighborGraph issue, Proposed fix (dense per-centre attention
+  with per-row masks) and Root cause (the dense route's per-centre
+  (nloc, nnei, nnei) batched products).
+
+Parity of the switch cosine, the neighbour set and the attention is pinned by
+the ``-m "not gpu"`` tests in ``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mlg_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CFLAGS = ["-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+          "-shared", "-fPIC", "-Wall"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``mlg_oracle.c`` into ``liboracle.so`` (gcc)."""
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            i64, i32, dbl = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+            p = ctypes.c_void_p
+            lib.oracle_cos_pi.restype = dbl
+            lib.oracle_cos_pi.argtypes = [dbl]
+            lib.oracle_switch.restype = None
+            lib.oracle_switch.argtypes = [i64, p, dbl, dbl, p]
+            lib.oracle_count.restype = ctypes.c_int
+            lib.oracle_count.argtypes = [i64, p, p, p, dbl, i32, p, p, ctypes.c_int]
+            lib.oracle_fill.restype = ctypes.c_int
+            lib.oracle_fill.argtypes = [i64, p, p, p, dbl, dbl, i32, p, p, p, p, p, p,
+                                        ctypes.c_int]
+            lib.oracle_centre.restype = i64
+            lib.oracle_centre.argtypes = [i64, p, p, p, dbl, dbl, i32, i64, i64, p, p, p, p,
+                                          p, p]
+            lib.oracle_attention.restype = ctypes.c_int
+            lib.oracle_attention.argtypes = [i64, p, p, i32, i32, p, p, p, p, p, ctypes.c_int]
+            lib.oracle_attention_map.restype = ctypes.c_int
+            lib.oracle_attention_map.argtypes = [p, p, i32, i32, p, p, p, i64, i32, p]
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _geom_args(coords, box, pbc):
+    coords = np.ascontiguousarray(coords, dtype=np.float64).reshape(-1, 3)
+    box = np.ascontiguousarray(box, dtype=np.float64).reshape(3, 3)
+    pbc = np.ascontiguousarray(pbc, dtype=np.uint8).reshape(3)
+    return coords, box, pbc
+
+
+def cos_pi(u: float) -> float:
+    """This project's reproducible cos(pi u) (Taylor series of sin)."""
+    return _load().oracle_cos_pi(float(u))
+
+
+def switch(r, rcut: float, r_on: float) -> np.ndarray:
+    """Smooth cosine switch s(r): 1 below r_on, 0 at rcut and beyond.
+
+    NeighborGraph issue, Measurements ("graph smooth" / "dense smooth"); the
+    onset r_on and the cosine shape follow the benchmark system definitions.
+    """
+    r = np.ascontiguousarray(r, dtype=np.float64).ravel()
+    s = np.empty_like(r)
+    _load().oracle_switch(r.size, _ptr(r), float(rcut), float(r_on), _ptr(s))
+    return s
+
+
+def counts(coords, box, pbc, rcut: float, nnei_max: int, nthreads: int = 0):
+    """Per-centre kept count min(raw, nnei_max) and raw in-cutoff count."""
+    coords, box, pbc = _geom_args(coords, box, pbc)
+    n = coords.shape[0]
+    kept = np.zeros(n, dtype=np.int32)
+    raw = np.zeros(n, dtype=np.int64)
+    rc = _load().oracle_count(n, _ptr(coords), _ptr(box), _ptr(pbc), float(rcut),
+                              int(nnei_max), _ptr(kept), _ptr(raw), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_count failed ({rc})")
+    return kept, raw
+
+
+def build_csr(coords, box, pbc, rcut: float, r_on: float, nnei_max: int,
+              nthreads: int = 0) -> dict:
+    """The whole destination-sorted CSR by brute force.
+
+    Returns row_ptr int64 [N+1], src int32 [E], shift int32 [E][3], vec
+    float64 [E][3] (source image minus destination), dist float64 [E],
+    sw float64 [E], raw int64 [N], n_truncated.
+    """
+    coords, box, pbc = _geom_args(coords, box, pbc)
+    n = coords.shape[0]
+    kept, raw = counts(coords, box, pbc, rcut, nnei_max, nthreads)
+    row_ptr = np.zeros(n + 1, dtype=np.int64)
+    np.cumsum(kept, out=row_ptr[1:])
+    e = int(row_ptr[-1])
+    src = np.zeros(e, dtype=np.int32)
+    shift = np.zeros((e, 3), dtype=np.int32)
+    vec = np.zeros((e, 3), dtype=np.float64)
+    dist = np.zeros(e, dtype=np.float64)
+    sw = np.zeros(e, dtype=np.float64)
+    rc = _load().oracle_fill(n, _ptr(coords), _ptr(box), _ptr(pbc), float(rcut), float(r_on),
+                             int(nnei_max), _ptr(row_ptr), _ptr(src), _ptr(shift), _ptr(vec),
+                             _ptr(dist), _ptr(sw), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_fill failed ({rc})")
+    return {"row_ptr": row_ptr, "src": src, "shift": shift, "vec": vec, "dist": dist,
+            "sw": sw, "raw": raw, "n_truncated": int(np.count_nonzero(raw > nnei_max))}
+
+
+def centre(coords, box, pbc, rcut: float, r_on: float, nnei_max: int, i: int) -> dict:
+    """The kept edges of one destination ``i`` (brute force over all sources)."""
+    coords, box, pbc = _geom_args(coords, box, pbc)
+    n = coords.shape[0]
+    cap = int(nnei_max)
+    src = np.zeros(cap, dtype=np.int32)
+    shift = np.zeros((cap, 3), dtype=np.int32)
+    vec = np.zeros((cap, 3), dtype=np.float64)
+    dist = np.zeros(cap, dtype=np.float64)
+    sw = np.zeros(cap, dtype=np.float64)
+    raw = np.zeros(1, dtype=np.int64)
+    k = _load().oracle_centre(n, _ptr(coords), _ptr(box), _ptr(pbc), float(rcut), float(r_on),
+                              int(nnei_max), int(i), cap, _ptr(src), _ptr(shift), _ptr(vec),
+                              _ptr(dist), _ptr(sw), _ptr(raw))
+    if k < 0:
+        raise ValueError(f"oracle_centre failed ({k})")
+    return {"src": src[:k], "shift": shift[:k], "vec": vec[:k], "dist": dist[:k],
+            "sw": sw[:k], "raw": int(raw[0])}
+
+
+def _as_f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def attention(row_ptr, sw, G, Wq, Wk, Wv, heads: int, nthreads: int = 0) -> np.ndarray:
+    """One block-dense attention layer over every centre of the CSR.
+
+    NeighborGraph issue, Proposed fix: per centre, Q = G Wq, K = G Wk,
+    V = G Wv; per head l_ab = s_a s_b (q_a . k_b) / sqrt(d), softmax over the
+    centre's real edges, O_a = sum_b P_ab V_b, heads concatenated. Computed in
+    fp64 from whatever precision the inputs hold.
+    """
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int64)
+    sw, G = _as_f64(sw), _as_f64(G)
+    Wq, Wk, Wv = _as_f64(Wq), _as_f64(Wk), _as_f64(Wv)
+    c = G.shape[1]
+    out = np.zeros_like(G)
+    rc = _load().oracle_attention(row_ptr.size - 1, _ptr(row_ptr), _ptr(sw), c, int(heads),
+                                  _ptr(G), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(out),
+                                  int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_attention failed ({rc})")
+    return out
+
+
+def attention_map(row_ptr, sw, G, Wq, Wk, heads: int, i: int, h: int) -> np.ndarray:
+    """Softmax map P[a][b] of centre ``i``, head ``h``."""
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int64)
+    sw, G, Wq, Wk = _as_f64(sw), _as_f64(G), _as_f64(Wq), _as_f64(Wk)
+    n = int(row_ptr[i + 1] - row_ptr[i])
+    P = np.zeros((max(n, 0), max(n, 0)), dtype=np.float64)
+    rc = _load().oracle_attention_map(_ptr(row_ptr), _ptr(sw), G.shape[1], int(heads), _ptr(G),
+                                      _ptr(Wq), _ptr(Wk), int(i), int(h), _ptr(P))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_map failed ({rc})")
+    return P
+
+
+def forward(row_ptr, sw, G0, W, heads: int, dtype: str = "f64", nthreads: int = 0):
+    """Stacked attention layers G^{l+1} = attention(G^l); returns every layer.
+
+    ``W`` is [n_layers][3][c][c]. For fp32 workloads (``dtype == "f32"``) the
+    inputs are the fp32-rounded values, s(r) is rounded to fp32 as the fp32
+    kernels read it, each layer is computed in fp64 and its output rounded to
+    fp32 before it feeds the next layer (the fp32 path stores every layer in
+    fp32).
+    """
+    sw = np.asarray(sw, dtype=np.float64)
+    if dtype == "f32":
+        sw = sw.astype(np.float32).astype(np.float64)
+    outs = []
+    g = np.asarray(G0)
+    for layer in range(np.asarray(W).shape[0]):
+        o = attention(row_ptr, sw, g, W[layer][0], W[layer][1], W[layer][2], heads, nthreads)
+        if dtype == "f32":
+            o = o.astype(np.float32)
+        outs.append(o)
+        g = o
+    return outs

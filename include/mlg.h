@@ -1,0 +1,200 @@
+/*
+ * mlg.h -- C ABI of the B200 neighbour-graph library (libmlg.so).
+ *
+ * Two stages of machine-learned interatomic potential inference, entirely on
+ * one GPU:
+ *
+ *   1. mlg_build_csr: an O(N) cell-list search for every periodic neighbour
+ *      image within rcut, emitted as a destination-sorted CSR edge list
+ *      (row_ptr, source index, integer image shift, edge vector, distance,
+ *      smooth switch s(r)).  It replaces the host-side edge construction and
+ *      the host-to-device copies that the deepmd-kit issue "DPA4 .pt2 LAMMPS
+ *      (C++ AOTI) inference 3-6x slower than Python (ASE) due to CPU-side
+ *      edge construction and data marshalling" measures as the bottleneck
+ *      (Root cause analysis, bottlenecks 1 and 2: createEdgeTensors() and the
+ *      synchronising copies), and it produces the destination CSR
+ *      (destination_order / destination_row_ptr) that the deepmd-kit issue
+ *      "NeighborGraph attention is 4-9x slower than dense and OOM-prone --
+ *      move to block-dense attention via the destination CSR" builds on
+ *      (Proposed fix).
+ *
+ *   2. mlg_block_attention: block-dense multi-head attention of every centre
+ *      over its own edges (NeighborGraph issue, Proposed fix: gather the
+ *      compact per-centre block through destination_row_ptr, run the dense
+ *      attention math with per-row masks for ragged tails, write back to the
+ *      edge axis; no (sum nnei^2, c) pair-axis tensor ever exists).
+ *
+ *   mlg_forward runs stage 1 and then n_layers of stage 2.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named "device" are CUDA device pointers (e.g. the data_ptr()
+ *    of a torch CUDA tensor); they are owned by the caller, never freed or
+ *    retained by the library.  Structs passed by pointer are read during the
+ *    call only (host memory).
+ *  - Every call is asynchronous and stream-ordered on `stream` (a
+ *    cudaStream_t; NULL = the legacy default stream).  The library never
+ *    synchronises, never allocates device or pinned memory, keeps no state
+ *    between calls and may be called from several host threads on different
+ *    streams with different workspaces.
+ *  - The return value is the host-side status (mlg_status): argument and
+ *    workspace checks, and the launch result (cudaGetLastError).  Errors that
+ *    depend on device data are OR-ed into the device word csr->status
+ *    (mlg_status_bits); read it after synchronising the stream.
+ *  - Coordinates and geometry are fp64 always.  Attention features and
+ *    weights are fp32 (MLG_F32) or fp64 (MLG_F64).
+ */
+#ifndef MLG_H
+#define MLG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the runtime's opaque stream handle). */
+typedef struct CUstream_st* mlg_stream_t;
+
+/* Host-side return codes. */
+typedef enum {
+    MLG_OK = 0,
+    MLG_ERR_INVALID_ARG = 1,  /* a NULL pointer, a non-positive size, rcut <= r_on, a non-finite box */
+    MLG_ERR_WORKSPACE = 2,    /* ws_bytes smaller than the matching *_workspace_bytes() */
+    MLG_ERR_CAPACITY = 3,     /* capacity < 0 */
+    MLG_ERR_INPUT_DATA = 4,   /* reserved for host-visible data errors */
+    MLG_ERR_UNSUPPORTED = 5,  /* a shape this build does not handle (see each call) */
+    MLG_ERR_CUDA = 6          /* a CUDA launch error (cudaGetLastError) */
+} mlg_status;
+
+/* Bits OR-ed into the device word csr->status. */
+typedef enum {
+    MLG_STATUS_NONFINITE_COORD = 1u, /* an atom had a NaN/Inf coordinate; it has no edges */
+    MLG_STATUS_TYPE_RANGE = 2u,      /* a type outside [0, n_types) */
+    MLG_STATUS_CAPACITY = 4u,        /* E > capacity: row_ptr and n_edges are complete,
+                                        edges at index >= capacity were not written,
+                                        attention skipped */
+    MLG_STATUS_IMAGE_RANGE = 8u,     /* an atom lies more than 511 box lengths outside the
+                                        box along a periodic axis; it was left out */
+    MLG_STATUS_TIES = 16u,           /* truncation met more than 256 candidates at one
+                                        distance; the kept set is not canonical */
+    MLG_STATUS_INTERNAL = 32u        /* the count and fill passes disagreed on a row (never
+                                        expected); that row is incomplete */
+} mlg_status_bits;
+
+/* Arithmetic type of attention features and weights. */
+typedef enum { MLG_F32 = 0, MLG_F64 = 1 } mlg_dtype;
+
+/* The atomic system (DPA4 LAMMPS issue, Reproduction: coordinates as double,
+ * atom types; the box and periodicity of the simulation cell). */
+typedef struct {
+    int64_t n_atoms;        /* N >= 1 */
+    const double* coords;   /* device [N][3], Angstrom; any values (need not be wrapped) */
+    const int32_t* types;   /* device [N] or NULL; validated into MLG_STATUS_TYPE_RANGE,
+                               not used by the attention */
+    int32_t n_types;        /* >= 1 when types != NULL */
+    double box[9];          /* HOST, row-major rows a1, a2, a3 (Angstrom).  Every entry must be
+                               finite.  Along a periodic axis k the row a_k must be (0..L_k..0)
+                               with L_k > 0 (orthorhombic cells; a sheared cell returns
+                               MLG_ERR_UNSUPPORTED).  Rows of open axes are not used for
+                               images (the shift is 0 there). */
+    uint8_t pbc[3];         /* HOST, 1 = periodic along axis k, 0 = open */
+} mlg_system;
+
+/* The destination CSR (NeighborGraph issue, Proposed fix: destination_order /
+ * destination_row_ptr).  All arrays are caller-owned DEVICE memory.
+ *
+ * Edges of destination i are rows [row_ptr[i], row_ptr[i+1]).  Inside a
+ * destination they are in canonical order of (source, shift x, shift y,
+ * shift z), ascending.  A destination with more than nnei_max in-cutoff
+ * neighbours keeps the nnei_max nearest, ties broken by (source, shift).
+ * For edge e of destination i with source j and shift S:
+ *   vec[e]  = (x_j + S_0 a1 + S_1 a2 + S_2 a3) - x_i,   fp64, rounded per op
+ *   dist[e] = |vec[e]| < rcut,                          fp64, IEEE sqrt
+ *   sw[e]   = s(dist): 1 below r_on, 0.5 (1 + cos(pi u)) with
+ *             u = (dist - r_on) / (rcut - r_on) up to rcut.
+ * N * nnei_max rows always suffice for `capacity`. */
+typedef struct {
+    int64_t capacity;       /* rows available in src/shift/vec/dist/sw (and in attention G) */
+    int64_t* row_ptr;       /* [N + 1] */
+    int32_t* src;           /* [capacity] */
+    int32_t* shift;         /* [capacity][3] */
+    double* vec;            /* [capacity][3] */
+    double* dist;           /* [capacity] */
+    double* sw;             /* [capacity] */
+    int64_t* n_edges;       /* device scalar: E = row_ptr[N] */
+    int64_t* n_truncated;   /* device scalar: destinations with more than nnei_max neighbours */
+    uint32_t* status;       /* device scalar: mlg_status_bits */
+} mlg_csr;
+
+/* Bytes of device workspace that mlg_build_csr needs for this system.  The
+ * cell grid depends on N, rcut, the box and pbc (not on the coordinates).
+ * Returns 0 for invalid arguments. */
+size_t mlg_build_csr_workspace_bytes(int64_t n_atoms, double rcut, const double box[9],
+                                     const uint8_t pbc[3]);
+
+/* Build the destination CSR of `sys` (see mlg_csr).  Resets *csr->status,
+ * *csr->n_truncated; writes row_ptr, n_edges and min(E, capacity) edges.
+ *   rcut      cutoff radius (> r_on > 0); strict r < rcut
+ *   r_on      onset of the cosine switch
+ *   nnei_max  per-destination cap (sel), 1..256, else MLG_ERR_UNSUPPORTED
+ *   ws        device workspace of ws_bytes >= mlg_build_csr_workspace_bytes(), 256-byte aligned
+ * The result is deterministic: bitwise identical across calls, streams and GPUs. */
+int mlg_build_csr(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+                  const mlg_csr* csr, void* ws, size_t ws_bytes, mlg_stream_t stream);
+
+/* Bytes of device workspace that mlg_block_attention needs (0 in this build). */
+size_t mlg_attention_workspace_bytes(int64_t n_centres, int32_t nnei_max, int32_t channels,
+                                     int32_t heads, mlg_dtype dtype);
+
+/* One block-dense attention layer over every destination of `csr`.
+ *   G_in, G_out  device [capacity][channels] in CSR edge order, dtype; rows >= E are not
+ *                touched.  G_out must not alias G_in.
+ *   Wq, Wk, Wv   device [channels][channels] row-major, y = x W (q = g Wq)
+ *   channels % heads == 0; head size d = channels / heads <= 64; channels <= 256
+ * Per destination i with n edges (rows a, b < n), per head h (columns h d .. h d + d):
+ *   l_ab = s_a s_b (q_a . k_b) / sqrt(d);  P_ab = exp(l_ab - max_b l) / sum_b exp(...);
+ *   G_out[a, h d + t] = sum_b P_ab v_b[t].
+ * Slots beyond a destination's n edges do not exist (masked).  Reads E from csr->row_ptr
+ * on the device; if *csr->status has MLG_STATUS_CAPACITY set, nothing is written. */
+int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                        int32_t channels, int32_t heads, mlg_dtype dtype, const void* G_in,
+                        void* G_out, const void* Wq, const void* Wk, const void* Wv, void* ws,
+                        size_t ws_bytes, mlg_stream_t stream);
+
+/* Bytes of device workspace for mlg_forward: the build's workspace plus, for
+ * n_layers >= 2, one [capacity][channels] buffer for the layer ping-pong. */
+size_t mlg_forward_workspace_bytes(int64_t n_atoms, double rcut, const double box[9],
+                                   const uint8_t pbc[3], int64_t capacity, int32_t channels,
+                                   int32_t n_layers, mlg_dtype dtype);
+
+/* mlg_build_csr followed by n_layers attention layers G^{l+1} = attention(G^l).
+ *   W   HOST array of 3 * n_layers device pointers: Wq, Wk, Wv of layer 0, then layer 1, ...
+ *   G0  device [capacity][channels]: edge features in the canonical order of the graph
+ *       this call builds (the build is deterministic, so a previous build of the same
+ *       coordinates gives that order)
+ *   G_out device [capacity][channels], must not alias G0
+ * Everything runs on `stream` without a host synchronisation (CUDA-graph capturable). */
+int mlg_forward(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+                int32_t channels, int32_t heads, int32_t n_layers, mlg_dtype dtype,
+                const void* const* W, const void* G0, void* G_out, const mlg_csr* csr,
+                void* ws, size_t ws_bytes, mlg_stream_t stream);
+
+/* Number of kernel launches that one mlg_forward call with these arguments
+ * issues on its stream (for accounting in benchmarks); 0 for invalid
+ * arguments. */
+int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
+                             const uint8_t pbc[3], int32_t n_layers);
+
+/* A static string naming a host status code. */
+const char* mlg_status_string(int status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int mlg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLG_H */

@@ -1,0 +1,391 @@
+// mlg_api.cu -- the C ABI of libmlg.so: argument checks, workspace layout and
+// kernel launches on the caller's stream.  No allocation, no synchronisation.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "mlg.h"
+#include "mlg_common.cuh"
+#include "mlg_build.cuh"
+#include "mlg_attn.cuh"
+
+using namespace mlg;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxNnei = 256;
+constexpr int kMaxReach = 62;  // stencil reach limit (image packing of the sort key)
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Layout of the build workspace.
+struct BuildLayout {
+  size_t grid, bbox, cell_count, cell_start, atom_cell, atom_rank, atom_w, recs, kept, raw,
+      partial, total;
+};
+
+int64_t scan_tiles(int64_t n) { return (n + kScanTile - 1) / kScanTile; }
+
+BuildLayout build_layout(int64_t n, int ncell_cap) {
+  BuildLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  L.grid = take(sizeof(CellGrid));
+  L.bbox = take(6 * sizeof(unsigned long long));
+  L.cell_count = take((size_t)(ncell_cap + 1) * sizeof(int));
+  L.cell_start = take((size_t)(ncell_cap + 1) * sizeof(int));
+  L.atom_cell = take((size_t)n * sizeof(int));
+  L.atom_rank = take((size_t)n * sizeof(int));
+  L.atom_w = take((size_t)n * sizeof(int));
+  L.recs = take((size_t)n * sizeof(Rec));
+  L.kept = take((size_t)n * sizeof(int));
+  L.raw = take((size_t)n * sizeof(int));
+  int64_t tiles = scan_tiles(n > ncell_cap ? n : ncell_cap + 1);
+  L.partial = take((size_t)(tiles + 2) * sizeof(long long));
+  L.total = off;
+  return L;
+}
+
+bool finite_box(const double* box) {
+  for (int k = 0; k < 9; ++k)
+    if (!std::isfinite(box[k])) return false;
+  return true;
+}
+
+// Cell grid that the host can fix: cells along periodic axes (size >= rcut
+// plus a margin, so one layer of neighbouring cells covers rcut), caps along
+// open axes, the stencil reach, and the total cell budget.
+int make_plan(int64_t n, double rcut, const double* box, const uint8_t* pbc, BuildPlan* p) {
+  if (n < 1 || n > (int64_t)INT32_MAX / 2 || !(rcut > 0.0) || !std::isfinite(rcut) ||
+      box == nullptr || pbc == nullptr || !finite_box(box))
+    return MLG_ERR_INVALID_ARG;
+  std::memset(p, 0, sizeof(*p));
+  const double delta = 1e-6 * (rcut > 1.0 ? rcut : 1.0);
+  p->rcd = rcut + delta;
+  const double budget = (double)(n > 32 ? 2 * n : 64);
+  double prod = 1.0;
+  int n_open = 0;
+  for (int k = 0; k < 3; ++k) {
+    p->periodic[k] = pbc[k] ? 1 : 0;
+    if (!p->periodic[k]) {
+      ++n_open;
+      continue;
+    }
+    for (int c = 0; c < 3; ++c)
+      if (c != k && box[3 * k + c] != 0.0) return MLG_ERR_UNSUPPORTED;  // sheared cell
+    double L = box[3 * k + k];
+    if (!(L > 0.0)) return MLG_ERR_INVALID_ARG;
+    p->L[k] = L;
+    p->invL[k] = 1.0 / L;
+    double q = std::floor(L / p->rcd);
+    p->n_fixed[k] = q < 1.0 ? 1 : (q > 1024.0 ? 1024 : (int)q);
+    prod *= p->n_fixed[k];
+  }
+  // coarsen periodic axes until the grid fits the cell budget
+  while (prod > budget) {
+    int kmax = -1;
+    for (int k = 0; k < 3; ++k)
+      if (p->periodic[k] && (kmax < 0 || p->n_fixed[k] > p->n_fixed[kmax])) kmax = k;
+    if (kmax < 0 || p->n_fixed[kmax] == 1) break;
+    prod /= p->n_fixed[kmax];
+    p->n_fixed[kmax] = (p->n_fixed[kmax] + 1) / 2;
+    prod *= p->n_fixed[kmax];
+  }
+  for (int k = 0; k < 3; ++k) {
+    if (!p->periodic[k]) continue;
+    p->inv_h[k] = (double)p->n_fixed[k] / p->L[k];
+    double reach = std::ceil(p->rcd * (double)p->n_fixed[k] / p->L[k]);
+    if (reach > kMaxReach) return MLG_ERR_UNSUPPORTED;  // box far smaller than rcut
+    p->D_fixed[k] = reach < 1.0 ? 1 : (int)reach;
+  }
+  int open_cap = 1;
+  if (n_open > 0) {
+    double room = budget / prod;
+    open_cap = (int)std::floor(std::pow(room, 1.0 / n_open) + 1e-9);
+    if (open_cap < 1) open_cap = 1;
+    if (open_cap > 1024) open_cap = 1024;
+  }
+  double cells = prod;
+  for (int k = 0; k < 3; ++k)
+    if (!p->periodic[k]) {
+      p->n_open_max[k] = open_cap;
+      cells *= open_cap;
+    }
+  p->any_open = n_open > 0;
+  p->ncell_cap = (int)cells;
+  return MLG_OK;
+}
+
+void taylor_coeffs(double* c) {
+  // (-1)^k / (2k+1)!, by c_k = -c_{k-1} / ((2k)(2k+1)), each division rounded
+  c[0] = 1.0;
+  for (int k = 1; k < 12; ++k) c[k] = -c[k - 1] / (double)((2 * k) * (2 * k + 1));
+}
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MLG_OK : MLG_ERR_CUDA;
+}
+
+// Exclusive scan of n ints into TOut offsets [n + 1].
+template <typename TOut>
+void launch_scan(const int* in, int64_t n, TOut* out, long long* partial, ScanTail tail,
+                 cudaStream_t s) {
+  if (n <= kScanSingleMax) {
+    k_scan_single<TOut><<<1, 1024, 0, s>>>(in, n, out, tail);
+    return;
+  }
+  int tiles = (int)scan_tiles(n);
+  k_scan_reduce<<<tiles, kScanThreads, 0, s>>>(in, n, partial);
+  k_scan_top<<<1, 1024, 0, s>>>(partial, tiles);
+  k_scan_down<TOut><<<tiles, kScanThreads, 0, s>>>(in, n, partial, tiles, out, tail);
+}
+
+int check_csr(const mlg_csr* csr) {
+  if (csr == nullptr || csr->capacity < 0) return csr ? MLG_ERR_CAPACITY : MLG_ERR_INVALID_ARG;
+  if (!csr->row_ptr || !csr->n_edges || !csr->n_truncated || !csr->status)
+    return MLG_ERR_INVALID_ARG;
+  if (csr->capacity > 0 &&
+      (!csr->src || !csr->shift || !csr->vec || !csr->dist || !csr->sw))
+    return MLG_ERR_INVALID_ARG;
+  return MLG_OK;
+}
+
+int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+               const mlg_csr* csr, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (sys == nullptr || sys->coords == nullptr) return MLG_ERR_INVALID_ARG;
+  if (!(r_on >= 0.0) || !(r_on < rcut) || !std::isfinite(r_on)) return MLG_ERR_INVALID_ARG;
+  if (nnei_max < 1) return MLG_ERR_INVALID_ARG;
+  if (nnei_max > kMaxNnei) return MLG_ERR_UNSUPPORTED;
+  if (sys->types != nullptr && sys->n_types < 1) return MLG_ERR_INVALID_ARG;
+  int rc = check_csr(csr);
+  if (rc != MLG_OK) return rc;
+  BuildPlan plan;
+  rc = make_plan(sys->n_atoms, rcut, sys->box, sys->pbc, &plan);
+  if (rc != MLG_OK) return rc;
+  const int64_t n = sys->n_atoms;
+  BuildLayout L = build_layout(n, plan.ncell_cap);
+  if (ws == nullptr || ws_bytes < L.total || ((uintptr_t)ws % kAlign) != 0)
+    return MLG_ERR_WORKSPACE;
+
+  char* w = static_cast<char*>(ws);
+  BuildArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.n = n;
+  a.coords = sys->coords;
+  a.types = sys->types;
+  a.n_types = sys->n_types;
+  std::memcpy(a.box, sys->box, sizeof(a.box));
+  a.rcut = rcut;
+  a.r_on = r_on;
+  a.rc2 = rcut * rcut;
+  a.nnei_max = nnei_max;
+  taylor_coeffs(a.taylor);
+  a.capacity = csr->capacity;
+  a.row_ptr = csr->row_ptr;
+  a.src = csr->src;
+  a.shift = csr->shift;
+  a.vec = csr->vec;
+  a.dist = csr->dist;
+  a.sw = csr->sw;
+  a.n_edges = csr->n_edges;
+  a.n_truncated = csr->n_truncated;
+  a.status = csr->status;
+  a.grid = reinterpret_cast<CellGrid*>(w + L.grid);
+  a.bbox = reinterpret_cast<unsigned long long*>(w + L.bbox);
+  a.cell_count = reinterpret_cast<int*>(w + L.cell_count);
+  a.cell_start = reinterpret_cast<int*>(w + L.cell_start);
+  a.atom_cell = reinterpret_cast<int*>(w + L.atom_cell);
+  a.atom_rank = reinterpret_cast<int*>(w + L.atom_rank);
+  a.atom_w = reinterpret_cast<int*>(w + L.atom_w);
+  a.recs = reinterpret_cast<Rec*>(w + L.recs);
+  a.kept = reinterpret_cast<int*>(w + L.kept);
+  a.raw = reinterpret_cast<int*>(w + L.raw);
+  a.partial = reinterpret_cast<long long*>(w + L.partial);
+
+  const int tb = 256;
+  const int atom_blocks = (int)((n + tb - 1) / tb);
+  int init_blocks = (plan.ncell_cap + 1 + tb - 1) / tb;
+  if (init_blocks > 1024) init_blocks = 1024;
+  k_init<<<init_blocks, tb, 0, stream>>>(a, plan.ncell_cap);
+  if (plan.any_open) {
+    int bb = atom_blocks < 592 ? atom_blocks : 592;
+    k_bbox<<<bb, tb, 0, stream>>>(a, plan);
+  }
+  k_bin<<<atom_blocks, tb, 0, stream>>>(a, plan);
+  launch_scan<int>(a.cell_count, plan.ncell_cap, a.cell_start, a.partial,
+                   ScanTail{nullptr, nullptr, 0}, stream);
+  k_scatter<<<atom_blocks, tb, 0, stream>>>(a);
+  k_count<<<(int)((n + kCountWarps - 1) / kCountWarps), kCountWarps * 32, 0, stream>>>(a);
+  launch_scan<long long>(a.kept, n, reinterpret_cast<long long*>(a.row_ptr), a.partial,
+                         ScanTail{a.n_edges, a.status, a.capacity}, stream);
+  const size_t fill_smem = (size_t)kFillWarps * 2 * kFillMaxCand * sizeof(unsigned long long);
+  k_fill<<<(int)((n + kFillWarps - 1) / kFillWarps), kFillWarps * 32, fill_smem, stream>>>(a);
+  return launch_status();
+}
+
+
+int attention_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max, int32_t channels,
+                   int32_t heads, mlg_dtype dtype, const void* G_in, void* G_out,
+                   const void* Wq, const void* Wk, const void* Wv, cudaStream_t stream) {
+  if (csr == nullptr || csr->row_ptr == nullptr || csr->sw == nullptr || csr->status == nullptr)
+    return MLG_ERR_INVALID_ARG;
+  if (n_centres < 0 || nnei_max < 1 || channels < 1 || heads < 1 || channels % heads != 0)
+    return MLG_ERR_INVALID_ARG;
+  if (!G_in || !G_out || !Wq || !Wk || !Wv) return MLG_ERR_INVALID_ARG;
+  if (G_in == G_out) return MLG_ERR_INVALID_ARG;
+  if (dtype != MLG_F32 && dtype != MLG_F64) return MLG_ERR_INVALID_ARG;
+  const int D = channels / heads;
+  if (nnei_max > kMaxNnei || channels > 256 || D > 64) return MLG_ERR_UNSUPPORTED;
+  if (n_centres == 0) return MLG_OK;
+  AttnArgs a;
+  a.row_ptr = csr->row_ptr;
+  a.sw = csr->sw;
+  a.n_centres = n_centres;
+  a.capacity = csr->capacity;
+  a.nnei_max = nnei_max;
+  a.C = channels;
+  a.H = heads;
+  a.D = D;
+  a.G = G_in;
+  a.out = G_out;
+  a.Wq = Wq;
+  a.Wk = Wk;
+  a.Wv = Wv;
+  a.status = csr->status;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t want = (int64_t)sms * 4;
+  int grid = (int)(n_centres < want ? n_centres : want);
+  if (dtype == MLG_F64) {
+    size_t smem = attn_generic_smem<double>(nnei_max, D);
+    if (smem > 227 * 1024) return MLG_ERR_UNSUPPORTED;
+    cudaFuncSetAttribute(k_attn_generic<double>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    k_attn_generic<double><<<grid, kAttnWarps * 32, smem, stream>>>(a);
+  } else {
+    size_t smem = attn_generic_smem<float>(nnei_max, D);
+    if (smem > 227 * 1024) return MLG_ERR_UNSUPPORTED;
+    cudaFuncSetAttribute(k_attn_generic<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    k_attn_generic<float><<<grid, kAttnWarps * 32, smem, stream>>>(a);
+  }
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mlg_build_csr_workspace_bytes(int64_t n_atoms, double rcut, const double box[9],
+                                     const uint8_t pbc[3]) {
+  BuildPlan plan;
+  if (make_plan(n_atoms, rcut, box, pbc, &plan) != MLG_OK) return 0;
+  return build_layout(n_atoms, plan.ncell_cap).total;
+}
+
+int mlg_build_csr(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+                  const mlg_csr* csr, void* ws, size_t ws_bytes, mlg_stream_t stream) {
+  return build_impl(sys, rcut, r_on, nnei_max, csr, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+size_t mlg_attention_workspace_bytes(int64_t n_centres, int32_t nnei_max, int32_t channels,
+                                     int32_t heads, mlg_dtype dtype) {
+  (void)n_centres;
+  (void)nnei_max;
+  (void)channels;
+  (void)heads;
+  (void)dtype;
+  return 0;
+}
+
+int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                        int32_t channels, int32_t heads, mlg_dtype dtype, const void* G_in,
+                        void* G_out, const void* Wq, const void* Wk, const void* Wv, void* ws,
+                        size_t ws_bytes, mlg_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  return attention_impl(csr, n_centres, nnei_max, channels, heads, dtype, G_in, G_out, Wq, Wk,
+                        Wv, (cudaStream_t)stream);
+}
+
+size_t mlg_forward_workspace_bytes(int64_t n_atoms, double rcut, const double box[9],
+                                   const uint8_t pbc[3], int64_t capacity, int32_t channels,
+                                   int32_t n_layers, mlg_dtype dtype) {
+  size_t b = mlg_build_csr_workspace_bytes(n_atoms, rcut, box, pbc);
+  if (b == 0 || capacity < 0 || channels < 1 || n_layers < 1) return 0;
+  size_t el = dtype == MLG_F64 ? 8 : 4;
+  if (n_layers >= 2) b = align_up(b) + align_up((size_t)capacity * channels * el);
+  return b;
+}
+
+int mlg_forward(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+                int32_t channels, int32_t heads, int32_t n_layers, mlg_dtype dtype,
+                const void* const* W, const void* G0, void* G_out, const mlg_csr* csr,
+                void* ws, size_t ws_bytes, mlg_stream_t stream) {
+  if (sys == nullptr || W == nullptr || G0 == nullptr || G_out == nullptr || n_layers < 1)
+    return MLG_ERR_INVALID_ARG;
+  if (G0 == G_out) return MLG_ERR_INVALID_ARG;
+  if (csr == nullptr) return MLG_ERR_INVALID_ARG;
+  size_t need = mlg_forward_workspace_bytes(sys->n_atoms, rcut, sys->box, sys->pbc,
+                                            csr->capacity, channels, n_layers, dtype);
+  size_t build_need = mlg_build_csr_workspace_bytes(sys->n_atoms, rcut, sys->box, sys->pbc);
+  if (need == 0 || build_need == 0) {
+    // let the build report the precise argument error
+    int rc = build_impl(sys, rcut, r_on, nnei_max, csr, nullptr, 0, (cudaStream_t)stream);
+    return rc == MLG_OK ? MLG_ERR_INVALID_ARG : rc;
+  }
+  if (ws == nullptr || ws_bytes < need) return MLG_ERR_WORKSPACE;
+  for (int k = 0; k < 3 * n_layers; ++k)
+    if (W[k] == nullptr) return MLG_ERR_INVALID_ARG;
+  int rc = build_impl(sys, rcut, r_on, nnei_max, csr, ws, build_need, (cudaStream_t)stream);
+  if (rc != MLG_OK) return rc;
+  void* pong = static_cast<char*>(ws) + align_up(build_need);
+  const void* in = G0;
+  for (int l = 0; l < n_layers; ++l) {
+    // the last layer lands in G_out; earlier ones alternate so that a layer
+    // never reads the buffer it writes
+    void* dst = ((n_layers - 1 - l) % 2 == 0) ? G_out : pong;
+    rc = attention_impl(csr, sys->n_atoms, nnei_max, channels, heads, dtype, in, dst,
+                        W[3 * l], W[3 * l + 1], W[3 * l + 2], (cudaStream_t)stream);
+    if (rc != MLG_OK) return rc;
+    in = dst;
+  }
+  return MLG_OK;
+}
+
+int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
+                             const uint8_t pbc[3], int32_t n_layers) {
+  BuildPlan plan;
+  if (n_layers < 0 || make_plan(n_atoms, rcut, box, pbc, &plan) != MLG_OK) return 0;
+  auto scan_launches = [](int64_t n) { return n <= kScanSingleMax ? 1 : 3; };
+  // init, [bbox], bin, scan(cells), scatter, count, scan(row_ptr), fill, layers
+  return 5 + (plan.any_open ? 1 : 0) + scan_launches(plan.ncell_cap) + scan_launches(n_atoms) +
+         n_layers;
+}
+
+const char* mlg_status_string(int status) {
+  switch (status) {
+    case MLG_OK: return "MLG_OK";
+    case MLG_ERR_INVALID_ARG: return "MLG_ERR_INVALID_ARG: invalid argument";
+    case MLG_ERR_WORKSPACE: return "MLG_ERR_WORKSPACE: workspace missing, too small or misaligned";
+    case MLG_ERR_CAPACITY: return "MLG_ERR_CAPACITY: negative edge capacity";
+    case MLG_ERR_INPUT_DATA: return "MLG_ERR_INPUT_DATA: invalid input data";
+    case MLG_ERR_UNSUPPORTED: return "MLG_ERR_UNSUPPORTED: shape or cell not supported";
+    case MLG_ERR_CUDA: return "MLG_ERR_CUDA: CUDA launch error";
+    default: return "unknown mlg status";
+  }
+}
+
+int mlg_version(void) { return 100; }
+
+}  // extern "C"

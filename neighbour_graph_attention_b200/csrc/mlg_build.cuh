@@ -1,0 +1,819 @@
+// mlg_build.cuh -- stage 1: on-device destination CSR of all periodic
+// neighbour images within rcut (sm_100a).
+//
+// What is built: the per-pair edge index / edge vector tensors of
+// createEdgeTensors() (deepmd-kit issue "DPA4 .pt2 LAMMPS (C++ AOTI) inference
+// 3-6x slower than Python (ASE)", Root cause analysis, bottleneck 1), emitted
+// directly as the destination CSR (issue "NeighborGraph attention is 4-9x
+// slower than dense", Proposed fix: destination_order / destination_row_ptr),
+// with the per-centre cap sel (DPA4 issue, Reproduction: sel=181).  The
+// search is the O(N) GPU cell list the DPA4 issue's Python path uses
+// (Root cause analysis: "GPU O(N) cell list"), in the count -> prefix scan ->
+// fill shape of its build_nlist_gpu() remark, rebuilt for sm_100a:
+//
+//   k_init     zero the cell histogram, counters and status
+//   k_bbox     (open axes only) bounding box of the finite coordinates
+//   k_bin      cell of each atom (wrapped into the box along periodic axes)
+//              and its rank inside the cell from a warp-aggregated atomic
+//   scan       exclusive scan of the histogram -> cell_start
+//   k_scatter  atom records (coords, index, wrap image) in cell order
+//   k_count    warp per destination: candidates of the stencil cells, exact
+//              fp64 test r^2 < rcut^2, count -> kept = min(count, nnei_max)
+//   scan       exclusive scan of kept -> row_ptr, E
+//   k_fill     warp per destination: collect accepted candidates in shared
+//              memory, select the nnei_max nearest when the row overflows,
+//              sort into canonical (source, shift) order, write SoA edges
+//
+// Bit-exactness: the vector, distance and switch of an edge are computed with
+// explicitly rounded operations (__dadd_rn, __dmul_rn, __dsqrt_rn, ...) in the
+// one order that defines them, so no contraction into FMA can change a bit.
+#pragma once
+
+#include "mlg_common.cuh"
+
+namespace mlg {
+
+// ------------------------------------------------------------------ types
+
+// An atom in cell order: original coordinates, index and packed wrap image
+// (10 bits per axis, bias 512).
+struct __align__(16) Rec {
+  double x, y, z;
+  int j;
+  int w;
+};
+
+__host__ __device__ __forceinline__ int pack_w(int w0, int w1, int w2) {
+  return (w0 + 512) | ((w1 + 512) << 10) | ((w2 + 512) << 20);
+}
+__device__ __forceinline__ int unpack_w(int p, int k) { return ((p >> (10 * k)) & 1023) - 512; }
+
+// The cell grid as the device uses it.
+struct CellGrid {
+  double lo[3];     // grid origin along open axes (0 along periodic axes)
+  double inv_h[3];  // cells per Angstrom (0 when an open axis has one cell)
+  double L[3];      // box length along periodic axes
+  double invL[3];
+  int n[3];         // cells per axis
+  int D[3];         // stencil reach in cells
+  int periodic[3];
+  int ncell;
+};
+
+// What the host fixes before launch.
+struct BuildPlan {
+  int periodic[3];
+  double L[3], invL[3], inv_h[3];
+  int n_fixed[3];     // periodic axes: cells
+  int D_fixed[3];     // periodic axes: stencil reach
+  int n_open_max[3];  // open axes: most cells allowed
+  double rcd;         // minimum cell size along open axes (rcut plus margin)
+  int any_open;
+  int ncell_cap;
+};
+
+struct BuildArgs {
+  int64_t n;
+  const double* coords;
+  const int32_t* types;
+  int32_t n_types;
+  double box[9];
+  double rcut, r_on, rc2;
+  int nnei_max;
+  double taylor[12];  // Taylor coefficients (-1)^k / (2k+1)! of sin
+  int64_t capacity;
+  int64_t* row_ptr;
+  int32_t* src;
+  int32_t* shift;
+  double* vec;
+  double* dist;
+  double* sw;
+  int64_t* n_edges;
+  int64_t* n_truncated;
+  uint32_t* status;
+  // workspace
+  CellGrid* grid;
+  unsigned long long* bbox;  // [6] ordered bits: min x, y, z, max x, y, z
+  int* cell_count;           // [ncell_cap + 1]
+  int* cell_start;           // [ncell_cap + 1]
+  int* atom_cell;            // [n]  (-1: left out)
+  int* atom_rank;            // [n]
+  int* atom_w;               // [n]
+  Rec* recs;                 // [n]
+  int* kept;                 // [n]
+  int* raw;                  // [n]
+  long long* partial;        // scan partials
+};
+
+constexpr int kFillMaxCand = 512;  // shared-memory candidates per destination
+constexpr int kCountWarps = 8;
+constexpr int kFillWarps = 4;
+
+// ------------------------------------------------------------- geometry
+
+// r^2 of candidate (x_j + S L) - x_i.  Along a periodic (axis-aligned) axis the
+// shift contributes S_k L_k; the other rows of the box contribute signed
+// zeros only, which leave r^2 unchanged.
+__device__ __forceinline__ double cand_r2(const CellGrid& g, const double* xi, const Rec& rc,
+                                          const int* S) {
+  double xj[3] = {rc.x, rc.y, rc.z};
+  double v[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    double xs = g.periodic[k] ? __dadd_rn(xj[k], __dmul_rn((double)S[k], g.L[k])) : xj[k];
+    v[k] = __dsub_rn(xs, xi[k]);
+  }
+  return __dadd_rn(__dadd_rn(__dmul_rn(v[0], v[0]), __dmul_rn(v[1], v[1])),
+                   __dmul_rn(v[2], v[2]));
+}
+
+// The edge vector as defined for output:
+//   sh_c = (S_0 a1_c + S_1 a2_c) + S_2 a3_c,  v_c = (x_j,c + sh_c) - x_i,c
+__device__ __forceinline__ double edge_vec(const double* box, const double* xi,
+                                           const double* xj, const int* S, double* v) {
+  double s0 = (double)S[0], s1 = (double)S[1], s2 = (double)S[2];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    double sh = __dadd_rn(__dmul_rn(s0, box[c]), __dmul_rn(s1, box[3 + c]));
+    sh = __dadd_rn(sh, __dmul_rn(s2, box[6 + c]));
+    v[c] = __dsub_rn(__dadd_rn(xj[c], sh), xi[c]);
+  }
+  return __dadd_rn(__dadd_rn(__dmul_rn(v[0], v[0]), __dmul_rn(v[1], v[1])),
+                   __dmul_rn(v[2], v[2]));
+}
+
+// Cosine switch: 1 below r_on, 0 from rcut, else 0.5 (1 + cos(pi u)) with
+// cos(pi u) = -sin(pi (u - 1/2)) and sin by its Taylor series through x^23
+// (Horner in x^2).  Every operation explicitly rounded.
+__device__ __forceinline__ double switch_fn(double r, double rcut, double r_on,
+                                            const double* c) {
+  if (r < r_on) return 1.0;
+  if (r >= rcut) return 0.0;
+  const double pi = 3.141592653589793;
+  double u = __ddiv_rn(__dsub_rn(r, r_on), __dsub_rn(rcut, r_on));
+  double x = __dmul_rn(pi, __dsub_rn(u, 0.5));
+  double x2 = __dmul_rn(x, x);
+  double p = c[11];
+#pragma unroll
+  for (int k = 10; k >= 0; --k) p = __dadd_rn(c[k], __dmul_rn(x2, p));
+  double sinx = __dmul_rn(x, p);
+  return __dmul_rn(0.5, __dadd_rn(1.0, -sinx));
+}
+
+// ------------------------------------------------------------ grid setup
+
+__device__ __forceinline__ CellGrid derive_grid(const BuildPlan& p,
+                                                const unsigned long long* bbox) {
+  CellGrid g;
+  int nc = 1;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    g.periodic[k] = p.periodic[k];
+    if (p.periodic[k]) {
+      g.lo[k] = 0.0;
+      g.L[k] = p.L[k];
+      g.invL[k] = p.invL[k];
+      g.inv_h[k] = p.inv_h[k];
+      g.n[k] = p.n_fixed[k];
+      g.D[k] = p.D_fixed[k];
+    } else {
+      g.L[k] = 0.0;
+      g.invL[k] = 0.0;
+      double lo = from_ordered_bits(bbox[k]);
+      double hi = from_ordered_bits(bbox[3 + k]);
+      int n = 1;
+      double ext = hi - lo;
+      if (lo <= hi && ext > 0.0) {
+        double q = floor(ext / p.rcd);
+        n = q < 1.0 ? 1 : (q > (double)p.n_open_max[k] ? p.n_open_max[k] : (int)q);
+        while (n > 1 && ext / (double)n < p.rcd) --n;
+      }
+      g.lo[k] = lo <= hi ? lo : 0.0;
+      g.n[k] = n;
+      g.inv_h[k] = n > 1 ? (double)n / ext : 0.0;
+      g.D[k] = n > 1 ? 1 : 0;
+    }
+    nc *= g.n[k];
+  }
+  g.ncell = nc;
+  return g;
+}
+
+// ----------------------------------------------------------------- kernels
+
+__global__ void k_init(BuildArgs a, int ncell_cap) {
+  int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t m = t; m <= ncell_cap; m += stride) a.cell_count[m] = 0;
+  if (t < 3) {
+    a.bbox[t] = ~0ull;
+    a.bbox[3 + t] = 0ull;
+  }
+  if (t == 0) {
+    *a.n_truncated = 0;
+    *a.status = 0u;
+  }
+}
+
+// Bounding box of the finite coordinates along open axes.
+__global__ void k_bbox(BuildArgs a, BuildPlan p) {
+  double lo[3] = {INFINITY, INFINITY, INFINITY}, hi[3] = {-INFINITY, -INFINITY, -INFINITY};
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < a.n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    double x0 = a.coords[3 * i], x1 = a.coords[3 * i + 1], x2 = a.coords[3 * i + 2];
+    if (!(isfinite(x0) && isfinite(x1) && isfinite(x2))) continue;
+    double x[3] = {x0, x1, x2};
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      lo[k] = fmin(lo[k], x[k]);
+      hi[k] = fmax(hi[k], x[k]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    if (p.periodic[k]) continue;
+    double l = lo[k], h = hi[k];
+    for (int o = 16; o > 0; o >>= 1) {
+      l = fmin(l, __shfl_xor_sync(kFull, l, o));
+      h = fmax(h, __shfl_xor_sync(kFull, h, o));
+    }
+    if (lane_id() == 0 && l <= h) {
+      atomicMin(&a.bbox[k], ordered_bits(l));
+      atomicMax(&a.bbox[3 + k], ordered_bits(h));
+    }
+  }
+}
+
+__global__ void k_bin(BuildArgs a, BuildPlan p) {
+  CellGrid g = derive_grid(p, a.bbox);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.grid = g;
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  int cell = -1;
+  uint32_t st = 0;
+  if (i < a.n) {
+    double x[3] = {a.coords[3 * i], a.coords[3 * i + 1], a.coords[3 * i + 2]};
+    int wpack = 0;
+    if (!(isfinite(x[0]) && isfinite(x[1]) && isfinite(x[2]))) {
+      st |= MLG_STATUS_NONFINITE_COORD;
+    } else {
+      int c[3], w[3];
+      bool ok = true;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        double y;
+        if (g.periodic[k]) {
+          double fq = floor(x[k] * g.invL[k]);
+          if (!(fabs(fq) <= 511.0)) {
+            ok = false;
+            fq = 0.0;
+          }
+          w[k] = (int)fq;
+          y = x[k] - fq * g.L[k];
+        } else {
+          w[k] = 0;
+          y = x[k] - g.lo[k];
+        }
+        double cf = floor(y * g.inv_h[k]);
+        int ck = cf < 0.0 ? 0 : (cf >= (double)g.n[k] ? g.n[k] - 1 : (int)cf);
+        c[k] = ck;
+      }
+      if (!ok) {
+        st |= MLG_STATUS_IMAGE_RANGE;
+      } else {
+        cell = (c[0] * g.n[1] + c[1]) * g.n[2] + c[2];
+        wpack = pack_w(w[0], w[1], w[2]);
+      }
+    }
+    if (a.types != nullptr) {
+      int t = a.types[i];
+      if (t < 0 || t >= a.n_types) st |= MLG_STATUS_TYPE_RANGE;
+    }
+    a.atom_cell[i] = cell;
+    a.atom_w[i] = wpack;
+  }
+  // warp-aggregated atomics on the cell histogram
+  unsigned act = __ballot_sync(kFull, cell >= 0);
+  if (cell >= 0) {
+    unsigned peers = __match_any_sync(act, cell);
+    int leader = __ffs(peers) - 1;
+    int base = 0;
+    if ((int)lane_id() == leader) base = atomicAdd(&a.cell_count[cell], __popc(peers));
+    base = __shfl_sync(peers, base, leader);
+    a.atom_rank[i] = base + __popc(peers & lanemask_lt());
+  }
+  st = __reduce_or_sync(kFull, st);
+  if (lane_id() == 0 && st) atomicOr(a.status, st);
+}
+
+__global__ void k_scatter(BuildArgs a) {
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= a.n) return;
+  int cell = a.atom_cell[i];
+  if (cell < 0) return;
+  Rec r;
+  r.x = a.coords[3 * i];
+  r.y = a.coords[3 * i + 1];
+  r.z = a.coords[3 * i + 2];
+  r.j = (int)i;
+  r.w = a.atom_w[i];
+  a.recs[a.cell_start[cell] + a.atom_rank[i]] = r;
+}
+
+// ----------------------------------------------------- candidate traversal
+
+struct WarpScratch {
+  int pre[33];
+  int start[32];
+  int tpack[32];
+};
+
+struct Centre {
+  double x[3];
+  int w[3];
+  int c[3];
+  int i;
+};
+
+__device__ __forceinline__ Centre load_centre(const BuildArgs& a, const CellGrid& g, int i,
+                                              int cell) {
+  Centre cc;
+  cc.i = i;
+  cc.x[0] = a.coords[3 * (int64_t)i];
+  cc.x[1] = a.coords[3 * (int64_t)i + 1];
+  cc.x[2] = a.coords[3 * (int64_t)i + 2];
+  int wp = a.atom_w[i];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) cc.w[k] = unpack_w(wp, k);
+  cc.c[2] = cell % g.n[2];
+  cc.c[1] = (cell / g.n[2]) % g.n[1];
+  cc.c[0] = cell / (g.n[2] * g.n[1]);
+  return cc;
+}
+
+// Visit every atom of the stencil cells of `cc` with its extended-cell image
+// T.  The stencil cells are taken 32 at a time; their atom ranges are
+// flattened with a warp prefix sum so that all lanes stay busy.  `f(valid,
+// rec, tpack)` is called by all 32 lanes together (it may use warp votes).
+template <class F>
+__device__ __forceinline__ void for_each_candidate(const CellGrid& g, const int* cell_start,
+                                                   const Centre& cc, WarpScratch& ws, F&& f) {
+  const int lane = lane_id();
+  const int w0 = 2 * g.D[0] + 1, w1 = 2 * g.D[1] + 1, w2 = 2 * g.D[2] + 1;
+  const int s3 = w0 * w1 * w2;
+  for (int chunk = 0; chunk < s3; chunk += 32) {
+    int s = chunk + lane;
+    int len = 0, start = 0, tp = 0;
+    if (s < s3) {
+      int d[3];
+      d[2] = s % w2 - g.D[2];
+      int t = s / w2;
+      d[1] = t % w1 - g.D[1];
+      d[0] = t / w1 - g.D[0];
+      int m[3], T[3];
+      bool ok = true;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        int e = cc.c[k] + d[k];
+        if (g.periodic[k]) {
+          T[k] = floordiv(e, g.n[k]);
+          m[k] = e - T[k] * g.n[k];
+        } else {
+          ok = ok && e >= 0 && e < g.n[k];
+          m[k] = e;
+          T[k] = 0;
+        }
+      }
+      if (ok) {
+        int cell = (m[0] * g.n[1] + m[1]) * g.n[2] + m[2];
+        start = cell_start[cell];
+        len = cell_start[cell + 1] - start;
+        tp = ((T[0] + 64) << 14) | ((T[1] + 64) << 7) | (T[2] + 64);
+      }
+    }
+    int incl = warp_incl_scan(len);
+    int total = __shfl_sync(kFull, incl, 31);
+    ws.pre[lane] = incl - len;
+    ws.start[lane] = start;
+    ws.tpack[lane] = tp;
+    if (lane == 31) ws.pre[32] = total;
+    __syncwarp();
+    int o = 0;
+    for (int base = 0; base < total; base += 32) {
+      int t = base + lane;
+      bool valid = t < total;
+      int r = 0, tpo = 0;
+      if (valid) {
+        while (ws.pre[o + 1] <= t) ++o;
+        r = ws.start[o] + (t - ws.pre[o]);
+        tpo = ws.tpack[o];
+      }
+      f(valid, r, tpo);
+    }
+    __syncwarp();
+  }
+}
+
+// Exact test of one candidate; returns true if (j, S) is an edge of cc.
+__device__ __forceinline__ bool test_candidate(const CellGrid& g, const Centre& cc,
+                                               const Rec& rc, int tpack, double rc2,
+                                               double* r2_out) {
+  int S[3];
+  S[0] = ((tpack >> 14) & 127) - 64 + cc.w[0] - unpack_w(rc.w, 0);
+  S[1] = ((tpack >> 7) & 127) - 64 + cc.w[1] - unpack_w(rc.w, 1);
+  S[2] = (tpack & 127) - 64 + cc.w[2] - unpack_w(rc.w, 2);
+  double r2 = cand_r2(g, cc.x, rc, S);
+  *r2_out = r2;
+  bool self = rc.j == cc.i && S[0] == 0 && S[1] == 0 && S[2] == 0;
+  return r2 < rc2 && !self;
+}
+
+__global__ void __launch_bounds__(kCountWarps * 32) k_count(BuildArgs a) {
+  __shared__ CellGrid sg;
+  __shared__ WarpScratch sw[kCountWarps];
+  __shared__ int s_trunc;
+  if (threadIdx.x == 0) {
+    sg = *a.grid;
+    s_trunc = 0;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  const int64_t i = (int64_t)blockIdx.x * kCountWarps + warp;
+  if (i < a.n) {
+    int cell = a.atom_cell[i];
+    int cnt = 0;
+    if (cell >= 0) {
+      Centre cc = load_centre(a, sg, (int)i, cell);
+      for_each_candidate(sg, a.cell_start, cc, sw[warp], [&](bool valid, int r, int tp) {
+        if (valid) {
+          double r2;
+          cnt += test_candidate(sg, cc, a.recs[r], tp, a.rc2, &r2) ? 1 : 0;
+        }
+      });
+      cnt = warp_sum(cnt);
+    }
+    if (lane_id() == 0) {
+      a.raw[i] = cnt;
+      a.kept[i] = cnt < a.nnei_max ? cnt : a.nnei_max;
+      if (cnt > a.nnei_max) atomicAdd(&s_trunc, 1);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && s_trunc) atomicAdd((unsigned long long*)a.n_truncated,
+                                             (unsigned long long)s_trunc);
+}
+
+// ------------------------------------------------------------ warp sorts
+
+__device__ __forceinline__ int next_pow2(int n) {
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
+// Ascending bitonic sort of k[0..n) (n <= kFillMaxCand) by one warp.
+__device__ void warp_sort_keys(unsigned long long* k, int n) {
+  const int lane = lane_id();
+  const int P = next_pow2(n);
+  for (int t = n + lane; t < P; t += 32) k[t] = ~0ull;
+  __syncwarp();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = lane; t < (P >> 1); t += 32) {
+        int lo = ((t & ~(stride - 1)) << 1) | (t & (stride - 1));
+        int hi = lo + stride;
+        bool up = (lo & size) == 0;
+        unsigned long long x = k[lo], y = k[hi];
+        if ((x > y) == up) {
+          k[lo] = y;
+          k[hi] = x;
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// Ascending bitonic sort of (d[t], k[t]) pairs by (d, k).
+__device__ void warp_sort_pairs(unsigned long long* d, unsigned long long* k, int n) {
+  const int lane = lane_id();
+  const int P = next_pow2(n);
+  for (int t = n + lane; t < P; t += 32) {
+    d[t] = ~0ull;
+    k[t] = ~0ull;
+  }
+  __syncwarp();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = lane; t < (P >> 1); t += 32) {
+        int lo = ((t & ~(stride - 1)) << 1) | (t & (stride - 1));
+        int hi = lo + stride;
+        bool up = (lo & size) == 0;
+        unsigned long long dx = d[lo], dy = d[hi], kx = k[lo], ky = k[hi];
+        bool gt = dx > dy || (dx == dy && kx > ky);
+        if (gt == up) {
+          d[lo] = dy;
+          d[hi] = dx;
+          k[lo] = ky;
+          k[hi] = kx;
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// ------------------------------------------------------------------- fill
+
+__device__ __forceinline__ unsigned long long edge_key(int j, int tpack) {
+  return ((unsigned long long)(unsigned)j << 21) | (unsigned long long)tpack;
+}
+
+// Threshold search for rows with more than kFillMaxCand candidates: find the
+// nnei_max-th smallest r^2 by bisection over its bit pattern (monotone for
+// non-negative doubles), then break ties at that distance by key.
+__device__ int fill_overflow_select(const BuildArgs& a, const CellGrid& g, const Centre& cc,
+                                    WarpScratch& ws, unsigned long long* keys, int n,
+                                    uint32_t* st) {
+  const unsigned lane = lane_id();
+  unsigned long long lo = 0ull, hi = (unsigned long long)__double_as_longlong(a.rc2);
+  while (lo < hi) {
+    unsigned long long mid = lo + ((hi - lo) >> 1);
+    int cnt = 0;
+    for_each_candidate(g, a.cell_start, cc, ws, [&](bool valid, int r, int tp) {
+      if (valid) {
+        double r2;
+        if (test_candidate(g, cc, a.recs[r], tp, a.rc2, &r2) &&
+            (unsigned long long)__double_as_longlong(r2) <= mid)
+          ++cnt;
+      }
+    });
+    cnt = warp_sum(cnt);
+    if (cnt >= n) hi = mid; else lo = mid + 1;
+  }
+  const unsigned long long thr = lo;
+  // below the threshold -> keys[0..nlt); at the threshold -> keys[256..)
+  int nlt = 0, neq = 0;
+  const int tie_base = 256, tie_cap = kFillMaxCand - 256;
+  for_each_candidate(g, a.cell_start, cc, ws, [&](bool valid, int r, int tp) {
+    bool lt = false, eq = false;
+    unsigned long long key = 0;
+    if (valid) {
+      const Rec rc = a.recs[r];
+      double r2;
+      if (test_candidate(g, cc, rc, tp, a.rc2, &r2)) {
+        unsigned long long b = (unsigned long long)__double_as_longlong(r2);
+        lt = b < thr;
+        eq = b == thr;
+        key = edge_key(rc.j, tp);
+      }
+    }
+    unsigned mlt = __ballot_sync(kFull, lt), meq = __ballot_sync(kFull, eq);
+    if (lt) {
+      int q = nlt + __popc(mlt & lanemask_lt());
+      if (q < tie_base) keys[q] = key;
+    }
+    if (eq) {
+      int q = neq + __popc(meq & lanemask_lt());
+      if (q < tie_cap) keys[tie_base + q] = key;
+    }
+    nlt += __popc(mlt);
+    neq += __popc(meq);
+  });
+  __syncwarp();
+  if (neq > tie_cap) {
+    if (lane == 0) *st |= MLG_STATUS_TIES;
+    neq = tie_cap;
+  }
+  warp_sort_keys(keys + tie_base, neq);
+  // nlt < n <= 256 and nlt + neq >= n hold when this pass saw what the count
+  // pass saw; clamp anyway so that only collected keys are ever used
+  const int nlt_c = nlt < n ? nlt : n;
+  int take = n - nlt_c;
+  if (take > neq) take = neq;
+  for (int t = lane; t < take; t += 32) keys[nlt_c + t] = keys[tie_base + t];
+  __syncwarp();
+  return nlt_c + take;
+}
+
+__global__ void __launch_bounds__(kFillWarps * 32) k_fill(BuildArgs a) {
+  __shared__ CellGrid sg;
+  __shared__ WarpScratch sws[kFillWarps];
+  extern __shared__ unsigned long long s_fill[];  // [warps][2][kFillMaxCand]
+  if (threadIdx.x == 0) sg = *a.grid;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  const unsigned lane = lane_id();
+  const int64_t i = (int64_t)blockIdx.x * kFillWarps + warp;
+  if (i >= a.n) return;
+  const int cell = a.atom_cell[i];
+  const int n = a.kept[i];
+  if (cell < 0 || n == 0) return;
+  const int raw = a.raw[i];
+  const int64_t p0 = a.row_ptr[i];
+  unsigned long long* keys = s_fill + (size_t)warp * 2 * kFillMaxCand;
+  unsigned long long* d2 = keys + kFillMaxCand;
+  Centre cc = load_centre(a, sg, (int)i, cell);
+  uint32_t st = 0;
+  int nv = 0;  // keys collected for this row; equals n unless the passes disagree
+  if (raw <= kFillMaxCand) {
+    int pos = 0;
+    for_each_candidate(sg, a.cell_start, cc, sws[warp], [&](bool valid, int r, int tp) {
+      bool acc = false;
+      unsigned long long key = 0, b = 0;
+      if (valid) {
+        const Rec rc = a.recs[r];
+        double r2;
+        acc = test_candidate(sg, cc, rc, tp, a.rc2, &r2);
+        key = edge_key(rc.j, tp);
+        b = (unsigned long long)__double_as_longlong(r2);
+      }
+      unsigned m = __ballot_sync(kFull, acc);
+      if (acc) {
+        int q = pos + __popc(m & lanemask_lt());
+        if (q < kFillMaxCand) {
+          keys[q] = key;
+          d2[q] = b;
+        }
+      }
+      pos += __popc(m);
+    });
+    __syncwarp();
+    const int m = pos < kFillMaxCand ? pos : kFillMaxCand;
+    if (m > n) warp_sort_pairs(d2, keys, m);
+    nv = n < m ? n : m;
+    warp_sort_keys(keys, nv);
+  } else {
+    nv = fill_overflow_select(a, sg, cc, sws[warp], keys, n, &st);
+    warp_sort_keys(keys, nv);
+  }
+  if (nv != n) st |= MLG_STATUS_INTERNAL;
+  // canonical order now in keys[0..nv): write the SoA edge arrays
+  for (int e = lane; e < nv; e += 32) {
+    unsigned long long key = keys[e];
+    int j = (int)(key >> 21);
+    if (j < 0 || (int64_t)j >= a.n) continue;
+    int tp = (int)(key & 0x1fffffull);
+    int wj = a.atom_w[j];
+    int S[3];
+    S[0] = ((tp >> 14) & 127) - 64 + cc.w[0] - unpack_w(wj, 0);
+    S[1] = ((tp >> 7) & 127) - 64 + cc.w[1] - unpack_w(wj, 1);
+    S[2] = (tp & 127) - 64 + cc.w[2] - unpack_w(wj, 2);
+    double xj[3] = {a.coords[3 * (int64_t)j], a.coords[3 * (int64_t)j + 1],
+                    a.coords[3 * (int64_t)j + 2]};
+    double v[3];
+    double r2 = edge_vec(a.box, cc.x, xj, S, v);
+    double r = __dsqrt_rn(r2);
+    int64_t p = p0 + e;
+    if (p < a.capacity) {
+      a.src[p] = j;
+      a.shift[3 * p] = S[0];
+      a.shift[3 * p + 1] = S[1];
+      a.shift[3 * p + 2] = S[2];
+      a.vec[3 * p] = v[0];
+      a.vec[3 * p + 1] = v[1];
+      a.vec[3 * p + 2] = v[2];
+      a.dist[p] = r;
+      a.sw[p] = switch_fn(r, a.rcut, a.r_on, a.taylor);
+    }
+  }
+  if (lane == 0 && st) atomicOr(a.status, st);
+}
+
+// ------------------------------------------------------------------ scans
+//
+// Exclusive scan of int counts into int or int64 offsets: reduce-then-scan
+// over tiles of 2048 (no inter-block waiting).  Small inputs use one block.
+
+constexpr int kScanThreads = 256;
+constexpr int kScanItems = 8;
+constexpr int kScanTile = kScanThreads * kScanItems;
+constexpr int kScanSingleMax = 1 << 16;
+
+// exclusive block scan (blockDim.x threads, multiple of 32, <= 1024)
+template <typename T>
+__device__ __forceinline__ T block_excl_scan(T v, T* total) {
+  __shared__ T s_w[33];
+  const int lane = lane_id(), warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  T incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    T u = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) s_w[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    T x = lane < nw ? s_w[lane] : T(0);
+    T xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      T u = __shfl_up_sync(kFull, xi, o);
+      if (lane >= o) xi += u;
+    }
+    if (lane < nw) s_w[lane] = xi - x;
+    if (lane == 31) s_w[32] = xi;
+  }
+  __syncthreads();
+  *total = s_w[32];
+  T r = s_w[warp] + incl - v;
+  __syncthreads();
+  return r;
+}
+
+// Finishing of a row_ptr scan: E, capacity check.
+struct ScanTail {
+  int64_t* n_edges;
+  uint32_t* status;
+  int64_t capacity;
+};
+
+template <typename TOut>
+__global__ void __launch_bounds__(1024) k_scan_single(const int* in, int64_t n, TOut* out,
+                                                      ScanTail tail) {
+  const int64_t per = (n + blockDim.x - 1) / blockDim.x;
+  const int64_t b = threadIdx.x * per;
+  const int64_t e = b + per < n ? b + per : n;
+  long long s = 0;
+  for (int64_t t = b; t < e; ++t) s += in[t];
+  long long tot;
+  long long off = block_excl_scan<long long>(s, &tot);
+  for (int64_t t = b; t < e; ++t) {
+    out[t] = (TOut)off;
+    off += in[t];
+  }
+  if (threadIdx.x == 0) {
+    out[n] = (TOut)tot;
+    if (tail.n_edges) {
+      *tail.n_edges = tot;
+      if (tot > tail.capacity) atomicOr(tail.status, (uint32_t)MLG_STATUS_CAPACITY);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_scan_reduce(const int* in, int64_t n,
+                                                              long long* partial) {
+  const int64_t base = (int64_t)blockIdx.x * kScanTile;
+  long long s = 0;
+#pragma unroll
+  for (int q = 0; q < kScanItems; ++q) {
+    int64_t t = base + q * kScanThreads + threadIdx.x;
+    if (t < n) s += in[t];
+  }
+  s = warp_sum(s);
+  __shared__ long long s_w[kScanThreads / 32];
+  if (lane_id() == 0) s_w[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long tot = 0;
+    for (int w = 0; w < kScanThreads / 32; ++w) tot += s_w[w];
+    partial[blockIdx.x] = tot;
+  }
+}
+
+// one block: exclusive scan of the tile sums in place; partial[ntiles] = total
+__global__ void __launch_bounds__(1024) k_scan_top(long long* partial, int ntiles) {
+  long long carry = 0;
+  for (int base = 0; base < ntiles; base += blockDim.x) {
+    int t = base + threadIdx.x;
+    long long v = t < ntiles ? partial[t] : 0;
+    long long tot;
+    long long ex = block_excl_scan<long long>(v, &tot);
+    if (t < ntiles) partial[t] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) partial[ntiles] = carry;
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(kScanThreads) k_scan_down(const int* in, int64_t n,
+                                                            const long long* partial,
+                                                            int ntiles, TOut* out,
+                                                            ScanTail tail) {
+  const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * kScanItems;
+  int v[kScanItems];
+  long long s = 0;
+#pragma unroll
+  for (int q = 0; q < kScanItems; ++q) {
+    int64_t t = base + q;
+    v[q] = t < n ? in[t] : 0;
+    s += v[q];
+  }
+  long long tot;
+  long long off = block_excl_scan<long long>(s, &tot) + partial[blockIdx.x];
+#pragma unroll
+  for (int q = 0; q < kScanItems; ++q) {
+    int64_t t = base + q;
+    if (t < n) out[t] = (TOut)off;
+    off += v[q];
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    long long total = partial[ntiles];
+    out[n] = (TOut)total;
+    if (tail.n_edges) {
+      *tail.n_edges = total;
+      if (total > tail.capacity) atomicOr(tail.status, (uint32_t)MLG_STATUS_CAPACITY);
+    }
+  }
+}
+
+}  // namespace mlg

@@ -1,0 +1,173 @@
+"""The C ABI without a GPU: exported symbols, struct layout, host-side checks.
+
+Every call below fails its argument or workspace checks before any CUDA call,
+so it runs on a machine without a GPU.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mlg.h")
+
+
+@pytest.fixture(scope="module")
+def mlg():
+    from neighbour_graph_attention_b200 import build
+
+    build.build()
+    from neighbour_graph_attention_b200 import mlg as m
+
+    return m
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(mlg_[a-z_0-9]+)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(mlg):
+    names = _declared_functions()
+    assert {"mlg_build_csr", "mlg_block_attention", "mlg_forward"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", mlg.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)$", out, re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(mlg.lib(), n)
+
+
+def test_struct_layout_matches_c(mlg, tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "mlg.h"\n'
+        "int main(void){\n"
+        ' printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(mlg_system), offsetof(mlg_system, coords),'
+        " offsetof(mlg_system, n_types), offsetof(mlg_system, box), offsetof(mlg_system, pbc),"
+        " sizeof(mlg_csr));\n"
+        ' printf("%zu %zu\\n", offsetof(mlg_csr, sw), offsetof(mlg_csr, status));\n'
+        " return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-o", str(exe)])
+    lines = subprocess.check_output([str(exe)], text=True).split("\n")
+    a = list(map(int, lines[0].split()))
+    b = list(map(int, lines[1].split()))
+    S, C = mlg.mlg_system, mlg.mlg_csr
+    assert a == [ctypes.sizeof(S), S.coords.offset, S.n_types.offset, S.box.offset,
+                 S.pbc.offset, ctypes.sizeof(C)]
+    assert b == [C.sw.offset, C.status.offset]
+
+
+def test_status_strings(mlg):
+    for code in range(7):
+        assert mlg.mlg_status_string(code).startswith("MLG_")
+    assert "unknown" in mlg.mlg_status_string(99)
+    assert mlg.mlg_version() >= 100
+
+
+FAKE = 0x1000  # a non-null device address that no host check dereferences
+
+
+def _fake_csr(mlg, capacity=100):
+    c = mlg.mlg_csr()
+    c.capacity = capacity
+    for name in ("row_ptr", "src", "shift", "vec", "dist", "sw", "n_edges", "n_truncated",
+                 "status"):
+        setattr(c, name, FAKE)
+    return c
+
+
+def _sys(mlg, n=64, box=None, pbc=(1, 1, 1)):
+    s = mlg.mlg_system()
+    s.n_atoms = n
+    s.coords = FAKE
+    s.types = None
+    s.n_types = 0
+    s.box[:] = list(np.ravel(np.diag([10.0] * 3) if box is None else box))
+    s.pbc[:] = list(pbc)
+    return s
+
+
+def _build(mlg, sys_, rcut=4.0, r_on=3.5, nnei=40, csr=None, ws=None, ws_bytes=0):
+    csr = csr or _fake_csr(mlg)
+    return mlg.lib().mlg_build_csr(ctypes.byref(sys_), rcut, r_on, nnei, ctypes.byref(csr),
+                                   ws, ws_bytes, None)
+
+
+def test_host_argument_checks(mlg):
+    assert _build(mlg, _sys(mlg, n=0)) == mlg.MLG_ERR_INVALID_ARG
+    assert _build(mlg, _sys(mlg), rcut=-1.0) == mlg.MLG_ERR_INVALID_ARG
+    assert _build(mlg, _sys(mlg), r_on=4.0) == mlg.MLG_ERR_INVALID_ARG      # r_on >= rcut
+    assert _build(mlg, _sys(mlg), nnei=0) == mlg.MLG_ERR_INVALID_ARG
+    assert _build(mlg, _sys(mlg), nnei=257) == mlg.MLG_ERR_UNSUPPORTED
+    bad_box = np.diag([10.0] * 3); bad_box[0, 1] = 1.0
+    assert _build(mlg, _sys(mlg, box=bad_box)) == mlg.MLG_ERR_UNSUPPORTED   # sheared cell
+    nan_box = np.diag([10.0, np.nan, 10.0])
+    assert _build(mlg, _sys(mlg, box=nan_box)) == mlg.MLG_ERR_INVALID_ARG
+    zero_len = np.diag([10.0, 0.0, 10.0])
+    assert _build(mlg, _sys(mlg, box=zero_len)) == mlg.MLG_ERR_INVALID_ARG
+    # an open axis ignores its box row: a zero row is fine there
+    assert _build(mlg, _sys(mlg, box=zero_len, pbc=(1, 0, 1))) == mlg.MLG_ERR_WORKSPACE
+    assert _build(mlg, _sys(mlg), csr=_fake_csr(mlg, capacity=-1)) == mlg.MLG_ERR_CAPACITY
+    c = _fake_csr(mlg); c.row_ptr = None
+    assert _build(mlg, _sys(mlg), csr=c) == mlg.MLG_ERR_INVALID_ARG
+    # a box far smaller than rcut: stencil beyond the supported reach
+    assert _build(mlg, _sys(mlg, box=np.diag([0.05] * 3)), rcut=4.0) == mlg.MLG_ERR_UNSUPPORTED
+
+
+def test_workspace_checks(mlg):
+    s = _sys(mlg)
+    need = mlg.mlg_build_csr_workspace_bytes(64, 4.0, np.diag([10.0] * 3), [1, 1, 1])
+    assert need > 0
+    assert _build(mlg, s, ws=None, ws_bytes=need) == mlg.MLG_ERR_WORKSPACE
+    assert _build(mlg, s, ws=FAKE * 16, ws_bytes=need - 1) == mlg.MLG_ERR_WORKSPACE
+    assert _build(mlg, s, ws=FAKE * 16 + 8, ws_bytes=need) == mlg.MLG_ERR_WORKSPACE  # misaligned
+    assert mlg.mlg_build_csr_workspace_bytes(0, 4.0, np.diag([10.0] * 3), [1, 1, 1]) == 0
+    # open axes: the cell budget bounds the workspace whatever the coordinates
+    w_open = mlg.mlg_build_csr_workspace_bytes(5964, 5.0, np.zeros((3, 3)), [0, 0, 0])
+    assert 0 < w_open < 5964 * 400
+    # forward adds one ping-pong feature buffer for >= 2 layers
+    f1 = mlg.mlg_forward_workspace_bytes(64, 4.0, np.diag([10.0] * 3), [1, 1, 1], 1000, 32, 1, 1)
+    f2 = mlg.mlg_forward_workspace_bytes(64, 4.0, np.diag([10.0] * 3), [1, 1, 1], 1000, 32, 2, 1)
+    assert f1 == need and f2 >= need + 1000 * 32 * 8
+
+
+def test_attention_argument_checks(mlg):
+    lib = mlg.lib()
+    c = _fake_csr(mlg)
+    call = lambda **k: lib.mlg_block_attention(
+        ctypes.byref(c), k.get("n", 10), k.get("nnei", 40), k.get("ch", 32), k.get("heads", 4),
+        k.get("dtype", 1), k.get("gin", FAKE), k.get("gout", FAKE * 2), FAKE, FAKE, FAKE,
+        None, 0, None)
+    assert call(heads=3) == mlg.MLG_ERR_INVALID_ARG          # channels % heads != 0
+    assert call(gin=None) == mlg.MLG_ERR_INVALID_ARG
+    assert call(gout=FAKE) == mlg.MLG_ERR_INVALID_ARG        # aliasing in/out
+    assert call(dtype=7) == mlg.MLG_ERR_INVALID_ARG
+    assert call(ch=512, heads=8) == mlg.MLG_ERR_UNSUPPORTED
+    assert call(ch=256, heads=2) == mlg.MLG_ERR_UNSUPPORTED  # head size 128 > 64
+    assert call(nnei=300) == mlg.MLG_ERR_UNSUPPORTED
+    assert call(n=-1) == mlg.MLG_ERR_INVALID_ARG
+
+
+def test_product_path_fails_loudly_without_library(tmp_path):
+    # the binding has no fallback: a missing library is an import error
+    code = (
+        "import importlib.util, sys\n"
+        f"spec = importlib.util.spec_from_file_location('m', r'{ROOT}/neighbour_graph_attention_b200/mlg.py')\n"
+        "m = importlib.util.module_from_spec(spec)\n"
+        "import os\n"
+        "os.path.exists = lambda p: False\n"
+        "try:\n"
+        "    spec.loader.exec_module(m)\n"
+        "except ImportError as e:\n"
+        "    print('IMPORT_ERROR', 'no CPU fallback' in str(e))\n")
+    out = subprocess.run(["python", "-c", code], capture_output=True, text=True)
+    assert "IMPORT_ERROR True" in out.stdout, out.stdout + out.stderr

@@ -1,0 +1,151 @@
+"""GPU parity of block-dense attention and of the whole forward.
+
+Block-dense per-centre attention over the destination CSR (NeighborGraph
+issue, Proposed fix). Tolerances: FP64 max-abs 1e-10; FP32 max-abs
+2e-5 * max|oracle| per layer (the oracle computes in fp64 from the fp32
+inputs and rounds each layer's output to fp32).
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+from neighbour_graph_attention_b200 import configs as C
+
+import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+
+@functools.lru_cache(maxsize=None)
+def graph(key, seed):
+    w = C.workload(key)
+    s = C.system(key, seed)
+    gpu, csr_t = U.gpu_build(s["coords"], s["box"], s["pbc"], w.rcut, w.r_on, w.nnei_max)
+    return gpu, csr_t
+
+
+@pytest.mark.parametrize("key,seed", [(1, 0), (1, 1), (2, 0), (2, 2), (3, 0), (4, 0), (4, 1)])
+def test_one_layer_matches_oracle(key, seed):
+    import oracle
+
+    w = C.workload(key)
+    gpu, csr_t = graph(key, seed)
+    e = gpu["n_edges"]
+    W = C.weights(key, seed)
+    G = C.features(key, seed, e)
+    out = U.gpu_attention(csr_t, w.n_atoms, w, G, W[0][0], W[0][1], W[0][2])
+    sw = gpu["sw"] if w.dtype == "f64" else gpu["sw"].astype(np.float32).astype(np.float64)
+    ref = oracle.attention(gpu["row_ptr"], sw, G, W[0][0], W[0][1], W[0][2], w.heads)
+    ok, err = U.attn_tolerance_ok(w, out, ref)
+    assert ok, err
+
+
+def test_largest_system_sampled_centres():
+    import oracle
+
+    key = 5
+    w = C.workload(key)
+    gpu, csr_t = graph(key, 0)
+    e = gpu["n_edges"]
+    W = C.weights(key, 0)
+    G = C.features(key, 0, e)
+    out = U.gpu_attention(csr_t, w.n_atoms, w, G, W[0][0], W[0][1], W[0][2])
+    rp = gpu["row_ptr"]
+    sw = gpu["sw"].astype(np.float32).astype(np.float64)
+    rng = np.random.default_rng(5)
+    sample = np.sort(np.concatenate([[0, w.n_atoms - 1], rng.choice(w.n_atoms, 254, False)]))
+    rows = np.concatenate([np.arange(rp[i], rp[i + 1]) for i in sample])
+    sub_rp = np.concatenate([[0], np.cumsum(rp[sample + 1] - rp[sample])])
+    ref = oracle.attention(sub_rp, sw[rows], G[rows], W[0][0], W[0][1], W[0][2], w.heads)
+    ok, err = U.attn_tolerance_ok(w, out[rows], ref)
+    assert ok, err
+
+
+@pytest.mark.parametrize("key", [3, 5])
+def test_sum_to_one_through_gpu(key):
+    # G column 0 = 1 and Wv = ones in row 0 only: every value vector is all
+    # ones, so every output is exactly a softmax-weighted mean of ones = 1
+    w = C.workload(key)
+    gpu, csr_t = graph(key, 0)
+    e = gpu["n_edges"]
+    G = C.features(key, 1, e)
+    G[:, 0] = 1.0
+    W = C.weights(key, 1)
+    Wv = np.zeros_like(W[0][2])
+    Wv[0, :] = 1.0
+    out = U.gpu_attention(csr_t, w.n_atoms, w, G, W[0][0], W[0][1], Wv)
+    assert np.max(np.abs(out.astype(np.float64) - 1.0)) <= 4e-6
+
+
+@pytest.mark.parametrize("key", [2, 4])
+def test_forward_matches_oracle(key):
+    import oracle
+
+    m = U.mlg()
+    w = C.workload(key)
+    s = C.system(key, 0)
+    gpu, _ = graph(key, 0)
+    e = gpu["n_edges"]
+    W = C.weights(key, 0)
+    G = C.features(key, 0, e)
+    dt = U.torch_dtype(w)
+    x = torch.as_tensor(s["coords"], device="cuda")
+    csr = m.Csr.empty(w.n_atoms, e)
+    g0 = torch.as_tensor(G, dtype=dt, device="cuda")
+    gout = torch.zeros_like(g0)
+    Wt = [torch.as_tensor(W[l][k], dtype=dt, device="cuda") for l in range(w.n_layers)
+          for k in range(3)]
+    need = m.mlg_forward_workspace_bytes(w.n_atoms, w.rcut, s["box"], s["pbc"], e, w.channels,
+                                         w.n_layers, U.mlg_dtype(w))
+    ws = m.workspace(need)
+    sysd = m.make_system(x, s["box"], s["pbc"])
+    m.mlg_forward(sysd, w.rcut, w.r_on, w.nnei_max, w.channels, w.heads, w.n_layers,
+                  U.mlg_dtype(w), Wt, g0, gout, csr, ws)
+    torch.cuda.synchronize()
+    assert int(csr.status.item()) == 0
+    U.assert_csr_equal(U.csr_to_numpy(csr), gpu)
+    outs = oracle.forward(gpu["row_ptr"], gpu["sw"], G, W, w.heads, w.dtype)
+    ok, err = U.attn_tolerance_ok(w, gout.cpu().numpy(), outs[-1])
+    assert ok, err
+
+
+def test_forward_graph_capture_and_side_stream():
+    m = U.mlg()
+    key = 2
+    w = C.workload(key)
+    s = C.system(key, 1)
+    gpu, _ = graph(key, 1)
+    e = gpu["n_edges"]
+    W = C.weights(key, 1)
+    G = C.features(key, 1, e)
+    x = torch.as_tensor(s["coords"], device="cuda")
+    csr = m.Csr.empty(w.n_atoms, e)
+    g0 = torch.as_tensor(G, device="cuda")
+    ref_out = torch.zeros_like(g0)
+    Wt = [torch.as_tensor(W[l][k], device="cuda") for l in range(w.n_layers) for k in range(3)]
+    need = m.mlg_forward_workspace_bytes(w.n_atoms, w.rcut, s["box"], s["pbc"], e, w.channels,
+                                         w.n_layers, m.MLG_F64)
+    ws = m.workspace(need)
+    sysd = m.make_system(x, s["box"], s["pbc"])
+    args = (sysd, w.rcut, w.r_on, w.nnei_max, w.channels, w.heads, w.n_layers, m.MLG_F64, Wt, g0)
+    m.mlg_forward(*args, ref_out, csr, ws)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    out2 = torch.zeros_like(g0)
+    with torch.cuda.stream(side):
+        m.mlg_forward(*args, out2, csr, ws, stream=side)
+    side.synchronize()
+    assert torch.equal(out2, ref_out)
+    out3 = torch.zeros_like(g0)
+    graph_ = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph_, stream=cap):
+            m.mlg_forward(*args, out3, csr, ws, stream=cap)
+    for _ in range(2):
+        out3.zero_()
+        graph_.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out3, ref_out)

@@ -181,6 +181,33 @@ int mlg_forward(const mlg_system* sys, double rcut, double r_on, int32_t nnei_ma
                 const void* const* W, const void* G0, void* G_out, const mlg_csr* csr,
                 void* ws, size_t ws_bytes, mlg_stream_t stream);
 
+/* Size of the library's built-in scratch array for mlg_build_csr_noalloc. */
+#define MLG_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* mlg_build_csr without a workspace argument and without any allocation.
+ * No counterpart in the pages: this is a deployment aid.  Some callers cannot
+ * allocate device memory: a force callback inside an MD engine that passes
+ * raw device pointers but owns every allocation itself (and cannot afford the
+ * device-wide synchronisation an allocation may trigger in its time step), or
+ * a host plugin without an allocator of its own.  For them the scratch lives
+ * in a fixed array of MLG_NOALLOC_SCRATCH_BYTES (8 MiB) in the library's own
+ * device memory; every GPU that loads the library holds that array until the
+ * process exits.
+ *   - Same arguments, results and device status as mlg_build_csr; the CSR
+ *     output buffers are still the caller's.
+ *   - Returns MLG_ERR_WORKSPACE, launching nothing, when the system needs more
+ *     scratch than the array holds (mlg_build_csr_workspace_bytes() >
+ *     MLG_NOALLOC_SCRATCH_BYTES; about 150,000 atoms for a periodic box).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture begins.
+ *   - Every call shares the one array, and the array keeps the contents of
+ *     the previous call; the build clears everything that must start at zero
+ *     itself.  Two calls whose work overlaps on the GPU (different streams
+ *     without ordering between them) race on the array: order them. */
+int mlg_build_csr_noalloc(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+                          const mlg_csr* csr, mlg_stream_t stream);
+
 /* Number of kernel launches that one mlg_forward call with these arguments
  * issues on its stream (for accounting in benchmarks); 0 for invalid
  * arguments. */

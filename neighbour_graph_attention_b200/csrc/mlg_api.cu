@@ -389,3 +389,67 @@ const char* mlg_status_string(int status) {
 int mlg_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free CSR build.
+//
+// For callers that cannot allocate device memory themselves: a force
+// callback inside an MD engine that hands the library raw device pointers
+// but owns every allocation (and must not stall its time step on the
+// device-wide synchronisation an allocation can cause), or a host plugin
+// that has no allocator of its own.  This entry point takes its scratch
+// from a fixed array in the library's own device memory instead of a
+// caller workspace.  It runs exactly the same kernels as mlg_build_csr.
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = MLG_NOALLOC_SCRATCH_BYTES;
+
+// One array per GPU that loads this library, held until the process exits.
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices];  // device address of the array, per device
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MLG_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MLG_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return MLG_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLG_OK;
+}
+
+}  // namespace
+
+extern "C" int mlg_build_csr_noalloc(const mlg_system* sys, double rcut, double r_on,
+                                     int32_t nnei_max, const mlg_csr* csr,
+                                     mlg_stream_t stream) {
+  if (sys == nullptr) return MLG_ERR_INVALID_ARG;
+  const size_t need = mlg_build_csr_workspace_bytes(sys->n_atoms, rcut, sys->box, sys->pbc);
+  if (need == 0)  // invalid arguments: let the regular checks name the error
+    return build_impl(sys, rcut, r_on, nnei_max, csr, nullptr, 0, (cudaStream_t)stream);
+  if (need > kNoAllocScratchBytes) return MLG_ERR_WORKSPACE;  // system too large for the array
+  void* scratch = nullptr;
+  int rc = noalloc_scratch(&scratch);
+  if (rc != MLG_OK) return rc;
+  return build_impl(sys, rcut, r_on, nnei_max, csr, scratch, kNoAllocScratchBytes,
+                    (cudaStream_t)stream);
+}

@@ -76,6 +76,9 @@ _lib.mlg_forward.restype = ctypes.c_int
 _lib.mlg_forward.argtypes = [ctypes.POINTER(mlg_system), _c_dbl, _c_dbl, _c_i32, _c_i32, _c_i32,
                              _c_i32, ctypes.c_int, ctypes.POINTER(_p), _p, _p,
                              ctypes.POINTER(mlg_csr), _p, _c_sz, _p]
+_lib.mlg_build_csr_noalloc.restype = ctypes.c_int
+_lib.mlg_build_csr_noalloc.argtypes = [ctypes.POINTER(mlg_system), _c_dbl, _c_dbl, _c_i32,
+                                       ctypes.POINTER(mlg_csr), _p]
 _lib.mlg_forward_launch_count.restype = ctypes.c_int
 _lib.mlg_forward_launch_count.argtypes = [_c_i64, _c_dbl, _p, _p, _c_i32]
 _lib.mlg_status_string.restype = ctypes.c_char_p
@@ -214,6 +217,20 @@ def mlg_build_csr(system: mlg_system, rcut: float, r_on: float, nnei_max: int, c
     code = _lib.mlg_build_csr(ctypes.byref(system), float(rcut), float(r_on), int(nnei_max),
                               ctypes.byref(c), _ptr(ws), nbytes, _stream_handle(stream))
     return _check(code, "mlg_build_csr", check)
+
+
+MLG_NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def mlg_build_csr_noalloc(system: mlg_system, rcut: float, r_on: float, nnei_max: int,
+                          csr: Csr, stream=None, check: bool = True) -> int:
+    """The CSR build with the library's built-in scratch array: no workspace, no
+    allocation (for callers that cannot allocate; see include/mlg.h). Calls
+    that overlap on the GPU share that array and race, so order them."""
+    c = csr.struct()
+    code = _lib.mlg_build_csr_noalloc(ctypes.byref(system), float(rcut), float(r_on),
+                                      int(nnei_max), ctypes.byref(c), _stream_handle(stream))
+    return _check(code, "mlg_build_csr_noalloc", check)
 
 
 def mlg_block_attention(csr: Csr, n_centres: int, nnei_max: int, channels: int, heads: int,

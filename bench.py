@@ -50,6 +50,9 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(C.WORKLOADS))
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--cells", type=int, default=None,
+                   help="profiling only: conventional cells per axis of a lattice workload "
+                        "(same shapes, fewer atoms)")
     p.add_argument("--impl", choices=["mlg", "reference"], default="mlg")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -261,6 +264,19 @@ def run_reference(args):
     return 0
 
 
+def select_workload(args):
+    """The workload, optionally with fewer lattice cells (profiling runs only)."""
+    import dataclasses
+
+    w = C.workload(args.workload)
+    if args.cells is not None and w.periodic and args.cells != w.cells:
+        per_cell = w.n_atoms // w.cells ** 3
+        w = dataclasses.replace(w, cells=args.cells, n_atoms=per_cell * args.cells ** 3,
+                                name=f"{w.name}-cells{args.cells}")
+        C.WORKLOADS[w.key] = w
+    return w, C.system(w.key, args.seed)
+
+
 def workload_config(w, args, extra=None):
     cfg = {"workload": f"{w.name}: {w.n_atoms} atoms, {w.lattice}, rcut {w.rcut} A, "
                        f"nnei_max {w.nnei_max}, c={w.channels}, heads={w.heads}, "
@@ -300,8 +316,7 @@ def main(argv=None):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = C.workload(args.workload)
-    s = C.system(args.workload, args.seed)
+    w, s = select_workload(args)
     W = C.weights(args.workload, args.seed)
     dt = torch.float64 if w.dtype == "f64" else torch.float32
     elem = 8 if w.dtype == "f64" else 4
@@ -331,16 +346,38 @@ def main(argv=None):
                                                    w.channels, w.n_layers, mdt), device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
-    def step(out=Gout):
-        m.mlg_forward(sysd, w.rcut, w.r_on, w.nnei_max, w.channels, w.heads, w.n_layers, mdt,
-                      Wt, G0, out, csr, ws, stream=stream)
+    stack_ws = m.workspace(m.mlg_attention_stack_workspace_bytes(E, w.channels, w.n_layers, mdt),
+                           device=dev)
+
+    # one step = the two calls mlg_forward makes: the CSR build, then the
+    # fused attention stack; an event between them times the attention
+    # launch inside the timed region
+    def build_call():
+        m.mlg_build_csr(sysd, w.rcut, w.r_on, w.nnei_max, csr, ws, stream=stream)
+
+    def stack_call():
+        m.mlg_attention_stack(csr, w.n_atoms, w.nnei_max, w.channels, w.heads, w.n_layers, mdt,
+                              Wt, G0, Gout, stack_ws, stream=stream)
+
+    def timed_steps(k):
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(k)]
+        with torch.cuda.stream(stream):
+            for e0, e1, e2 in evs:
+                flush.fill_(1.0)          # L2 flush, outside the timed events
+                e0.record(stream)
+                build_call()
+                e1.record(stream)
+                stack_call()
+                e2.record(stream)
+        stream.synchronize()
+        return [(e0.elapsed_time(e1), e1.elapsed_time(e2)) for e0, e1, e2 in evs]
 
     def timed_loop(fn, k):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(k)]
         with torch.cuda.stream(stream):
             for a, b in evs:
-                flush.fill_(1.0)          # L2 flush, outside the timed events
+                flush.fill_(1.0)
                 a.record(stream)
                 fn()
                 b.record(stream)
@@ -348,24 +385,26 @@ def main(argv=None):
         return [a.elapsed_time(b) for a, b in evs]
 
     # warm-up, then a load pre-roll that lets the clock sampler see the GPU busy
-    timed_loop(step, args.warmup)
+    timed_steps(args.warmup)
     sampler = ClockSampler(dev.index)
     sampler.start()
     t_pre = time.perf_counter()
     while time.perf_counter() - t_pre < 1.0:
-        timed_loop(step, 20)
+        timed_steps(20)
 
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t0 = time.perf_counter()
-    step_ms = timed_loop(step, args.steps)
+    parts = timed_steps(args.steps)
     torch.cuda.synchronize(dev)
     t1 = time.perf_counter()
     if world > 1:
         dist.barrier()
     sampler.stop()
-    total_ms = float(sum(step_ms))
+    build_ms_steps = [p[0] for p in parts]
+    attn_ms_steps = [p[1] for p in parts]
+    total_ms = float(sum(build_ms_steps) + sum(attn_ms_steps))
     if world > 1:
         tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -377,25 +416,18 @@ def main(argv=None):
     if status != 0:
         raise RuntimeError(f"device status {status:#x} after the timed steps")
 
-    # live per-kernel timing for the roofline: one attention layer (one kernel
-    # launch) and the whole build (several kernels), same stream, L2 flushed
-    gin, gout = G0, torch.empty_like(G0)
-    attn_ms = timed_loop(lambda: m.mlg_block_attention(
-        csr, w.n_atoms, w.nnei_max, w.channels, w.heads, mdt, gin, gout, Wt[0], Wt[1], Wt[2],
-        stream=stream), args.steps)
-    build_ms = timed_loop(lambda: m.mlg_build_csr(sysd, w.rcut, w.r_on, w.nnei_max, csr, ws,
-                                                  stream=stream), args.steps)
-    attn_avg = statistics.mean(attn_ms)
-    build_avg = statistics.mean(build_ms)
-    flops = attention_flops(row_ptr, w.channels)
+    attn_avg = statistics.mean(attn_ms_steps)
+    build_avg = statistics.mean(build_ms_steps)
+    flops = attention_flops(row_ptr, w.channels) * w.n_layers
     peak_fp = FP64_PEAK_TFLOPS if w.dtype == "f64" else FP32_PEAK_TFLOPS
     achieved_tf = flops / (attn_avg * 1e-3) / 1e12
     hbm_peak, hbm_src = load_peaks()
     bbytes = build_bytes(w.n_atoms, E)
-    abytes = attention_bytes(w.n_atoms, E, w.channels, elem)
-    attn_kernel = "k_attn_generic<double>" if w.dtype == "f64" else "k_attn_generic<float>"
+    abytes = attention_bytes(w.n_atoms, E, w.channels, elem) + \
+        (w.n_layers - 1) * 3.0 * w.channels * w.channels * elem
     roofline = {"bound": "alu", "achieved": achieved_tf, "peak": peak_fp, "unit": "TFLOP/s",
-                "frac": achieved_tf / peak_fp, "traffic": None, "kernel": attn_kernel,
+                "frac": achieved_tf / peak_fp, "traffic": None,
+                "kernel": "attention stack (k_attn_tile: all %d layer(s) fused)" % w.n_layers,
                 "algorithmic_flops_per_launch": flops,
                 "peak_basis": ("derived: 148 SMs x %d %s FMA/clk x 2 x 1.965 GHz" %
                                (64 if w.dtype == "f64" else 128, w.dtype.upper())),
@@ -405,10 +437,10 @@ def main(argv=None):
                       "frac": build_gbs / hbm_peak, "peak_source": hbm_src,
                       "algorithmic_bytes": bbytes, "ms": build_avg,
                       "note": "whole build stage (several kernels)"}
-    layers_share = w.n_layers * attn_avg / max(ms_per_step, 1e-9)
+    layers_share = attn_avg / max(ms_per_step, 1e-9)
 
     # end to end through the C ABI with host buffers: pinned H2D of the
-    # step's inputs (coordinates, edge features), forward, D2H of the result
+    # step's inputs (coordinates, edge features), mlg_forward, D2H of the result
     x_h = torch.as_tensor(s["coords"]).pin_memory()
     g_h = G0.cpu().pin_memory()
     out_h = torch.empty(Gout.shape, dtype=dt).pin_memory()
@@ -434,7 +466,8 @@ def main(argv=None):
     h2d = x_h.numel() * x_h.element_size() + g_h.numel() * g_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
 
-    launches = m.mlg_forward_launch_count(w.n_atoms, w.rcut, s["box"], s["pbc"], w.n_layers)
+    launches = m.mlg_forward_launch_count(w.n_atoms, w.rcut, s["box"], s["pbc"], w.nnei_max,
+                                          w.channels, w.heads, w.n_layers, mdt)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -449,7 +482,7 @@ def main(argv=None):
             "config": workload_config(w, args, {"n_edges": E}),
             "roofline": roofline,
             "roofline_build": roofline_build,
-            "stages": {"build_ms": build_avg, "attention_ms_per_layer": attn_avg,
+            "stages": {"build_ms": build_avg, "attention_ms": attn_avg,
                        "n_layers": w.n_layers, "attention_share_of_step": layers_share},
             "e2e": {"value": e2e_value, "unit": "atoms/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_total / args.steps},

@@ -79,8 +79,10 @@ typedef enum {
                                         box along a periodic axis; it was left out */
     MLG_STATUS_TIES = 16u,           /* truncation met more than 256 candidates at one
                                         distance; the kept set is not canonical */
-    MLG_STATUS_INTERNAL = 32u        /* the count and fill passes disagreed on a row (never
+    MLG_STATUS_INTERNAL = 32u,       /* the count and fill passes disagreed on a row (never
                                         expected); that row is incomplete */
+    MLG_STATUS_TIMEOUT = 64u         /* a bounded wait for an on-chip copy ran out (never
+                                        expected); the attention output is incomplete */
 } mlg_status_bits;
 
 /* Arithmetic type of attention features and weights. */
@@ -163,6 +165,24 @@ int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                         void* G_out, const void* Wq, const void* Wk, const void* Wv, void* ws,
                         size_t ws_bytes, mlg_stream_t stream);
 
+/* Bytes of device workspace that mlg_attention_stack needs: one [capacity][channels] buffer
+ * for n_layers >= 2 (used only by centres the fused kernels do not cover), else 0. */
+size_t mlg_attention_stack_workspace_bytes(int64_t capacity, int32_t channels, int32_t n_layers,
+                                           mlg_dtype dtype);
+
+/* n_layers stacked block-dense attention layers, G^{l+1} = attention(G^l) with the layer-l
+ * weights; G^0 = G_in, the last layer's output in G_out.  Same per-layer definition as
+ * mlg_block_attention.  A centre's output rows depend only on its own input rows, so the
+ * layers of a centre run back to back on chip (one fused launch for the supported shapes)
+ * and intermediate layers never reach global memory.
+ *   W   HOST array of 3 * n_layers device pointers: Wq, Wk, Wv of layer 0, then layer 1, ...
+ *   ws  device workspace of ws_bytes >= mlg_attention_stack_workspace_bytes() (may be NULL
+ *       when that is 0) */
+int mlg_attention_stack(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                        int32_t channels, int32_t heads, int32_t n_layers, mlg_dtype dtype,
+                        const void* const* W, const void* G_in, void* G_out, void* ws,
+                        size_t ws_bytes, mlg_stream_t stream);
+
 /* Bytes of device workspace for mlg_forward: the build's workspace plus, for
  * n_layers >= 2, one [capacity][channels] buffer for the layer ping-pong. */
 size_t mlg_forward_workspace_bytes(int64_t n_atoms, double rcut, const double box[9],
@@ -212,7 +232,8 @@ int mlg_build_csr_noalloc(const mlg_system* sys, double rcut, double r_on, int32
  * issues on its stream (for accounting in benchmarks); 0 for invalid
  * arguments. */
 int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
-                             const uint8_t pbc[3], int32_t n_layers);
+                             const uint8_t pbc[3], int32_t nnei_max, int32_t channels,
+                             int32_t heads, int32_t n_layers, mlg_dtype dtype);
 
 /* A static string naming a host status code. */
 const char* mlg_status_string(int status);

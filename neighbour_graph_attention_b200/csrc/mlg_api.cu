@@ -10,6 +10,8 @@
 #include "mlg_common.cuh"
 #include "mlg_build.cuh"
 #include "mlg_attn.cuh"
+#include "mlg_attn_tile.cuh"
+#include "mlg_attn_hg.cuh"
 
 using namespace mlg;
 
@@ -232,54 +234,215 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
 }
 
 
-int attention_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max, int32_t channels,
-                   int32_t heads, mlg_dtype dtype, const void* G_in, void* G_out,
-                   const void* Wq, const void* Wk, const void* Wv, cudaStream_t stream) {
-  if (csr == nullptr || csr->row_ptr == nullptr || csr->sw == nullptr || csr->status == nullptr)
-    return MLG_ERR_INVALID_ARG;
-  if (n_centres < 0 || nnei_max < 1 || channels < 1 || heads < 1 || channels % heads != 0)
-    return MLG_ERR_INVALID_ARG;
-  if (!G_in || !G_out || !Wq || !Wk || !Wv) return MLG_ERR_INVALID_ARG;
-  if (G_in == G_out) return MLG_ERR_INVALID_ARG;
-  if (dtype != MLG_F32 && dtype != MLG_F64) return MLG_ERR_INVALID_ARG;
-  const int D = channels / heads;
-  if (nnei_max > kMaxNnei || channels > 256 || D > 64) return MLG_ERR_UNSUPPORTED;
-  if (n_centres == 0) return MLG_OK;
+int sm_count() {
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+// One layer of the generic kernel over the centres with more than min_n edges.
+int launch_generic(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max, int32_t C, int32_t H,
+                   mlg_dtype dtype, const void* G_in, void* G_out, const void* Wq,
+                   const void* Wk, const void* Wv, int min_n, cudaStream_t stream) {
   AttnArgs a;
   a.row_ptr = csr->row_ptr;
   a.sw = csr->sw;
   a.n_centres = n_centres;
   a.capacity = csr->capacity;
   a.nnei_max = nnei_max;
-  a.C = channels;
-  a.H = heads;
-  a.D = D;
+  a.C = C;
+  a.H = H;
+  a.D = C / H;
   a.G = G_in;
   a.out = G_out;
   a.Wq = Wq;
   a.Wk = Wk;
   a.Wv = Wv;
   a.status = csr->status;
-  int sms = 148;
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t want = (int64_t)sms * 4;
+  a.min_n = min_n;
+  int64_t want = (int64_t)sm_count() * 4;
   int grid = (int)(n_centres < want ? n_centres : want);
   if (dtype == MLG_F64) {
-    size_t smem = attn_generic_smem<double>(nnei_max, D);
+    size_t smem = attn_generic_smem<double>(nnei_max, a.D);
     if (smem > 227 * 1024) return MLG_ERR_UNSUPPORTED;
     cudaFuncSetAttribute(k_attn_generic<double>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     k_attn_generic<double><<<grid, kAttnWarps * 32, smem, stream>>>(a);
   } else {
-    size_t smem = attn_generic_smem<float>(nnei_max, D);
+    size_t smem = attn_generic_smem<float>(nnei_max, a.D);
     if (smem > 227 * 1024) return MLG_ERR_UNSUPPORTED;
     cudaFuncSetAttribute(k_attn_generic<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     k_attn_generic<float><<<grid, kAttnWarps * 32, smem, stream>>>(a);
   }
   return launch_status();
+}
+
+// Tile kernel instantiations: (dtype, channels, head size) -> tile rows R.
+template <typename T, int C, int D, int R, int NT, int TM, int TN, int XB>
+int launch_tile(TileArgs& ta, cudaStream_t stream) {
+  using Cfg = TileCfg<T, C, D, R, NT, TM, TN, XB>;
+  auto kern = k_attn_tile<T, C, D, R, NT, TM, TN, XB>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) !=
+      cudaSuccess)
+    return launch_status() == MLG_OK ? MLG_ERR_CUDA : MLG_ERR_CUDA;
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, Cfg::SMEM);
+  if (occ < 1) occ = 1;
+  int64_t want = (int64_t)sm_count() * occ;
+  int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
+  if (grid < 1) grid = 1;
+  kern<<<grid, NT, Cfg::SMEM, stream>>>(ta);
+  return launch_status();
+}
+
+// Returns the tile rows R of the fused kernel for this shape (0: none).
+int tile_rows(mlg_dtype dtype, int C, int D) {
+  if (dtype == MLG_F64 && C == 32 && D == 8) return 40;
+  if (dtype == MLG_F32 && C == 32 && D == 8) return 128;
+  if (dtype == MLG_F32 && C == 64 && D == 16) return 128;
+  return 0;
+}
+
+int launch_tile_shape(mlg_dtype dtype, int C, int D, TileArgs& ta, cudaStream_t s) {
+  if (dtype == MLG_F64 && C == 32 && D == 8)
+    return launch_tile<double, 32, 8, 40, 256, 5, 3, 1>(ta, s);
+  if (dtype == MLG_F32 && C == 32 && D == 8)
+    return launch_tile<float, 32, 8, 128, 256, 8, 6, 2>(ta, s);
+  if (dtype == MLG_F32 && C == 64 && D == 16)
+    return launch_tile<float, 64, 16, 128, 512, 8, 6, 2>(ta, s);
+  return MLG_ERR_UNSUPPORTED;
+}
+
+// Head-group kernel instantiations for wide features: (dtype, channels, head size) -> R.
+template <typename T, int C, int D, int HG, int R, int NT, int TM, int TN, int KC>
+int launch_hg(HgArgs& ha, cudaStream_t stream) {
+  using Cfg = HgCfg<T, C, D, HG, R, NT, TM, TN, KC>;
+  auto kern = k_attn_hg<T, C, D, HG, R, NT, TM, TN, KC>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) !=
+      cudaSuccess)
+    return MLG_ERR_CUDA;
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, Cfg::SMEM);
+  if (occ < 1) occ = 1;
+  int64_t gx = ((int64_t)sm_count() * occ + Cfg::NG - 1) / Cfg::NG;
+  if (gx > ha.n_centres) gx = ha.n_centres;
+  if (gx < 1) gx = 1;
+  kern<<<dim3((unsigned)gx, Cfg::NG), NT, Cfg::SMEM, stream>>>(ha);
+  return launch_status();
+}
+
+int hg_rows(mlg_dtype dtype, int C, int D) {
+  if (dtype == MLG_F64 && C == 128 && D == 32) return 128;
+  if (dtype == MLG_F32 && C == 128 && D == 16) return 96;
+  return 0;
+}
+
+int launch_hg_shape(mlg_dtype dtype, int C, int D, HgArgs& ha, cudaStream_t s) {
+  if (dtype == MLG_F64 && C == 128 && D == 32)
+    return launch_hg<double, 128, 32, 1, 128, 256, 8, 6, 16>(ha, s);
+  if (dtype == MLG_F32 && C == 128 && D == 16)
+    return launch_hg<float, 128, 16, 2, 96, 256, 6, 6, 16>(ha, s);
+  return MLG_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int check_attention_args(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                         int32_t channels, int32_t heads, mlg_dtype dtype, const void* G_in,
+                         void* G_out) {
+  if (csr == nullptr || csr->row_ptr == nullptr || csr->sw == nullptr || csr->status == nullptr)
+    return MLG_ERR_INVALID_ARG;
+  if (n_centres < 0 || nnei_max < 1 || channels < 1 || heads < 1 || channels % heads != 0)
+    return MLG_ERR_INVALID_ARG;
+  if (!G_in || !G_out) return MLG_ERR_INVALID_ARG;
+  if (G_in == G_out) return MLG_ERR_INVALID_ARG;
+  if (dtype != MLG_F32 && dtype != MLG_F64) return MLG_ERR_INVALID_ARG;
+  const int D = channels / heads;
+  if (nnei_max > kMaxNnei || channels > 256 || D > 64) return MLG_ERR_UNSUPPORTED;
+  return MLG_OK;
+}
+
+// n_layers attention layers G^{l+1} = attention(G^l), G^0 = G_in, result in
+// G_out.  `pong` is a [capacity][channels] buffer, needed only for
+// n_layers >= 2 on the generic path.
+int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                         int32_t channels, int32_t heads, mlg_dtype dtype, int32_t n_layers,
+                         const void* const* W, const void* G_in, void* G_out, void* pong,
+                         cudaStream_t stream) {
+  int rc = check_attention_args(csr, n_centres, nnei_max, channels, heads, dtype, G_in, G_out);
+  if (rc != MLG_OK) return rc;
+  if (n_layers < 1 || W == nullptr) return MLG_ERR_INVALID_ARG;
+  for (int k = 0; k < 3 * n_layers; ++k)
+    if (W[k] == nullptr) return MLG_ERR_INVALID_ARG;
+  if (n_layers >= 2 && pong == nullptr) return MLG_ERR_WORKSPACE;
+  if (n_centres == 0) return MLG_OK;
+  const int D = channels / heads;
+  int R = tile_rows(dtype, channels, D);
+  bool tile_ok = R > 0 && n_layers <= kMaxFusedLayers && aligned16(G_in) && aligned16(G_out);
+  for (int k = 0; tile_ok && k < 3 * n_layers; ++k) tile_ok = aligned16(W[k]);
+  int min_n = 0;  // generic path: centres with more than min_n edges
+  if (tile_ok) {
+    TileArgs ta;
+    std::memset(&ta, 0, sizeof(ta));
+    ta.row_ptr = csr->row_ptr;
+    ta.sw = csr->sw;
+    ta.n_centres = n_centres;
+    ta.capacity = csr->capacity;
+    ta.n_layers = n_layers;
+    ta.G = G_in;
+    ta.out = G_out;
+    for (int k = 0; k < 3 * n_layers; ++k) ta.W[k] = W[k];
+    ta.status = csr->status;
+    rc = launch_tile_shape(dtype, channels, D, ta, stream);
+    if (rc != MLG_OK) return rc;
+    if (nnei_max <= R) return MLG_OK;  // no centre can exceed the tile
+    min_n = R;
+  }
+  // head-group kernel (one launch per layer) when there is one for the shape
+  int Rg = tile_ok ? 0 : hg_rows(dtype, channels, D);
+  bool hg_ok = Rg > 0 && aligned16(G_in) && aligned16(G_out) && (n_layers < 2 || aligned16(pong));
+  for (int k = 0; hg_ok && k < 3 * n_layers; ++k) hg_ok = aligned16(W[k]);
+  if (hg_ok) min_n = nnei_max <= Rg ? -1 : Rg;  // -1: no generic launch needed
+  // per layer: head-group kernel and/or the generic kernel for the centres left
+  const void* in = G_in;
+  for (int l = 0; l < n_layers; ++l) {
+    void* dst = ((n_layers - 1 - l) % 2 == 0) ? G_out : pong;
+    if (hg_ok) {
+      HgArgs ha;
+      ha.row_ptr = csr->row_ptr;
+      ha.sw = csr->sw;
+      ha.n_centres = n_centres;
+      ha.capacity = csr->capacity;
+      ha.G = in;
+      ha.out = dst;
+      ha.Wq = W[3 * l];
+      ha.Wk = W[3 * l + 1];
+      ha.Wv = W[3 * l + 2];
+      ha.status = csr->status;
+      rc = launch_hg_shape(dtype, channels, D, ha, stream);
+      if (rc != MLG_OK) return rc;
+    }
+    if (min_n >= 0) {
+      rc = launch_generic(csr, n_centres, nnei_max, channels, heads, dtype, in, dst, W[3 * l],
+                          W[3 * l + 1], W[3 * l + 2], min_n, stream);
+      if (rc != MLG_OK) return rc;
+    }
+    in = dst;
+  }
+  return MLG_OK;
+}
+
+int forward_launches(int64_t n_atoms, int32_t nnei_max, int32_t channels, int32_t heads,
+                     int32_t n_layers, mlg_dtype dtype) {
+  const int D = heads > 0 ? channels / heads : 0;
+  int R = tile_rows(dtype, channels, D);
+  if (R > 0 && n_layers <= kMaxFusedLayers) return 1 + (nnei_max > R ? n_layers : 0);
+  int Rg = hg_rows(dtype, channels, D);
+  if (Rg > 0) return n_layers * (1 + (nnei_max > Rg ? 1 : 0));
+  (void)n_atoms;
+  return n_layers;
 }
 
 }  // namespace
@@ -314,8 +477,28 @@ int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                         size_t ws_bytes, mlg_stream_t stream) {
   (void)ws;
   (void)ws_bytes;
-  return attention_impl(csr, n_centres, nnei_max, channels, heads, dtype, G_in, G_out, Wq, Wk,
-                        Wv, (cudaStream_t)stream);
+  const void* W[3] = {Wq, Wk, Wv};
+  if (!Wq || !Wk || !Wv) return MLG_ERR_INVALID_ARG;
+  return attention_stack_impl(csr, n_centres, nnei_max, channels, heads, dtype, 1, W, G_in, G_out,
+                              nullptr, (cudaStream_t)stream);
+}
+
+size_t mlg_attention_stack_workspace_bytes(int64_t capacity, int32_t channels, int32_t n_layers,
+                                           mlg_dtype dtype) {
+  if (capacity < 0 || channels < 1 || n_layers < 1) return 0;
+  size_t el = dtype == MLG_F64 ? 8 : 4;
+  return n_layers >= 2 ? align_up((size_t)(capacity > 0 ? capacity : 1) * channels * el) : 0;
+}
+
+int mlg_attention_stack(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                        int32_t channels, int32_t heads, int32_t n_layers, mlg_dtype dtype,
+                        const void* const* W, const void* G_in, void* G_out, void* ws,
+                        size_t ws_bytes, mlg_stream_t stream) {
+  if (csr == nullptr) return MLG_ERR_INVALID_ARG;
+  size_t need = mlg_attention_stack_workspace_bytes(csr->capacity, channels, n_layers, dtype);
+  if (need > 0 && (ws == nullptr || ws_bytes < need)) return MLG_ERR_WORKSPACE;
+  return attention_stack_impl(csr, n_centres, nnei_max, channels, heads, dtype, n_layers, W, G_in,
+                              G_out, need > 0 ? ws : nullptr, (cudaStream_t)stream);
 }
 
 size_t mlg_forward_workspace_bytes(int64_t n_atoms, double rcut, const double box[9],
@@ -349,28 +532,20 @@ int mlg_forward(const mlg_system* sys, double rcut, double r_on, int32_t nnei_ma
     if (W[k] == nullptr) return MLG_ERR_INVALID_ARG;
   int rc = build_impl(sys, rcut, r_on, nnei_max, csr, ws, build_need, (cudaStream_t)stream);
   if (rc != MLG_OK) return rc;
-  void* pong = static_cast<char*>(ws) + align_up(build_need);
-  const void* in = G0;
-  for (int l = 0; l < n_layers; ++l) {
-    // the last layer lands in G_out; earlier ones alternate so that a layer
-    // never reads the buffer it writes
-    void* dst = ((n_layers - 1 - l) % 2 == 0) ? G_out : pong;
-    rc = attention_impl(csr, sys->n_atoms, nnei_max, channels, heads, dtype, in, dst,
-                        W[3 * l], W[3 * l + 1], W[3 * l + 2], (cudaStream_t)stream);
-    if (rc != MLG_OK) return rc;
-    in = dst;
-  }
-  return MLG_OK;
+  void* pong = n_layers >= 2 ? static_cast<char*>(ws) + align_up(build_need) : nullptr;
+  return attention_stack_impl(csr, sys->n_atoms, nnei_max, channels, heads, dtype, n_layers, W,
+                              G0, G_out, pong, (cudaStream_t)stream);
 }
 
 int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
-                             const uint8_t pbc[3], int32_t n_layers) {
+                             const uint8_t pbc[3], int32_t nnei_max, int32_t channels,
+                             int32_t heads, int32_t n_layers, mlg_dtype dtype) {
   BuildPlan plan;
-  if (n_layers < 0 || make_plan(n_atoms, rcut, box, pbc, &plan) != MLG_OK) return 0;
+  if (n_layers < 1 || make_plan(n_atoms, rcut, box, pbc, &plan) != MLG_OK) return 0;
   auto scan_launches = [](int64_t n) { return n <= kScanSingleMax ? 1 : 3; };
-  // init, [bbox], bin, scan(cells), scatter, count, scan(row_ptr), fill, layers
+  // init, [bbox], bin, scan(cells), scatter, count, scan(row_ptr), fill, attention
   return 5 + (plan.any_open ? 1 : 0) + scan_launches(plan.ncell_cap) + scan_launches(n_atoms) +
-         n_layers;
+         forward_launches(n_atoms, nnei_max, channels, heads, n_layers, dtype);
 }
 
 const char* mlg_status_string(int status) {

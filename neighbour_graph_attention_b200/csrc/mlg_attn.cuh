@@ -33,6 +33,7 @@ struct AttnArgs {
   const void* Wk;
   const void* Wv;
   uint32_t* status;
+  int min_n;  // only centres with more than min_n edges (0: all)
 };
 
 template <typename T>
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn_generic(AttnArgs a) {
   for (int64_t i = blockIdx.x; i < a.n_centres; i += gridDim.x) {
     const int64_t base = a.row_ptr[i];
     const int n = (int)(a.row_ptr[i + 1] - base);
-    if (n <= 0 || n > NM || base + n > a.capacity) continue;
+    if (n <= a.min_n || n > NM || base + n > a.capacity) continue;
     for (int t = threadIdx.x; t < n; t += blockDim.x) sS[t] = (T)a.sw[base + t];
     __syncthreads();
     for (int h = 0; h < a.H; ++h) {

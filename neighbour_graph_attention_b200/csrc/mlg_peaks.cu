@@ -1,0 +1,151 @@
+// mlg_peaks.cu -- throughput microbenchmarks of the pipes the attention and
+// build kernels use, on the GPU they run on (prints one JSON object).
+//   fp64 FMA (DFMA), fp32 FMA (FFMA), fp64 tensor-core MMA (mma.sync f64
+//   m8n8k4 and m16n8k16), and the special-function pipe (ex2.approx.f32).
+// Each kernel runs independent dependency chains per thread so that the pipe,
+// not latency, limits it; results feed a global store so nothing is removed.
+#include <cstdio>
+#include <cuda_runtime.h>
+
+template <typename T>
+__global__ void k_fma(T* out, int iters, T seed) {
+  T a[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = seed + T(threadIdx.x + j);
+  const T b = T(0.999999), c = T(1e-7);
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = fma(a[j], b, c);
+  }
+  T s = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) s += a[j];
+  if (s == T(-1)) out[blockIdx.x] = s;
+}
+
+__global__ void k_ex2(float* out, int iters) {
+  float a[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = -1e-3f * (threadIdx.x + j);
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float r;
+        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(a[j]));
+        a[j] = r - 1.0f;
+      }
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) s += a[j];
+  if (s == -1.f) out[blockIdx.x] = s;
+}
+
+__global__ void k_dmma884(double* out, int iters) {
+  double a = 1.0 + threadIdx.x * 1e-9, b = 0.5;
+  double c[4][2];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = 0.0;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        asm volatile(
+            "mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+            : "+d"(c[j][0]), "+d"(c[j][1])
+            : "d"(a), "d"(b));
+  }
+  double s = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) s += c[j][0] + c[j][1];
+  if (s == -1.0) out[blockIdx.x] = s;
+}
+
+__global__ void k_dmma16816(double* out, int iters) {
+  double a[8], b[4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = 1.0 + (threadIdx.x + i) * 1e-9;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) b[i] = 0.5;
+  double c[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[j][i] = 0.0;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      asm volatile(
+          "mma.sync.aligned.m16n8k16.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, "
+          "{%4,%5,%6,%7,%8,%9,%10,%11}, {%12,%13,%14,%15}, {%0,%1,%2,%3};"
+          : "+d"(c[j][0]), "+d"(c[j][1]), "+d"(c[j][2]), "+d"(c[j][3])
+          : "d"(a[0]), "d"(a[1]), "d"(a[2]), "d"(a[3]), "d"(a[4]), "d"(a[5]), "d"(a[6]),
+            "d"(a[7]), "d"(b[0]), "d"(b[1]), "d"(b[2]), "d"(b[3]));
+  }
+  double s = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s += c[j][i];
+  if (s == -1.0) out[blockIdx.x] = s;
+}
+
+template <class F>
+float time_ms(F launch) {
+  cudaEvent_t a, b;
+  cudaEventCreate(&a);
+  cudaEventCreate(&b);
+  launch();
+  cudaDeviceSynchronize();
+  float best = 1e30f;
+  for (int r = 0; r < 5; ++r) {
+    cudaEventRecord(a);
+    launch();
+    cudaEventRecord(b);
+    cudaEventSynchronize(b);
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, a, b);
+    if (ms < best) best = ms;
+  }
+  cudaEventDestroy(a);
+  cudaEventDestroy(b);
+  return best;
+}
+
+int main() {
+  int dev = 0, sms = 0, clk = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&clk, cudaDevAttrClockRate, dev);
+  double* dbuf;
+  float* fbuf;
+  cudaMalloc(&dbuf, 1 << 20);
+  cudaMalloc(&fbuf, 1 << 20);
+  const int blocks = sms * 8, threads = 256, iters = 4096;
+  const double lanes = (double)blocks * threads;
+  float t;
+  t = time_ms([&] { k_fma<double><<<blocks, threads>>>(dbuf, iters, 1.0); });
+  double dfma = lanes * iters * 16 * 8 * 2 / (t * 1e-3) / 1e12;
+  t = time_ms([&] { k_fma<float><<<blocks, threads>>>(fbuf, iters, 1.0f); });
+  double ffma = lanes * iters * 16 * 8 * 2 / (t * 1e-3) / 1e12;
+  t = time_ms([&] { k_ex2<<<blocks, threads>>>(fbuf, iters / 4); });
+  double ex2 = lanes * (iters / 4) * 16 * 8 / (t * 1e-3) / 1e12;
+  const double warps = (double)blocks * threads / 32;
+  t = time_ms([&] { k_dmma884<<<blocks, threads>>>(dbuf, iters / 4); });
+  double dmma884 = warps * (iters / 4) * 16 * (2.0 * 8 * 8 * 4) / (t * 1e-3) / 1e12;
+  t = time_ms([&] { k_dmma16816<<<blocks, threads>>>(dbuf, iters / 16); });
+  double dmma16816 = warps * (iters / 16) * 4 * (2.0 * 16 * 8 * 16) / (t * 1e-3) / 1e12;
+  cudaError_t e = cudaGetLastError();
+  printf("{\"sm_count\": %d, \"clock_khz_attr\": %d, \"fp64_fma_tflops\": %.3f, "
+         "\"fp32_fma_tflops\": %.3f, \"ex2_tops\": %.4f, \"dmma_m8n8k4_tflops\": %.3f, "
+         "\"dmma_m16n8k16_tflops\": %.3f, \"cuda\": \"%s\"}\n",
+         sms, clk, dfma, ffma, ex2, dmma884, dmma16816, cudaGetErrorString(e));
+  cudaFree(dbuf);
+  cudaFree(fbuf);
+  return e == cudaSuccess ? 0 : 1;
+}

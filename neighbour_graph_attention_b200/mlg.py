@@ -41,6 +41,7 @@ MLG_STATUS_CAPACITY = 4
 MLG_STATUS_IMAGE_RANGE = 8
 MLG_STATUS_TIES = 16
 MLG_STATUS_INTERNAL = 32
+MLG_STATUS_TIMEOUT = 64
 
 MLG_F32 = 0
 MLG_F64 = 1
@@ -80,7 +81,14 @@ _lib.mlg_build_csr_noalloc.restype = ctypes.c_int
 _lib.mlg_build_csr_noalloc.argtypes = [ctypes.POINTER(mlg_system), _c_dbl, _c_dbl, _c_i32,
                                        ctypes.POINTER(mlg_csr), _p]
 _lib.mlg_forward_launch_count.restype = ctypes.c_int
-_lib.mlg_forward_launch_count.argtypes = [_c_i64, _c_dbl, _p, _p, _c_i32]
+_lib.mlg_forward_launch_count.argtypes = [_c_i64, _c_dbl, _p, _p, _c_i32, _c_i32, _c_i32, _c_i32,
+                                          ctypes.c_int]
+_lib.mlg_attention_stack_workspace_bytes.restype = _c_sz
+_lib.mlg_attention_stack_workspace_bytes.argtypes = [_c_i64, _c_i32, _c_i32, ctypes.c_int]
+_lib.mlg_attention_stack.restype = ctypes.c_int
+_lib.mlg_attention_stack.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32, _c_i32,
+                                     _c_i32, ctypes.c_int, ctypes.POINTER(_p), _p, _p, _p, _c_sz,
+                                     _p]
 _lib.mlg_status_string.restype = ctypes.c_char_p
 _lib.mlg_status_string.argtypes = [ctypes.c_int]
 _lib.mlg_version.restype = ctypes.c_int
@@ -197,10 +205,33 @@ def mlg_forward_workspace_bytes(n_atoms: int, rcut: float, box, pbc, capacity: i
                                                 int(n_layers), int(dtype)))
 
 
-def mlg_forward_launch_count(n_atoms: int, rcut: float, box, pbc, n_layers: int) -> int:
+def mlg_forward_launch_count(n_atoms: int, rcut: float, box, pbc, nnei_max: int,
+                             channels: int, heads: int, n_layers: int, dtype: int) -> int:
     b, q = _box_pbc(box, pbc)
     return int(_lib.mlg_forward_launch_count(int(n_atoms), float(rcut), b.ctypes.data,
-                                             q.ctypes.data, int(n_layers)))
+                                             q.ctypes.data, int(nnei_max), int(channels),
+                                             int(heads), int(n_layers), int(dtype)))
+
+
+def mlg_attention_stack_workspace_bytes(capacity: int, channels: int, n_layers: int,
+                                        dtype: int) -> int:
+    return int(_lib.mlg_attention_stack_workspace_bytes(int(capacity), int(channels),
+                                                        int(n_layers), int(dtype)))
+
+
+def mlg_attention_stack(csr: Csr, n_centres: int, nnei_max: int, channels: int, heads: int,
+                        n_layers: int, dtype: int, W, G_in, G_out, ws=None,
+                        ws_bytes: int | None = None, stream=None, check: bool = True) -> int:
+    """Launch ``n_layers`` fused attention layers. ``W``: 3 * n_layers device tensors."""
+    ptrs = (_p * len(W))(*[_ptr(w) for w in W])
+    c = csr.struct()
+    nbytes = 0 if ws is None else (int(ws.numel() * ws.element_size()) if ws_bytes is None
+                                   else int(ws_bytes))
+    code = _lib.mlg_attention_stack(ctypes.byref(c), int(n_centres), int(nnei_max),
+                                    int(channels), int(heads), int(n_layers), int(dtype), ptrs,
+                                    _ptr(G_in), _ptr(G_out), _ptr(ws), nbytes,
+                                    _stream_handle(stream))
+    return _check(code, "mlg_attention_stack", check)
 
 
 def _check(code: int, where: str, check: bool):

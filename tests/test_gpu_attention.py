@@ -149,3 +149,52 @@ def test_forward_graph_capture_and_side_stream():
         graph_.replay()
     torch.cuda.synchronize()
     assert torch.equal(out3, ref_out)
+
+
+def _random_graph(n_atoms, density, rcut, nnei_max, seed):
+    rng = np.random.default_rng(seed)
+    L = (n_atoms / density) ** (1.0 / 3.0)
+    x = rng.uniform(0.0, L, size=(n_atoms, 3))
+    gpu, csr_t = U.gpu_build(x, np.diag([L] * 3), [1, 1, 1], rcut, rcut - 0.5, nnei_max)
+    return gpu, csr_t
+
+
+@pytest.mark.parametrize("dtype,channels,heads,n_layers,density,nnei", [
+    ("f64", 32, 4, 3, 0.13, 64),   # ~40 edges: fused tile (<= 40) + generic for larger rows
+    ("f32", 64, 4, 1, 0.41, 181),  # ~128 edges: fused tile (<= 128) + generic for larger
+    ("f32", 32, 4, 2, 0.004, 128), # dilute: many centres without edges between full ones
+    ("f64", 128, 4, 2, 0.3, 96),   # head-group kernel, two layers (ping-pong)
+    ("f32", 128, 8, 2, 0.31, 181), # head-group kernel (<= 96 edges) + generic for larger
+])
+def test_stack_mixed_row_sizes(dtype, channels, heads, n_layers, density, nnei):
+    import oracle
+    from neighbour_graph_attention_b200.configs import Workload
+
+    m = U.mlg()
+    gpu, csr_t = _random_graph(3000, density, 4.2, nnei, 17)
+    counts = np.diff(gpu["row_ptr"])
+    e = gpu["n_edges"]
+    w = Workload(0, "random", "random", 0, 0, 0, 3000, 4.2, 3.7, nnei, channels, heads, n_layers,
+                 dtype)
+    rng = np.random.default_rng(5)
+    W = rng.normal(0, 1 / np.sqrt(channels), (n_layers, 3, channels, channels)).astype(w.np_dtype)
+    G = rng.normal(0, 1, (e, channels)).astype(w.np_dtype)
+    dt = U.torch_dtype(w)
+    g0 = torch.zeros((csr_t.capacity, channels), dtype=dt, device="cuda")
+    g0[:e] = torch.as_tensor(G, device="cuda")
+    gout = torch.zeros_like(g0)
+    Wt = [torch.as_tensor(W[l][k], device="cuda") for l in range(n_layers) for k in range(3)]
+    ws = m.workspace(m.mlg_attention_stack_workspace_bytes(csr_t.capacity, channels, n_layers,
+                                                           U.mlg_dtype(w)))
+    m.mlg_attention_stack(csr_t, 3000, nnei, channels, heads, n_layers, U.mlg_dtype(w), Wt, g0,
+                          gout, ws)
+    torch.cuda.synchronize()
+    assert int(csr_t.status.item()) == 0
+    outs = oracle.forward(gpu["row_ptr"], gpu["sw"], G, W, heads, dtype)
+    ok, err = U.attn_tolerance_ok(w, gout[:e].cpu().numpy(), outs[-1])
+    assert ok, (err, counts.min(), counts.max())
+    if density in (0.13, 0.41, 0.31):    # both sides of the tile limit are exercised
+        limit = {0.13: 40, 0.41: 128, 0.31: 96}[density]
+        assert counts.min() <= limit < counts.max()
+    # rows past E are never written
+    assert bool((gout[e:] == 0).all())

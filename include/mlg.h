@@ -77,8 +77,8 @@ typedef enum {
                                         attention skipped */
     MLG_STATUS_IMAGE_RANGE = 8u,     /* an atom lies more than 511 box lengths outside the
                                         box along a periodic axis; it was left out */
-    MLG_STATUS_TIES = 16u,           /* truncation met more than 256 candidates at one
-                                        distance; the kept set is not canonical */
+    MLG_STATUS_TIES = 16u,           /* reserved (no longer raised: ties at the cap are
+                                        broken exactly by (source, shift)) */
     MLG_STATUS_INTERNAL = 32u,       /* the count and fill passes disagreed on a row (never
                                         expected); that row is incomplete */
     MLG_STATUS_TIMEOUT = 64u         /* a bounded wait for an on-chip copy ran out (never

@@ -25,7 +25,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // Layout of the build workspace.
 struct BuildLayout {
-  size_t grid, bbox, cell_count, cell_start, atom_cell, atom_rank, atom_w, recs, kept, raw,
+  size_t grid, bbox, cell_count, cell_start, atom_cell, atom_rank, atom_w, recs, pos4, kept, raw,
       partial, total;
 };
 
@@ -47,6 +47,7 @@ BuildLayout build_layout(int64_t n, int ncell_cap) {
   L.atom_rank = take((size_t)n * sizeof(int));
   L.atom_w = take((size_t)n * sizeof(int));
   L.recs = take((size_t)n * sizeof(Rec));
+  L.pos4 = take((size_t)n * sizeof(float4));
   L.kept = take((size_t)n * sizeof(int));
   L.raw = take((size_t)n * sizeof(int));
   int64_t tiles = scan_tiles(n > ncell_cap ? n : ncell_cap + 1);
@@ -71,6 +72,7 @@ int make_plan(int64_t n, double rcut, const double* box, const uint8_t* pbc, Bui
   std::memset(p, 0, sizeof(*p));
   const double delta = 1e-6 * (rcut > 1.0 ? rcut : 1.0);
   p->rcd = rcut + delta;
+  p->rc2 = rcut * rcut;
   const double budget = (double)(n > 32 ? 2 * n : 64);
   double prod = 1.0;
   int n_open = 0;
@@ -106,6 +108,7 @@ int make_plan(int64_t n, double rcut, const double* box, const uint8_t* pbc, Bui
     double reach = std::ceil(p->rcd * (double)p->n_fixed[k] / p->L[k]);
     if (reach > kMaxReach) return MLG_ERR_UNSUPPORTED;  // box far smaller than rcut
     p->D_fixed[k] = reach < 1.0 ? 1 : (int)reach;
+    if (p->D_fixed[k] > p->max_reach) p->max_reach = p->D_fixed[k];
   }
   int open_cap = 1;
   if (n_open > 0) {
@@ -160,6 +163,8 @@ int check_csr(const mlg_csr* csr) {
   return MLG_OK;
 }
 
+int sm_count();
+
 int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
                const mlg_csr* csr, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (sys == nullptr || sys->coords == nullptr) return MLG_ERR_INVALID_ARG;
@@ -208,6 +213,7 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   a.atom_rank = reinterpret_cast<int*>(w + L.atom_rank);
   a.atom_w = reinterpret_cast<int*>(w + L.atom_w);
   a.recs = reinterpret_cast<Rec*>(w + L.recs);
+  a.pos4 = reinterpret_cast<float4*>(w + L.pos4);
   a.kept = reinterpret_cast<int*>(w + L.kept);
   a.raw = reinterpret_cast<int*>(w + L.raw);
   a.partial = reinterpret_cast<long long*>(w + L.partial);
@@ -225,11 +231,28 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   launch_scan<int>(a.cell_count, plan.ncell_cap, a.cell_start, a.partial,
                    ScanTail{nullptr, nullptr, 0}, stream);
   k_scatter<<<atom_blocks, tb, 0, stream>>>(a);
-  k_count<<<(int)((n + kCountWarps - 1) / kCountWarps), kCountWarps * 32, 0, stream>>>(a);
+  // per-cell scans when every stencil reach is 1 (at most 27 stencil cells);
+  // otherwise (boxes narrower than the cutoff) the per-centre scans
+  // (a grid of few cells would leave most SMs idle: per-centre scans there)
+  const bool per_cell = plan.max_reach <= 1 && plan.ncell_cap >= 4 * sm_count();
+  if (per_cell) {
+    const size_t sm_count_ = cellscan_smem(false), sm_fill = cellscan_smem(true);
+    cudaFuncSetAttribute(k_cellscan<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)sm_count_);
+    cudaFuncSetAttribute(k_cellscan<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)sm_fill);
+    k_cellscan<false><<<plan.ncell_cap, kCellWarps * 32, sm_count_, stream>>>(a);
+  } else {
+    k_count<<<(int)((n + kCountWarps - 1) / kCountWarps), kCountWarps * 32, 0, stream>>>(a);
+  }
   launch_scan<long long>(a.kept, n, reinterpret_cast<long long*>(a.row_ptr), a.partial,
                          ScanTail{a.n_edges, a.status, a.capacity}, stream);
-  const size_t fill_smem = (size_t)kFillWarps * 2 * kFillMaxCand * sizeof(unsigned long long);
-  k_fill<<<(int)((n + kFillWarps - 1) / kFillWarps), kFillWarps * 32, fill_smem, stream>>>(a);
+  if (per_cell) {
+    k_cellscan<true><<<plan.ncell_cap, kCellWarps * 32, cellscan_smem(true), stream>>>(a);
+  } else {
+    const size_t fill_smem = (size_t)kFillWarps * 2 * kFillMaxCand * sizeof(unsigned long long);
+    k_fill<<<(int)((n + kFillWarps - 1) / kFillWarps), kFillWarps * 32, fill_smem, stream>>>(a);
+  }
   return launch_status();
 }
 

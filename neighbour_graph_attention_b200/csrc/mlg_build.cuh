@@ -58,6 +58,8 @@ struct CellGrid {
   int D[3];         // stencil reach in cells
   int periodic[3];
   int ncell;
+  float Lf[3];      // box lengths as float (0 along open axes)
+  float r2lo, r2hi; // fp32 prefilter: r2f < r2lo surely inside, r2f > r2hi surely outside
 };
 
 // What the host fixes before launch.
@@ -68,8 +70,10 @@ struct BuildPlan {
   int D_fixed[3];     // periodic axes: stencil reach
   int n_open_max[3];  // open axes: most cells allowed
   double rcd;         // minimum cell size along open axes (rcut plus margin)
+  double rc2;         // rcut * rcut
   int any_open;
   int ncell_cap;
+  int max_reach;      // largest stencil reach over the axes
 };
 
 struct BuildArgs {
@@ -100,12 +104,13 @@ struct BuildArgs {
   int* atom_rank;            // [n]
   int* atom_w;               // [n]
   Rec* recs;                 // [n]
+  float4* pos4;              // [n] cell order: position in the grid frame (fp32), atom index
   int* kept;                 // [n]
   int* raw;                  // [n]
   long long* partial;        // scan partials
 };
 
-constexpr int kFillMaxCand = 512;  // shared-memory candidates per destination
+constexpr int kFillMaxCand = 256;  // shared-memory candidates per destination
 constexpr int kCountWarps = 8;
 constexpr int kFillWarps = 4;
 
@@ -166,6 +171,7 @@ __device__ __forceinline__ CellGrid derive_grid(const BuildPlan& p,
                                                 const unsigned long long* bbox) {
   CellGrid g;
   int nc = 1;
+  double ext = 0.0;  // largest coordinate span of the grid frame
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
     g.periodic[k] = p.periodic[k];
@@ -189,6 +195,7 @@ __device__ __forceinline__ CellGrid derive_grid(const BuildPlan& p,
         while (n > 1 && ext / (double)n < p.rcd) --n;
       }
       g.lo[k] = lo <= hi ? lo : 0.0;
+      if (lo <= hi) ext = fmax(ext, hi - lo);
       g.n[k] = n;
       g.inv_h[k] = n > 1 ? (double)n / ext : 0.0;
       g.D[k] = n > 1 ? 1 : 0;
@@ -196,6 +203,23 @@ __device__ __forceinline__ CellGrid derive_grid(const BuildPlan& p,
     nc *= g.n[k];
   }
   g.ncell = nc;
+  // fp32 prefilter margin.  Positions are stored in the grid frame (wrapped
+  // along periodic axes, shifted by the bounding-box origin along open ones),
+  // |p| <= ext; an image adds +-L.  Each fp32 coordinate of a difference
+  // carries at most 4 roundings of 2^-24 * 2 ext, so |delta_k| <= 2^-20 * ext
+  // bounds its error with room to spare; r^2 then moves by at most
+  // 2 sqrt(3) rcut delta + 3 delta^2 plus the fp32 rounding of the sum.
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    if (g.periodic[k]) ext = fmax(ext, g.L[k]);
+    g.Lf[k] = (float)g.L[k];
+  }
+  const double rc = p.rcd, rc2 = rc * rc;
+  const double dlt = 2.0 * 9.5367431640625e-07 * (ext + rc);  // 2 * 2^-20 * (ext + rc)
+  const double margin = 2.0 * (3.4641016151377544 * rc * dlt + 3.0 * dlt * dlt) +
+                        16.0 * 5.9604644775390625e-08 * rc2;
+  g.r2lo = __double2float_rd(fmax(0.0, p.rc2 - margin));
+  g.r2hi = __double2float_ru(p.rc2 + margin);
   return g;
 }
 
@@ -290,6 +314,10 @@ __global__ void k_bin(BuildArgs a, BuildPlan p) {
     }
     a.atom_cell[i] = cell;
     a.atom_w[i] = wpack;
+    if (cell < 0) {  // left out of the cell lists: no centre scan will visit it
+      a.kept[i] = 0;
+      a.raw[i] = 0;
+    }
   }
   // warp-aggregated atomics on the cell histogram
   unsigned act = __ballot_sync(kFull, cell >= 0);
@@ -306,6 +334,9 @@ __global__ void k_bin(BuildArgs a, BuildPlan p) {
 }
 
 __global__ void k_scatter(BuildArgs a) {
+  __shared__ CellGrid sg;
+  if (threadIdx.x == 0) sg = *a.grid;
+  __syncthreads();
   int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.n) return;
   int cell = a.atom_cell[i];
@@ -316,7 +347,14 @@ __global__ void k_scatter(BuildArgs a) {
   r.z = a.coords[3 * i + 2];
   r.j = (int)i;
   r.w = a.atom_w[i];
-  a.recs[a.cell_start[cell] + a.atom_rank[i]] = r;
+  const int pos = a.cell_start[cell] + a.atom_rank[i];
+  a.recs[pos] = r;
+  double x[3] = {r.x, r.y, r.z};
+  float y[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k)
+    y[k] = (float)(sg.periodic[k] ? x[k] - (double)unpack_w(r.w, k) * sg.L[k] : x[k] - sg.lo[k]);
+  a.pos4[pos] = make_float4(y[0], y[1], y[2], __int_as_float((int)i));
 }
 
 // ----------------------------------------------------- candidate traversal
@@ -528,126 +566,80 @@ __device__ __forceinline__ unsigned long long edge_key(int j, int tpack) {
   return ((unsigned long long)(unsigned)j << 21) | (unsigned long long)tpack;
 }
 
-// Threshold search for rows with more than kFillMaxCand candidates: find the
-// nnei_max-th smallest r^2 by bisection over its bit pattern (monotone for
-// non-negative doubles), then break ties at that distance by key.
+// Selection for rows with more than kFillMaxCand candidates, without a
+// candidate buffer: bisection over the bit pattern of r^2 (monotone for
+// non-negative doubles) finds the nnei_max-th smallest distance; a second
+// bisection over the key (source, image) orders the candidates at exactly that
+// distance.  Each probe rescans the row's candidates.  Writes the n kept keys
+// to keys[0..n) (any order) and returns how many it wrote.
 __device__ int fill_overflow_select(const BuildArgs& a, const CellGrid& g, const Centre& cc,
                                     WarpScratch& ws, unsigned long long* keys, int n,
                                     uint32_t* st) {
-  const unsigned lane = lane_id();
-  unsigned long long lo = 0ull, hi = (unsigned long long)__double_as_longlong(a.rc2);
-  while (lo < hi) {
-    unsigned long long mid = lo + ((hi - lo) >> 1);
+  (void)st;
+  // count of candidates with (r2 bits, key) <= (b2, bk) in lexicographic order
+  auto count_le = [&](unsigned long long b2, unsigned long long bk) {
     int cnt = 0;
     for_each_candidate(g, a.cell_start, cc, ws, [&](bool valid, int r, int tp) {
       if (valid) {
+        const Rec rc = a.recs[r];
         double r2;
-        if (test_candidate(g, cc, a.recs[r], tp, a.rc2, &r2) &&
-            (unsigned long long)__double_as_longlong(r2) <= mid)
-          ++cnt;
+        if (test_candidate(g, cc, rc, tp, a.rc2, &r2)) {
+          const unsigned long long b = (unsigned long long)__double_as_longlong(r2);
+          const unsigned long long k = edge_key(rc.j, tp);
+          if (b < b2 || (b == b2 && k <= bk)) ++cnt;
+        }
       }
     });
-    cnt = warp_sum(cnt);
-    if (cnt >= n) hi = mid; else lo = mid + 1;
+    return warp_sum(cnt);
+  };
+  unsigned long long lo = 0ull, hi = (unsigned long long)__double_as_longlong(a.rc2);
+  while (lo < hi) {  // smallest distance bits t with count(r2 <= t) >= n
+    const unsigned long long mid = lo + ((hi - lo) >> 1);
+    if (count_le(mid, ~0ull) >= n) hi = mid; else lo = mid + 1;
   }
-  const unsigned long long thr = lo;
-  // below the threshold -> keys[0..nlt); at the threshold -> keys[256..)
-  int nlt = 0, neq = 0;
-  const int tie_base = 256, tie_cap = kFillMaxCand - 256;
+  const unsigned long long t2 = lo;
+  unsigned long long klo = 0ull, khi = (1ull << 53) - 1;
+  while (klo < khi) {  // smallest key kt with count((r2, key) <= (t2, kt)) >= n
+    const unsigned long long mid = klo + ((khi - klo) >> 1);
+    if (count_le(t2, mid) >= n) khi = mid; else klo = mid + 1;
+  }
+  const unsigned long long tk = klo;
+  int pos = 0;
   for_each_candidate(g, a.cell_start, cc, ws, [&](bool valid, int r, int tp) {
-    bool lt = false, eq = false;
+    bool take = false;
     unsigned long long key = 0;
     if (valid) {
       const Rec rc = a.recs[r];
       double r2;
       if (test_candidate(g, cc, rc, tp, a.rc2, &r2)) {
-        unsigned long long b = (unsigned long long)__double_as_longlong(r2);
-        lt = b < thr;
-        eq = b == thr;
+        const unsigned long long b = (unsigned long long)__double_as_longlong(r2);
         key = edge_key(rc.j, tp);
+        take = b < t2 || (b == t2 && key <= tk);
       }
     }
-    unsigned mlt = __ballot_sync(kFull, lt), meq = __ballot_sync(kFull, eq);
-    if (lt) {
-      int q = nlt + __popc(mlt & lanemask_lt());
-      if (q < tie_base) keys[q] = key;
+    const unsigned m = __ballot_sync(kFull, take);
+    if (take) {
+      const int q = pos + __popc(m & lanemask_lt());
+      if (q < n) keys[q] = key;
     }
-    if (eq) {
-      int q = neq + __popc(meq & lanemask_lt());
-      if (q < tie_cap) keys[tie_base + q] = key;
-    }
-    nlt += __popc(mlt);
-    neq += __popc(meq);
+    pos += __popc(m);
   });
   __syncwarp();
-  if (neq > tie_cap) {
-    if (lane == 0) *st |= MLG_STATUS_TIES;
-    neq = tie_cap;
-  }
-  warp_sort_keys(keys + tie_base, neq);
-  // nlt < n <= 256 and nlt + neq >= n hold when this pass saw what the count
-  // pass saw; clamp anyway so that only collected keys are ever used
-  const int nlt_c = nlt < n ? nlt : n;
-  int take = n - nlt_c;
-  if (take > neq) take = neq;
-  for (int t = lane; t < take; t += 32) keys[nlt_c + t] = keys[tie_base + t];
-  __syncwarp();
-  return nlt_c + take;
+  return pos < n ? pos : n;
 }
 
-__global__ void __launch_bounds__(kFillWarps * 32) k_fill(BuildArgs a) {
-  __shared__ CellGrid sg;
-  __shared__ WarpScratch sws[kFillWarps];
-  extern __shared__ unsigned long long s_fill[];  // [warps][2][kFillMaxCand]
-  if (threadIdx.x == 0) sg = *a.grid;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5;
+// Sort the collected keys of one row into canonical order and write its
+// edges.  keys/d2 hold m collected candidates (keys and exact r^2 bits); the
+// row keeps n = min(raw, nnei_max).  Returns status bits.
+__device__ uint32_t finish_row(const BuildArgs& a, const Centre& cc, unsigned long long* keys,
+                               unsigned long long* d2, int n, int m, int64_t p0) {
   const unsigned lane = lane_id();
-  const int64_t i = (int64_t)blockIdx.x * kFillWarps + warp;
-  if (i >= a.n) return;
-  const int cell = a.atom_cell[i];
-  const int n = a.kept[i];
-  if (cell < 0 || n == 0) return;
-  const int raw = a.raw[i];
-  const int64_t p0 = a.row_ptr[i];
-  unsigned long long* keys = s_fill + (size_t)warp * 2 * kFillMaxCand;
-  unsigned long long* d2 = keys + kFillMaxCand;
-  Centre cc = load_centre(a, sg, (int)i, cell);
   uint32_t st = 0;
-  int nv = 0;  // keys collected for this row; equals n unless the passes disagree
-  if (raw <= kFillMaxCand) {
-    int pos = 0;
-    for_each_candidate(sg, a.cell_start, cc, sws[warp], [&](bool valid, int r, int tp) {
-      bool acc = false;
-      unsigned long long key = 0, b = 0;
-      if (valid) {
-        const Rec rc = a.recs[r];
-        double r2;
-        acc = test_candidate(sg, cc, rc, tp, a.rc2, &r2);
-        key = edge_key(rc.j, tp);
-        b = (unsigned long long)__double_as_longlong(r2);
-      }
-      unsigned m = __ballot_sync(kFull, acc);
-      if (acc) {
-        int q = pos + __popc(m & lanemask_lt());
-        if (q < kFillMaxCand) {
-          keys[q] = key;
-          d2[q] = b;
-        }
-      }
-      pos += __popc(m);
-    });
-    __syncwarp();
-    const int m = pos < kFillMaxCand ? pos : kFillMaxCand;
-    if (m > n) warp_sort_pairs(d2, keys, m);
-    nv = n < m ? n : m;
-    warp_sort_keys(keys, nv);
-  } else {
-    nv = fill_overflow_select(a, sg, cc, sws[warp], keys, n, &st);
-    warp_sort_keys(keys, nv);
-  }
+  if (m > kFillMaxCand) m = kFillMaxCand;
+  if (m > n) warp_sort_pairs(d2, keys, m);
+  const int nv = n < m ? n : m;
+  warp_sort_keys(keys, nv);
   if (nv != n) st |= MLG_STATUS_INTERNAL;
-  // canonical order now in keys[0..nv): write the SoA edge arrays
   for (int e = lane; e < nv; e += 32) {
     unsigned long long key = keys[e];
     int j = (int)(key >> 21);
@@ -676,7 +668,286 @@ __global__ void __launch_bounds__(kFillWarps * 32) k_fill(BuildArgs a) {
       a.sw[p] = switch_fn(r, a.rcut, a.r_on, a.taylor);
     }
   }
-  if (lane == 0 && st) atomicOr(a.status, st);
+  return st;
+}
+
+// One row from the global cell lists (rows beyond the shared-memory
+// candidate capacity take the threshold search).
+__device__ uint32_t fill_row_global(const BuildArgs& a, const CellGrid& g, const Centre& cc,
+                                    WarpScratch& ws, unsigned long long* keys,
+                                    unsigned long long* d2, int n, int raw, int64_t p0) {
+  uint32_t st = 0;
+  if (raw <= kFillMaxCand) {
+    int pos = 0;
+    for_each_candidate(g, a.cell_start, cc, ws, [&](bool valid, int r, int tp) {
+      bool acc = false;
+      unsigned long long key = 0, b = 0;
+      if (valid) {
+        const Rec rc = a.recs[r];
+        double r2;
+        acc = test_candidate(g, cc, rc, tp, a.rc2, &r2);
+        key = edge_key(rc.j, tp);
+        b = (unsigned long long)__double_as_longlong(r2);
+      }
+      unsigned m = __ballot_sync(kFull, acc);
+      if (acc) {
+        int q = pos + __popc(m & lanemask_lt());
+        if (q < kFillMaxCand) {
+          keys[q] = key;
+          d2[q] = b;
+        }
+      }
+      pos += __popc(m);
+    });
+    __syncwarp();
+    st |= finish_row(a, cc, keys, d2, n, pos, p0);
+  } else {
+    const int nv = fill_overflow_select(a, g, cc, ws, keys, n, &st);
+    st |= finish_row(a, cc, keys, d2, nv, nv, p0);
+    if (nv != n) st |= MLG_STATUS_INTERNAL;
+  }
+  return st;
+}
+
+__global__ void __launch_bounds__(kFillWarps * 32) k_fill(BuildArgs a) {
+  __shared__ CellGrid sg;
+  __shared__ WarpScratch sws[kFillWarps];
+  extern __shared__ unsigned long long s_fill[];  // [warps][2][kFillMaxCand]
+  if (threadIdx.x == 0) sg = *a.grid;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  const int64_t i = (int64_t)blockIdx.x * kFillWarps + warp;
+  if (i >= a.n) return;
+  const int cell = a.atom_cell[i];
+  const int n = a.kept[i];
+  if (cell < 0 || n == 0) return;
+  unsigned long long* keys = s_fill + (size_t)warp * 2 * kFillMaxCand;
+  Centre cc = load_centre(a, sg, (int)i, cell);
+  uint32_t st = fill_row_global(a, sg, cc, sws[warp], keys, keys + kFillMaxCand, n, a.raw[i],
+                                a.row_ptr[i]);
+  if (lane_id() == 0 && st) atomicOr(a.status, st);
+}
+
+// ------------------------------------------------------------ per-cell scans
+//
+// One CTA per cell: every centre of a cell has the same 27 stencil cells, so
+// their atoms are staged once in shared memory as fp32 positions with the
+// image offset T L already added.  A candidate then costs one 16-byte
+// shared load and a few fp32 operations; only candidates within the margin
+// of rcut^2 (r2lo <= r2f <= r2hi) take the exact fp64 test, so the accept
+// decision is the fp64 one bit for bit.  Cells whose stencil holds more than
+// kCellCand atoms fall back to the per-centre traversal of global memory.
+
+constexpr int kCellCand = 768;
+constexpr int kCellWarps = 8;
+
+struct CellStage {
+  int pre[33];      // candidate offset of each stencil cell
+  int start[32];
+  int tpack[32];
+  int ncand;
+  int fallback;
+  int trunc;
+  float4 cand[kCellCand];   // position + image offset, atom index in .w
+  int cq[kCellCand];        // cell-order index (record of the exact data)
+  int ct[kCellCand];        // packed image of the stencil cell
+};
+
+template <bool FILL>
+__global__ void __launch_bounds__(kCellWarps * 32, 2) k_cellscan(BuildArgs a) {
+  __shared__ CellGrid sg;
+  __shared__ WarpScratch sws[kCellWarps];
+  extern __shared__ __align__(16) unsigned char s_dyn[];
+  CellStage& cs = *reinterpret_cast<CellStage*>(s_dyn);
+  unsigned long long* s_keys =
+      reinterpret_cast<unsigned long long*>(s_dyn + ((sizeof(CellStage) + 15) / 16) * 16);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) sg = *a.grid;
+  __syncthreads();
+  const int cell = blockIdx.x;
+  if (cell >= sg.ncell) return;
+  const int c_lo = a.cell_start[cell], c_hi = a.cell_start[cell + 1];
+  if (c_lo == c_hi) return;
+  const int cz = cell % sg.n[2], cy = (cell / sg.n[2]) % sg.n[1], cx = cell / (sg.n[2] * sg.n[1]);
+  if (warp == 0) {
+    // stencil (reach <= 1 on every axis: at most 27 cells)
+    const int w0 = 2 * sg.D[0] + 1, w1 = 2 * sg.D[1] + 1, w2 = 2 * sg.D[2] + 1;
+    const int s3 = w0 * w1 * w2;
+    int len = 0, start = 0, tp = 0;
+    if (lane < s3) {
+      int d[3];
+      d[2] = lane % w2 - sg.D[2];
+      d[1] = (lane / w2) % w1 - sg.D[1];
+      d[0] = lane / (w2 * w1) - sg.D[0];
+      const int c[3] = {cx, cy, cz};
+      int m[3], T[3];
+      bool ok = true;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        int e = c[k] + d[k];
+        if (sg.periodic[k]) {
+          T[k] = floordiv(e, sg.n[k]);
+          m[k] = e - T[k] * sg.n[k];
+        } else {
+          ok = ok && e >= 0 && e < sg.n[k];
+          m[k] = e;
+          T[k] = 0;
+        }
+      }
+      if (ok) {
+        int cc = (m[0] * sg.n[1] + m[1]) * sg.n[2] + m[2];
+        start = a.cell_start[cc];
+        len = a.cell_start[cc + 1] - start;
+        tp = ((T[0] + 64) << 14) | ((T[1] + 64) << 7) | (T[2] + 64);
+      }
+    }
+    int incl = warp_incl_scan(len);
+    cs.pre[lane] = incl - len;
+    cs.start[lane] = start;
+    cs.tpack[lane] = tp;
+    if (lane == 31) {
+      cs.pre[32] = incl;
+      cs.ncand = incl;
+      cs.fallback = incl > kCellCand;
+      cs.trunc = 0;
+    }
+  }
+  __syncthreads();
+  const int K = cs.ncand;
+  if (!cs.fallback) {
+    // stage the candidates: warp w copies stencil cells w, w + 8, ...
+    for (int sidx = warp; sidx < 32; sidx += kCellWarps) {
+      const int len = cs.pre[sidx + 1] - cs.pre[sidx];
+      if (len == 0) continue;
+      const int tp = cs.tpack[sidx];
+      const float ox = (float)(((tp >> 14) & 127) - 64) * sg.Lf[0];
+      const float oy = (float)(((tp >> 7) & 127) - 64) * sg.Lf[1];
+      const float oz = (float)((tp & 127) - 64) * sg.Lf[2];
+      for (int t = lane; t < len; t += 32) {
+        const int q = cs.start[sidx] + t;
+        float4 p = a.pos4[q];
+        p.x += ox;
+        p.y += oy;
+        p.z += oz;
+        const int dst = cs.pre[sidx] + t;
+        cs.cand[dst] = p;
+        cs.cq[dst] = q;
+        cs.ct[dst] = tp;
+      }
+    }
+  }
+  __syncthreads();
+  const int self_tp = (64 << 14) | (64 << 7) | 64;
+  unsigned long long* keys = s_keys + (size_t)warp * 2 * kFillMaxCand;
+  uint32_t st = 0;
+  for (int ci = c_lo + warp; ci < c_hi; ci += kCellWarps) {
+    const Rec rci = a.recs[ci];
+    const int i = rci.j;
+    Centre cc;
+    cc.i = i;
+    cc.x[0] = rci.x;
+    cc.x[1] = rci.y;
+    cc.x[2] = rci.z;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) cc.w[k] = unpack_w(rci.w, k);
+    cc.c[0] = cx;
+    cc.c[1] = cy;
+    cc.c[2] = cz;
+    if (cs.fallback) {
+      if (!FILL) {
+        int cnt = 0;
+        for_each_candidate(sg, a.cell_start, cc, sws[warp], [&](bool valid, int r, int tp) {
+          if (valid) {
+            double r2;
+            cnt += test_candidate(sg, cc, a.recs[r], tp, a.rc2, &r2) ? 1 : 0;
+          }
+        });
+        cnt = warp_sum(cnt);
+        if (lane == 0) {
+          a.raw[i] = cnt;
+          a.kept[i] = cnt < a.nnei_max ? cnt : a.nnei_max;
+          if (cnt > a.nnei_max) atomicAdd(&cs.trunc, 1);
+        }
+      } else {
+        const int n = a.kept[i];
+        if (n > 0)
+          st |= fill_row_global(a, sg, cc, sws[warp], keys, keys + kFillMaxCand, n, a.raw[i],
+                                a.row_ptr[i]);
+      }
+      continue;
+    }
+    const float4 pi = a.pos4[ci];
+    const int n = FILL ? a.kept[i] : 0;
+    if (FILL && n == 0) continue;
+    const bool need_d2 = FILL && a.raw[i] > n;
+    int cnt = 0;
+    for (int base = 0; base < K; base += 32) {
+      const int t = base + lane;
+      bool acc = false;
+      int tp = 0, q = 0, j = -1;
+      if (t < K) {
+        const float4 c4 = cs.cand[t];
+        const float dx = c4.x - pi.x, dy = c4.y - pi.y, dz = c4.z - pi.z;
+        const float r2f = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
+        tp = cs.ct[t];
+        j = __float_as_int(c4.w);
+        if (r2f < sg.r2lo) {
+          acc = !(j == i && tp == self_tp);
+        } else if (r2f <= sg.r2hi) {
+          double r2;
+          q = cs.cq[t];
+          acc = test_candidate(sg, cc, a.recs[q], tp, a.rc2, &r2);
+        }
+      }
+      if (!FILL) {
+        cnt += acc ? 1 : 0;
+      } else {
+        const unsigned m = __ballot_sync(kFull, acc);
+        if (acc) {
+          const int qd = cnt + __popc(m & lanemask_lt());
+          if (qd < kFillMaxCand) {
+            keys[qd] = edge_key(j, tp);
+            if (need_d2) {
+              double r2;
+              test_candidate(sg, cc, a.recs[cs.cq[t]], tp, a.rc2, &r2);
+              keys[kFillMaxCand + qd] = (unsigned long long)__double_as_longlong(r2);
+            }
+          }
+        }
+        cnt += __popc(m);
+      }
+    }
+    if (!FILL) {
+      cnt = warp_sum(cnt);
+      if (lane == 0) {
+        a.raw[i] = cnt;
+        a.kept[i] = cnt < a.nnei_max ? cnt : a.nnei_max;
+        if (cnt > a.nnei_max) atomicAdd(&cs.trunc, 1);
+      }
+    } else {
+      __syncwarp();
+      if (cnt > kFillMaxCand) {
+        // more candidates than a warp holds: threshold search from global memory
+        st |= fill_row_global(a, sg, cc, sws[warp], keys, keys + kFillMaxCand, n, cnt,
+                              a.row_ptr[i]);
+      } else {
+        st |= finish_row(a, cc, keys, keys + kFillMaxCand, n, cnt, a.row_ptr[i]);
+      }
+    }
+  }
+  if (FILL) {
+    st = __reduce_or_sync(kFull, st);
+    if (lane == 0 && st) atomicOr(a.status, st);
+  } else {
+    __syncthreads();
+    if (tid == 0 && cs.trunc)
+      atomicAdd((unsigned long long*)a.n_truncated, (unsigned long long)cs.trunc);
+  }
+}
+
+inline size_t cellscan_smem(bool fill) {
+  size_t base = ((sizeof(CellStage) + 15) / 16) * 16;
+  return base + (fill ? (size_t)kCellWarps * 2 * kFillMaxCand * sizeof(unsigned long long) : 0);
 }
 
 // ------------------------------------------------------------------ scans
@@ -687,7 +958,7 @@ __global__ void __launch_bounds__(kFillWarps * 32) k_fill(BuildArgs a) {
 constexpr int kScanThreads = 256;
 constexpr int kScanItems = 8;
 constexpr int kScanTile = kScanThreads * kScanItems;
-constexpr int kScanSingleMax = 1 << 16;
+constexpr int kScanSingleMax = 1 << 13;
 
 // exclusive block scan (blockDim.x threads, multiple of 32, <= 1024)
 template <typename T>
@@ -727,25 +998,32 @@ struct ScanTail {
   int64_t capacity;
 };
 
+// One block: tiles of 1024 x 4 items, each thread a contiguous int4, carry
+// from tile to tile.
 template <typename TOut>
 __global__ void __launch_bounds__(1024) k_scan_single(const int* in, int64_t n, TOut* out,
                                                       ScanTail tail) {
-  const int64_t per = (n + blockDim.x - 1) / blockDim.x;
-  const int64_t b = threadIdx.x * per;
-  const int64_t e = b + per < n ? b + per : n;
-  long long s = 0;
-  for (int64_t t = b; t < e; ++t) s += in[t];
-  long long tot;
-  long long off = block_excl_scan<long long>(s, &tot);
-  for (int64_t t = b; t < e; ++t) {
-    out[t] = (TOut)off;
-    off += in[t];
+  long long carry = 0;
+  for (int64_t base = 0; base < n; base += 4096) {
+    const int64_t t0 = base + 4 * (int64_t)threadIdx.x;
+    int v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = t0 + u < n ? in[t0 + u] : 0;
+    const long long s = (long long)v[0] + v[1] + v[2] + v[3];
+    long long tot;
+    long long off = block_excl_scan<long long>(s, &tot) + carry;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (t0 + u < n) out[t0 + u] = (TOut)off;
+      off += v[u];
+    }
+    carry += tot;
   }
   if (threadIdx.x == 0) {
-    out[n] = (TOut)tot;
+    out[n] = (TOut)carry;
     if (tail.n_edges) {
-      *tail.n_edges = tot;
-      if (tot > tail.capacity) atomicOr(tail.status, (uint32_t)MLG_STATUS_CAPACITY);
+      *tail.n_edges = carry;
+      if (carry > tail.capacity) atomicOr(tail.status, (uint32_t)MLG_STATUS_CAPACITY);
     }
   }
 }

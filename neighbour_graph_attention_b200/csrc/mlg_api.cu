@@ -12,6 +12,7 @@
 #include "mlg_attn.cuh"
 #include "mlg_attn_tile.cuh"
 #include "mlg_attn_hg.cuh"
+#include "mlg_attn_dmma.cuh"
 
 using namespace mlg;
 
@@ -320,17 +321,40 @@ int launch_tile(TileArgs& ta, cudaStream_t stream) {
   return launch_status();
 }
 
+// R = 40: 5 row blocks x 4 heads = 20 attention items and 60 projection
+// blocks per centre, so 10 warps share both phases evenly.
+template <int R, int NT>
+int launch_dmma(TileArgs& ta, cudaStream_t stream) {
+  using Cfg = DmmaCfg<R, NT>;
+  auto kern = k_attn_dmma<R, NT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) !=
+      cudaSuccess)
+    return MLG_ERR_CUDA;
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, Cfg::SMEM);
+  if (occ < 1) occ = 1;
+  int64_t want = (int64_t)sm_count() * occ;
+  int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
+  if (grid < 1) grid = 1;
+  kern<<<grid, NT, Cfg::SMEM, stream>>>(ta);
+  return launch_status();
+}
+
+// fp64, 32 channels, head size 8: FP64 tensor-core kernel, tile rows by nnei_max
+int dmma_rows(int nnei_max) { return nnei_max <= 40 ? 40 : 64; }
+
 // Returns the tile rows R of the fused kernel for this shape (0: none).
-int tile_rows(mlg_dtype dtype, int C, int D) {
-  if (dtype == MLG_F64 && C == 32 && D == 8) return 40;
+int tile_rows(mlg_dtype dtype, int C, int D, int nnei_max) {
+  if (dtype == MLG_F64 && C == 32 && D == 8) return dmma_rows(nnei_max);
   if (dtype == MLG_F32 && C == 32 && D == 8) return 128;
   if (dtype == MLG_F32 && C == 64 && D == 16) return 128;
   return 0;
 }
 
-int launch_tile_shape(mlg_dtype dtype, int C, int D, TileArgs& ta, cudaStream_t s) {
+int launch_tile_shape(mlg_dtype dtype, int C, int D, int nnei_max, TileArgs& ta,
+                      cudaStream_t s) {
   if (dtype == MLG_F64 && C == 32 && D == 8)
-    return launch_tile<double, 32, 8, 40, 256, 5, 3, 1>(ta, s);
+    return dmma_rows(nnei_max) == 40 ? launch_dmma<40, 320>(ta, s) : launch_dmma<64, 256>(ta, s);
   if (dtype == MLG_F32 && C == 32 && D == 8)
     return launch_tile<float, 32, 8, 128, 256, 8, 6, 2>(ta, s);
   if (dtype == MLG_F32 && C == 64 && D == 16)
@@ -402,7 +426,7 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
   if (n_layers >= 2 && pong == nullptr) return MLG_ERR_WORKSPACE;
   if (n_centres == 0) return MLG_OK;
   const int D = channels / heads;
-  int R = tile_rows(dtype, channels, D);
+  int R = tile_rows(dtype, channels, D, nnei_max);
   bool tile_ok = R > 0 && n_layers <= kMaxFusedLayers && aligned16(G_in) && aligned16(G_out);
   for (int k = 0; tile_ok && k < 3 * n_layers; ++k) tile_ok = aligned16(W[k]);
   int min_n = 0;  // generic path: centres with more than min_n edges
@@ -418,7 +442,7 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
     ta.out = G_out;
     for (int k = 0; k < 3 * n_layers; ++k) ta.W[k] = W[k];
     ta.status = csr->status;
-    rc = launch_tile_shape(dtype, channels, D, ta, stream);
+    rc = launch_tile_shape(dtype, channels, D, nnei_max, ta, stream);
     if (rc != MLG_OK) return rc;
     if (nnei_max <= R) return MLG_OK;  // no centre can exceed the tile
     min_n = R;
@@ -460,7 +484,7 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
 int forward_launches(int64_t n_atoms, int32_t nnei_max, int32_t channels, int32_t heads,
                      int32_t n_layers, mlg_dtype dtype) {
   const int D = heads > 0 ? channels / heads : 0;
-  int R = tile_rows(dtype, channels, D);
+  int R = tile_rows(dtype, channels, D, nnei_max);
   if (R > 0 && n_layers <= kMaxFusedLayers) return 1 + (nnei_max > R ? n_layers : 0);
   int Rg = hg_rows(dtype, channels, D);
   if (Rg > 0) return n_layers * (1 + (nnei_max > Rg ? 1 : 0));

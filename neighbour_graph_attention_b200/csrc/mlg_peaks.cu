@@ -4,6 +4,7 @@
 //   m8n8k4 and m16n8k16), and the special-function pipe (ex2.approx.f32).
 // Each kernel runs independent dependency chains per thread so that the pipe,
 // not latency, limits it; results feed a global store so nothing is removed.
+#include <cstdint>
 #include <cstdio>
 #include <cuda_runtime.h>
 
@@ -95,6 +96,62 @@ __global__ void k_dmma16816(double* out, int iters) {
   if (s == -1.0) out[blockIdx.x] = s;
 }
 
+__global__ void k_tf32_16816(float* out, int iters) {
+  uint32_t a[4], b[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] = __float_as_uint(1.0f + (threadIdx.x + i) * 1e-6f);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) b[i] = __float_as_uint(0.5f);
+  float c[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[j][i] = 0.f;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      asm volatile(
+          "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+          "{%8,%9}, {%0,%1,%2,%3};"
+          : "+f"(c[j][0]), "+f"(c[j][1]), "+f"(c[j][2]), "+f"(c[j][3])
+          : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s += c[j][i];
+  if (s == -1.f) out[blockIdx.x] = s;
+}
+
+__global__ void k_bf16_16816(float* out, int iters) {
+  uint32_t a[4], b[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] = 0x3f803f80u + threadIdx.x;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) b[i] = 0x3f003f00u;
+  float c[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[j][i] = 0.f;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      asm volatile(
+          "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+          "{%8,%9}, {%0,%1,%2,%3};"
+          : "+f"(c[j][0]), "+f"(c[j][1]), "+f"(c[j][2]), "+f"(c[j][3])
+          : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s += c[j][i];
+  if (s == -1.f) out[blockIdx.x] = s;
+}
+
 template <class F>
 float time_ms(F launch) {
   cudaEvent_t a, b;
@@ -140,11 +197,16 @@ int main() {
   double dmma884 = warps * (iters / 4) * 16 * (2.0 * 8 * 8 * 4) / (t * 1e-3) / 1e12;
   t = time_ms([&] { k_dmma16816<<<blocks, threads>>>(dbuf, iters / 16); });
   double dmma16816 = warps * (iters / 16) * 4 * (2.0 * 16 * 8 * 16) / (t * 1e-3) / 1e12;
+  t = time_ms([&] { k_tf32_16816<<<blocks, threads>>>(fbuf, iters / 4); });
+  double tf32 = warps * (iters / 4) * 4 * (2.0 * 16 * 8 * 8) / (t * 1e-3) / 1e12;
+  t = time_ms([&] { k_bf16_16816<<<blocks, threads>>>(fbuf, iters / 4); });
+  double bf16 = warps * (iters / 4) * 4 * (2.0 * 16 * 8 * 16) / (t * 1e-3) / 1e12;
   cudaError_t e = cudaGetLastError();
   printf("{\"sm_count\": %d, \"clock_khz_attr\": %d, \"fp64_fma_tflops\": %.3f, "
          "\"fp32_fma_tflops\": %.3f, \"ex2_tops\": %.4f, \"dmma_m8n8k4_tflops\": %.3f, "
-         "\"dmma_m16n8k16_tflops\": %.3f, \"cuda\": \"%s\"}\n",
-         sms, clk, dfma, ffma, ex2, dmma884, dmma16816, cudaGetErrorString(e));
+         "\"dmma_m16n8k16_tflops\": %.3f, \"mma_sync_tf32_m16n8k8_tflops\": %.3f, "
+         "\"mma_sync_bf16_m16n8k16_tflops\": %.3f, \"cuda\": \"%s\"}\n",
+         sms, clk, dfma, ffma, ex2, dmma884, dmma16816, tf32, bf16, cudaGetErrorString(e));
   cudaFree(dbuf);
   cudaFree(fbuf);
   return e == cudaSuccess ? 0 : 1;

@@ -7,6 +7,9 @@ destination into the destination CSR (NeighborGraph issue, Proposed fix), with
 the per-centre cap sel / nnei_max (DPA4 issue, Reproduction; NeighborGraph
 issue, Measurements).
 """
+import json
+import os
+
 import numpy as np
 import pytest
 from scipy.spatial import cKDTree
@@ -21,11 +24,11 @@ def _rows(csr):
 
 # ---------------------------------------------------------------- lattices
 
-# shells of the ideal lattices as {d^2 in units of a^2/16 : multiplicity}
-DIAMOND_SHELLS = {3: 4, 8: 12, 11: 12, 16: 6, 19: 12, 24: 24, 27: 16, 32: 12, 35: 24,
-                  40: 24, 43: 12, 48: 8}
-# {d^2 in units of a^2/4 : multiplicity}
-BCC_SHELLS = {3: 8, 4: 6, 8: 12, 11: 24, 12: 8, 16: 6, 19: 24}
+# shells of the ideal lattices {d^2 in units of a^2/16 (diamond) or a^2/4 (BCC) : sites},
+# from tests/golden/lattice_shells.json
+_GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "lattice_shells.json")))
+DIAMOND_SHELLS = {int(k): v for k, v in _GOLDEN["diamond"]["shells"].items()}
+BCC_SHELLS = {int(k): v for k, v in _GOLDEN["bcc"]["shells"].items()}
 
 
 def _shell_hist(d, a, unit):

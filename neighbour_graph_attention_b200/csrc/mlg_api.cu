@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cstring>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "mlg.h"
@@ -13,6 +14,7 @@
 #include "mlg_attn_tile.cuh"
 #include "mlg_attn_hg.cuh"
 #include "mlg_attn_dmma.cuh"
+#include "mlg_attn_tc.cuh"
 
 using namespace mlg;
 
@@ -135,6 +137,15 @@ void taylor_coeffs(double* c) {
   for (int k = 1; k < 12; ++k) c[k] = -c[k - 1] / (double)((2 * k) * (2 * k + 1));
 }
 
+// Ask for the largest shared-memory carveout, so that the occupancy the
+// shared memory allows is the occupancy the launch gets.
+template <typename K>
+void prefer_shared(K kern, size_t smem) {
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                       (int)cudaSharedmemCarveoutMaxShared);
+}
+
 int launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MLG_OK : MLG_ERR_CUDA;
@@ -238,10 +249,8 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   const bool per_cell = plan.max_reach <= 1 && plan.ncell_cap >= 4 * sm_count();
   if (per_cell) {
     const size_t sm_count_ = cellscan_smem(false), sm_fill = cellscan_smem(true);
-    cudaFuncSetAttribute(k_cellscan<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)sm_count_);
-    cudaFuncSetAttribute(k_cellscan<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)sm_fill);
+    prefer_shared(k_cellscan<false>, sm_count_);
+    prefer_shared(k_cellscan<true>, sm_fill);
     k_cellscan<false><<<plan.ncell_cap, kCellWarps * 32, sm_count_, stream>>>(a);
   } else {
     k_count<<<(int)((n + kCountWarps - 1) / kCountWarps), kCountWarps * 32, 0, stream>>>(a);
@@ -327,9 +336,8 @@ template <int R, int NT>
 int launch_dmma(TileArgs& ta, cudaStream_t stream) {
   using Cfg = DmmaCfg<R, NT>;
   auto kern = k_attn_dmma<R, NT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) !=
-      cudaSuccess)
-    return MLG_ERR_CUDA;
+  prefer_shared(kern, Cfg::SMEM);
+  if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
   int occ = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, Cfg::SMEM);
   if (occ < 1) occ = 1;
@@ -337,6 +345,75 @@ int launch_dmma(TileArgs& ta, cudaStream_t stream) {
   int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
   if (grid < 1) grid = 1;
   kern<<<grid, NT, Cfg::SMEM, stream>>>(ta);
+  return launch_status();
+}
+
+// Blocks of `kern` that fit on one SM by registers, shared memory, warps.
+template <typename K>
+int resident_blocks(K kern, int nt, size_t dyn_smem) {
+  cudaFuncAttributes fa;
+  int dev = 0, regs_sm = 65536, smem_sm = 233472, reserved = 1024, thr_sm = 2048;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
+  const int regs_warp = ((fa.numRegs * 32 + 255) / 256) * 256;
+  int by_regs = regs_sm / (regs_warp * (nt / 32));
+  int by_smem = (int)(smem_sm / (dyn_smem + fa.sharedSizeBytes + reserved));
+  int by_thr = thr_sm / nt;
+  int b = by_regs < by_smem ? by_regs : by_smem;
+  b = b < by_thr ? b : by_thr;
+  return b < 1 ? 1 : b;
+}
+
+// A 2-D tensor map over G [rows][C] fp32 with a {4 x 128} box (16-byte inner
+// extent), for the tcgen05 kernel's slab loads.  Encoded on the host per call
+// (no device work, no allocation).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool encode_slab_map(CUtensorMap* map, const void* G, int64_t rows, int C) {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr)
+      return false;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)(rows > 0 ? rows : 1)};
+  const cuuint64_t strides[1] = {(cuuint64_t)C * 4};
+  const cuuint32_t box[2] = {4, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(G), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32, 32 or 64 channels: projection on tcgen05 (3xTF32), tiles of 128 rows.
+// TMEM columns per CTA: 128 (c = 32) or 256 (c = 64); the grid keeps the
+// resident CTAs within the 512 columns of an SM.
+template <int C, int D, int NT>
+int launch_tc(TileArgs& ta, cudaStream_t stream) {
+  using Cfg = TcCfg<C, D, NT>;
+  auto kern = k_attn_tc<C, D, NT>;
+  prefer_shared(kern, Cfg::SMEM);
+  if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
+  CUtensorMap map;
+  if (!encode_slab_map(&map, ta.G, ta.capacity, C)) return MLG_ERR_CUDA;
+  int occ = resident_blocks(kern, NT, Cfg::SMEM);
+  const int tmem_cap = 512 / Cfg::NCOL;
+  if (occ > tmem_cap) occ = tmem_cap;
+  int64_t want = (int64_t)sm_count() * occ;
+  int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
+  if (grid < 1) grid = 1;
+  kern<<<grid, NT, Cfg::SMEM, stream>>>(ta, map);
   return launch_status();
 }
 
@@ -355,10 +432,8 @@ int launch_tile_shape(mlg_dtype dtype, int C, int D, int nnei_max, TileArgs& ta,
                       cudaStream_t s) {
   if (dtype == MLG_F64 && C == 32 && D == 8)
     return dmma_rows(nnei_max) == 40 ? launch_dmma<40, 320>(ta, s) : launch_dmma<64, 256>(ta, s);
-  if (dtype == MLG_F32 && C == 32 && D == 8)
-    return launch_tile<float, 32, 8, 128, 256, 8, 6, 2>(ta, s);
-  if (dtype == MLG_F32 && C == 64 && D == 16)
-    return launch_tile<float, 64, 16, 128, 512, 8, 6, 2>(ta, s);
+  if (dtype == MLG_F32 && C == 32 && D == 8) return launch_tc<32, 8, 512>(ta, s);
+  if (dtype == MLG_F32 && C == 64 && D == 16) return launch_tc<64, 16, 512>(ta, s);
   return MLG_ERR_UNSUPPORTED;
 }
 
@@ -367,9 +442,8 @@ template <typename T, int C, int D, int HG, int R, int NT, int TM, int TN, int K
 int launch_hg(HgArgs& ha, cudaStream_t stream) {
   using Cfg = HgCfg<T, C, D, HG, R, NT, TM, TN, KC>;
   auto kern = k_attn_hg<T, C, D, HG, R, NT, TM, TN, KC>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) !=
-      cudaSuccess)
-    return MLG_ERR_CUDA;
+  prefer_shared(kern, Cfg::SMEM);
+  if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
   int occ = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, Cfg::SMEM);
   if (occ < 1) occ = 1;

@@ -215,70 +215,8 @@ __global__ void __launch_bounds__(NT) k_attn_hg(HgArgs a) {
     }
     __syncthreads();
 
-    // ---- 2. attention of the group's heads
-    const int ntask = meta.task0[0][ncent];
-    for (int task = warp; task < ntask; task += NT / 32) {
-      int ci = 0;
-      while (meta.task0[0][ci + 1] <= task) ++ci;
-      const int base = meta.off[0][ci];
-      const int n = meta.off[0][ci + 1] - base;
-      const int p = (task - meta.task0[0][ci]) * 32 + lane;
-      const bool valid = p < n * HG;
-      const int h = valid ? p / n : 0;
-      const int row = valid ? p - h * n : 0;
-      T q[D], o[D];
-      const T* qrow = sQ + (base + row) * QS + h * D;
-#pragma unroll
-      for (int t = 0; t < D; ++t) {
-        q[t] = qrow[t];
-        o[t] = T(0);
-      }
-      T mx = T(-INFINITY), l = T(0);
-      const T* kb = sQ + base * QS + GW + h * D;
-      const T* vb = sQ + base * QS + 2 * GW + h * D;
-      for (int b0 = 0; b0 < n; b0 += 8) {
-        T s[8];
-        T bm = T(-INFINITY);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int b = b0 + j;
-          T dot = T(0);
-          if (b < n) {
-            const T* kr = kb + b * QS;
-#pragma unroll
-            for (int t = 0; t < D; ++t) dot = fma(q[t], kr[t], dot);
-          } else {
-            dot = T(-INFINITY);
-          }
-          s[j] = dot;
-          bm = bm > dot ? bm : dot;
-        }
-        if (bm > mx) {
-          const T sc = softmax_exp<T>(mx - bm);
-          l *= sc;
-#pragma unroll
-          for (int t = 0; t < D; ++t) o[t] *= sc;
-          mx = bm;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int b = b0 + j;
-          if (b < n) {
-            const T pj = softmax_exp<T>(s[j] - mx);
-            l += pj;
-            const T* vr = vb + b * QS;
-#pragma unroll
-            for (int t = 0; t < D; ++t) o[t] = fma(pj, vr[t], o[t]);
-          }
-        }
-      }
-      if (valid) {
-        const T rl = T(1) / l;
-        T* qo = sQ + (base + row) * QS + h * D;   // this lane's own q slot
-#pragma unroll
-        for (int t = 0; t < D; ++t) qo[t] = o[t] * rl;
-      }
-    }
+    // ---- 2. attention of the group's heads (outputs into the q slots)
+    tile_attention<T, HG, D, GW, NT, QS>(sQ, meta, 0, warp, lane);
     __syncthreads();
     // ---- 3. the group's output columns, row by row (coalesced segments)
     constexpr int OV = GW * (int)sizeof(T) / 16;

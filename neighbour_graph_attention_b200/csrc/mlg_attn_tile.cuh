@@ -164,6 +164,115 @@ struct TileCfg {
 
 
 
+// One key block of the running-max softmax for one lane (query row, head):
+// logits of keys [b0, b0 + 8) (masked to -inf at and beyond n when TAIL),
+// rescale of the running sum and output when the block raises the maximum,
+// then accumulation of exp(l - max) v.  fp32 logits are in log2 units (q
+// carries log2 e), fp64 ones in natural units.
+template <typename T, int D, bool TAIL>
+__device__ __forceinline__ void softmax_block(const T* q, T* o, T& mx, T& l, const T* kb,
+                                              const T* vb, int b0, int n, int QS) {
+  T s[8];
+  T bm = T(-INFINITY);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int b = b0 + j;
+    T acc = T(0);
+    if (!TAIL || b < n) {
+      const T* kr = kb + b * QS;
+      if constexpr (sizeof(T) == 4 && D % 2 == 0) {
+        float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < D; t += 2)
+          a2 = __ffma2_rn(make_float2(q[t], q[t + 1]),
+                          *reinterpret_cast<const float2*>(kr + t), a2);
+        acc = a2.x + a2.y;
+      } else {
+#pragma unroll
+        for (int t = 0; t < D; ++t) acc = fma(q[t], kr[t], acc);
+      }
+    } else {
+      acc = T(-INFINITY);
+    }
+    s[j] = acc;
+    bm = bm > acc ? bm : acc;
+  }
+  if (bm > mx) {
+    const T sc = softmax_exp<T>(mx - bm);  // exp(-inf) = 0 on the first block
+    l *= sc;
+#pragma unroll
+    for (int t = 0; t < D; ++t) o[t] *= sc;
+    mx = bm;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int b = b0 + j;
+    if (!TAIL || b < n) {
+      const T pj = softmax_exp<T>(s[j] - mx);
+      l += pj;
+      const T* vr = vb + b * QS;
+      if constexpr (sizeof(T) == 4 && D % 2 == 0) {
+        const float2 p2 = make_float2(pj, pj);
+#pragma unroll
+        for (int t = 0; t < D; t += 2) {
+          float2 o2 = __ffma2_rn(p2, *reinterpret_cast<const float2*>(vr + t),
+                                 make_float2(o[t], o[t + 1]));
+          o[t] = o2.x;
+          o[t + 1] = o2.y;
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < D; ++t) o[t] = fma(pj, vr[t], o[t]);
+      }
+    }
+  }
+}
+
+// Attention of one tile from its QKV rows in shared memory [rows][QS]: head h
+// of the HEADS handled here has q at column h d, k at KOFF + h d and v at
+// 2 KOFF + h d; q carries s_a / sqrt(d) (times log2 e in fp32), k carries s_b.
+// Warp tasks: 32 consecutive (head, row) pairs of one centre; lanes of a warp
+// walk the keys in lock-step, so k_b and v_b are broadcast reads.  The output
+// of (row, h) overwrites the q slot that only its own lane read.
+template <typename T, int HEADS, int D, int KOFF, int NT, int QS>
+__device__ __forceinline__ void tile_attention(T* sQ, const TileMeta& meta, int buf, int warp,
+                                               int lane) {
+  const int ncent = meta.ncent[buf];
+  const int ntask = meta.task0[buf][ncent];
+  for (int task = warp; task < ntask; task += NT / 32) {
+    int ci = 0;
+    while (meta.task0[buf][ci + 1] <= task) ++ci;
+    const int base = meta.off[buf][ci];
+    const int n = meta.off[buf][ci + 1] - base;
+    const int p = (task - meta.task0[buf][ci]) * 32 + lane;
+    const bool valid = p < n * HEADS;
+    const int h = valid ? p / n : 0;
+    const int row = valid ? p - h * n : 0;
+    T q[D], o[D];
+    const T* qrow = sQ + (base + row) * QS + h * D;
+#pragma unroll
+    for (int t = 0; t < D; ++t) {
+      q[t] = qrow[t];
+      o[t] = T(0);
+    }
+    T mx = T(-INFINITY), l = T(0);
+    const T* kb = sQ + base * QS + KOFF + h * D;
+    const T* vb = sQ + base * QS + 2 * KOFF + h * D;
+    const int nfull = n & ~7;
+    for (int b0 = 0; b0 < nfull; b0 += 8)
+      softmax_block<T, D, false>(q, o, mx, l, kb, vb, b0, n, QS);
+    if (nfull < n) softmax_block<T, D, true>(q, o, mx, l, kb, vb, nfull, n, QS);
+    if (valid) {
+      // this lane alone read the q slot of (row, h): reuse it for the output
+      // (the padded QKV stride spreads rows over banks; X's stride would not)
+      const T rl = T(1) / l;
+      T* qo = sQ + (base + row) * QS + h * D;
+#pragma unroll
+      for (int t = 0; t < D; ++t) qo[t] = o[t] * rl;
+    }
+  }
+}
+
 template <typename T, int C, int D, int R, int NT, int TM, int TN, int XB>
 __global__ void __launch_bounds__(NT) k_attn_tile(TileArgs a) {
   using Cfg = TileCfg<T, C, D, R, NT, TM, TN, XB>;
@@ -344,71 +453,7 @@ __global__ void __launch_bounds__(NT) k_attn_tile(TileArgs a) {
       if (a.n_layers > 1) weights_pending = more;
 
       // ---- 2. attention: warp tasks of 32 (head, row) pairs of one centre
-      const int ntask = meta.task0[buf][ncent];
-      for (int task = warp; task < ntask; task += NT / 32) {
-        int ci = 0;
-        while (meta.task0[buf][ci + 1] <= task) ++ci;
-        const int base = meta.off[buf][ci];
-        const int n = meta.off[buf][ci + 1] - base;
-        const int p = (task - meta.task0[buf][ci]) * 32 + lane;
-        const bool valid = p < n * H;
-        const int h = valid ? p / n : 0;
-        const int row = valid ? p - h * n : 0;
-        T q[D], o[D];
-        const T* qrow = sQ + (base + row) * QS + h * D;
-#pragma unroll
-        for (int t = 0; t < D; ++t) {
-          q[t] = qrow[t];
-          o[t] = T(0);
-        }
-        T mx = T(-INFINITY), l = T(0);
-        const T* kb = sQ + base * QS + C + h * D;
-        const T* vb = sQ + base * QS + 2 * C + h * D;
-        for (int b0 = 0; b0 < n; b0 += 8) {
-          T s[8];
-          T bm = T(-INFINITY);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int b = b0 + j;
-            T acc = T(0);
-            if (b < n) {
-              const T* kr = kb + b * QS;
-#pragma unroll
-              for (int t = 0; t < D; ++t) acc = fma(q[t], kr[t], acc);
-            } else {
-              acc = T(-INFINITY);
-            }
-            s[j] = acc;
-            bm = bm > acc ? bm : acc;
-          }
-          if (bm > mx) {
-            const T sc = softmax_exp<T>(mx - bm);  // exp(-inf) = 0 on the first block
-            l *= sc;
-#pragma unroll
-            for (int t = 0; t < D; ++t) o[t] *= sc;
-            mx = bm;
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int b = b0 + j;
-            if (b < n) {
-              const T pj = softmax_exp<T>(s[j] - mx);
-              l += pj;
-              const T* vr = vb + b * QS;
-#pragma unroll
-              for (int t = 0; t < D; ++t) o[t] = fma(pj, vr[t], o[t]);
-            }
-          }
-        }
-        if (valid) {
-          // this lane alone read the q slot of (row, h): reuse it for the output
-          // (the padded QKV stride spreads rows over banks; X's stride would not)
-          const T rl = T(1) / l;
-          T* qo = sQ + (base + row) * QS + h * D;
-#pragma unroll
-          for (int t = 0; t < D; ++t) qo[t] = o[t] * rl;
-        }
-      }
+      tile_attention<T, C / D, D, C, NT, QS>(sQ, meta, buf, warp, lane);
       __syncthreads();
       for (int e = tid; e < rows * C; e += NT) {
         const int r = e / C, col = e - r * C;

@@ -91,6 +91,25 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(x: float, device) -> float:
+    """The max of x over the ranks of the default process group (x alone at N = 1)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, n_atoms: int, steps: int, total_ms: float) -> float:
+    """Atoms per second of N independent replicas timed by the slowest rank."""
+    return world * n_atoms * steps / (total_ms / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -404,13 +423,9 @@ def main(argv=None):
     sampler.stop()
     build_ms_steps = [p[0] for p in parts]
     attn_ms_steps = [p[1] for p in parts]
-    total_ms = float(sum(build_ms_steps) + sum(attn_ms_steps))
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(float(sum(build_ms_steps) + sum(attn_ms_steps)), dev)
     ms_per_step = total_ms / args.steps
-    value = world * w.n_atoms * args.steps / (total_ms / 1e3)
+    value = replica_throughput(world, w.n_atoms, args.steps, total_ms)
 
     status = int(csr.status.item())
     if status != 0:
@@ -457,12 +472,8 @@ def main(argv=None):
 
     timed_loop(e2e_step, 3)
     e2e_ms = timed_loop(e2e_step, args.steps)
-    e2e_total = float(sum(e2e_ms))
-    if world > 1:
-        tt = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_total = float(tt.item())
-    e2e_value = world * w.n_atoms * args.steps / (e2e_total / 1e3)
+    e2e_total = max_over_ranks(float(sum(e2e_ms)), dev)
+    e2e_value = replica_throughput(world, w.n_atoms, args.steps, e2e_total)
     h2d = x_h.numel() * x_h.element_size() + g_h.numel() * g_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
 

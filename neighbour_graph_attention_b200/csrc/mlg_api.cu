@@ -244,21 +244,24 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
                    ScanTail{nullptr, nullptr, 0}, stream);
   k_scatter<<<atom_blocks, tb, 0, stream>>>(a);
   // per-cell scans when every stencil reach is 1 (at most 27 stencil cells);
-  // otherwise (boxes narrower than the cutoff) the per-centre scans
-  // (a grid of few cells would leave most SMs idle: per-centre scans there)
-  const bool per_cell = plan.max_reach <= 1 && plan.ncell_cap >= 4 * sm_count();
+  // otherwise (boxes narrower than the cutoff) the per-centre scans.  A grid
+  // of few cells splits each cell's centres over several CTAs.
+  const bool per_cell = plan.max_reach <= 1;
+  int nsplit = (4 * sm_count() + plan.ncell_cap - 1) / plan.ncell_cap;
+  nsplit = nsplit < 1 ? 1 : (nsplit > 8 ? 8 : nsplit);
+  const dim3 cell_grid((unsigned)plan.ncell_cap, (unsigned)nsplit);
   if (per_cell) {
     const size_t sm_count_ = cellscan_smem(false), sm_fill = cellscan_smem(true);
     prefer_shared(k_cellscan<false>, sm_count_);
     prefer_shared(k_cellscan<true>, sm_fill);
-    k_cellscan<false><<<plan.ncell_cap, kCellWarps * 32, sm_count_, stream>>>(a);
+    k_cellscan<false><<<cell_grid, kCellWarps * 32, sm_count_, stream>>>(a);
   } else {
     k_count<<<(int)((n + kCountWarps - 1) / kCountWarps), kCountWarps * 32, 0, stream>>>(a);
   }
   launch_scan<long long>(a.kept, n, reinterpret_cast<long long*>(a.row_ptr), a.partial,
                          ScanTail{a.n_edges, a.status, a.capacity}, stream);
   if (per_cell) {
-    k_cellscan<true><<<plan.ncell_cap, kCellWarps * 32, cellscan_smem(true), stream>>>(a);
+    k_cellscan<true><<<cell_grid, kCellWarps * 32, cellscan_smem(true), stream>>>(a);
   } else {
     const size_t fill_smem = (size_t)kFillWarps * 2 * kFillMaxCand * sizeof(unsigned long long);
     k_fill<<<(int)((n + kFillWarps - 1) / kFillWarps), kFillWarps * 32, fill_smem, stream>>>(a);

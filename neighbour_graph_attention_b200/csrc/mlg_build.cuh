@@ -764,10 +764,11 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2) k_cellscan(BuildArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) sg = *a.grid;
   __syncthreads();
+  // blockIdx.y splits a cell's centres over several CTAs (small grids)
   const int cell = blockIdx.x;
   if (cell >= sg.ncell) return;
   const int c_lo = a.cell_start[cell], c_hi = a.cell_start[cell + 1];
-  if (c_lo == c_hi) return;
+  if (c_lo + (int)blockIdx.y * kCellWarps >= c_hi) return;
   const int cz = cell % sg.n[2], cy = (cell / sg.n[2]) % sg.n[1], cx = cell / (sg.n[2] * sg.n[1]);
   if (warp == 0) {
     // stencil (reach <= 1 on every axis: at most 27 cells)
@@ -840,7 +841,8 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2) k_cellscan(BuildArgs a) {
   const int self_tp = (64 << 14) | (64 << 7) | 64;
   unsigned long long* keys = s_keys + (size_t)warp * 2 * kFillMaxCand;
   uint32_t st = 0;
-  for (int ci = c_lo + warp; ci < c_hi; ci += kCellWarps) {
+  for (int ci = c_lo + blockIdx.y * kCellWarps + warp; ci < c_hi;
+       ci += gridDim.y * kCellWarps) {
     const Rec rci = a.recs[ci];
     const int i = rci.j;
     Centre cc;

@@ -139,22 +139,29 @@ __global__ void __launch_bounds__(NT) k_attn_dmma(TileArgs a) {
       cp_async_wait<0>();
       __syncthreads();
 
-      // ---- projection: 8x8 output blocks (row block, column block) over the warps
+      // ---- projection: pairs of 8x8 output blocks (row block, two adjacent
+      // column blocks) over the warps; the pair shares the A fragment and
+      // gives two independent accumulator chains
       const int nrb = prow / 8;
-      for (int item = warp; item < nrb * 12; item += NW) {
-        const int mb = item / 12, nb = item - mb * 12;
-        double c0v = 0.0, c1v = 0.0;
+      for (int item = warp; item < nrb * 6; item += NW) {
+        const int mb = item / 6, nb = (item - mb * 6) * 2;
+        double c0v = 0.0, c1v = 0.0, c2v = 0.0, c3v = 0.0;
 #pragma unroll
         for (int k = 0; k < C / 4; ++k) {
           const double av = sX[(mb * 8 + lr) * XS + k * 4 + lc];
-          const double bv = sW[(k * 4 + lc) * WS + nb * 8 + lr];
-          dmma884(c0v, c1v, av, bv);
+          const double bv0 = sW[(k * 4 + lc) * WS + nb * 8 + lr];
+          const double bv1 = sW[(k * 4 + lc) * WS + nb * 8 + 8 + lr];
+          dmma884(c0v, c1v, av, bv0);
+          dmma884(c2v, c3v, av, bv1);
         }
         const int r = mb * 8 + lr, col = nb * 8 + 2 * lc;
         const double s = sS[r];
+        // the two blocks never straddle q / k / v (32 is a multiple of 16)
         const double f = col < C ? s * rsd : (col < 2 * C ? s : 1.0);
         sQ[r * QS + col] = c0v * f;
         sQ[r * QS + col + 1] = c1v * f;
+        sQ[r * QS + col + 8] = c2v * f;
+        sQ[r * QS + col + 9] = c3v * f;
       }
       __syncthreads();
       if (layer + 1 < a.n_layers) load_weights(layer + 1);
@@ -213,20 +220,24 @@ __global__ void __launch_bounds__(NT) k_attn_dmma(TileArgs a) {
         sum += __shfl_xor_sync(kFull, sum, 2);
         // O = P V: the A operand (row lr, key 4 kk + lc) sits in lane
         // (lr, (kk & 1) * 2 + lc / 2), element lc & 1, of accumulator kk / 2
-        double o0 = 0.0, o1 = 0.0;
+        // two accumulator chains (even / odd key steps), summed at the end
+        double o0 = 0.0, o1 = 0.0, o2 = 0.0, o3 = 0.0;
         const int src_lo = (lane & ~3) | (lc >> 1), src_hi = src_lo | 2;
 #pragma unroll
-        for (int kk = 0; kk < 2 * NB; ++kk) {
-          const int j = kk >> 1;
+        for (int j = 0; j < NB; ++j) {
           if (j < nbk) {
-            const int src = (kk & 1) ? src_hi : src_lo;
-            const double v0 = __shfl_sync(kFull, s[j][0], src);
-            const double v1 = __shfl_sync(kFull, s[j][1], src);
-            const double av = (lc & 1) ? v1 : v0;
-            const double bv = sQ[(off + kk * 4 + lc) * QS + 2 * C + h * D + lr];
-            dmma884(o0, o1, av, bv);
+            const double w0 = __shfl_sync(kFull, s[j][0], src_lo);
+            const double w1 = __shfl_sync(kFull, s[j][1], src_lo);
+            const double x0 = __shfl_sync(kFull, s[j][0], src_hi);
+            const double x1 = __shfl_sync(kFull, s[j][1], src_hi);
+            const double bv0 = sQ[(off + (2 * j) * 4 + lc) * QS + 2 * C + h * D + lr];
+            const double bv1 = sQ[(off + (2 * j + 1) * 4 + lc) * QS + 2 * C + h * D + lr];
+            dmma884(o0, o1, (lc & 1) ? w1 : w0, bv0);
+            dmma884(o2, o3, (lc & 1) ? x1 : x0, bv1);
           }
         }
+        o0 += o2;
+        o1 += o3;
         const double inv = 1.0 / sum;
         const int r = ib * 8 + lr;
         if (r < n) {

@@ -117,7 +117,11 @@ struct TcCfg {
   static constexpr size_t OFF_AHI = OFF_REG;                 // inside the QKV region
   static constexpr size_t OFF_ALO = OFF_AHI + A_BYTES;
   static constexpr size_t OFF_X = OFF_ALO + A_BYTES;
-  static constexpr size_t OFF_S = OFF_REG + (REG_BYTES + 15) / 16 * 16;
+  // a slab buffer of its own (prefetched during the previous tile) when the
+  // shared memory allows two CTAs per SM with it
+  static constexpr bool PREFETCH = (C <= 32);
+  static constexpr size_t OFF_XP = OFF_REG + (REG_BYTES + 1023) / 1024 * 1024;
+  static constexpr size_t OFF_S = PREFETCH ? OFF_XP + X_BYTES : OFF_REG + (REG_BYTES + 15) / 16 * 16;
   static constexpr size_t OFF_META = OFF_S + (size_t)R * 4;
   static constexpr size_t OFF_BAR = (OFF_META + sizeof(TileMeta) + 15) / 16 * 16;
   static constexpr size_t SMEM = OFF_BAR + 32;
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
   float* sQ = reinterpret_cast<float*>(smem + Cfg::OFF_REG);
   char* sAhi = reinterpret_cast<char*>(smem + Cfg::OFF_AHI);
   char* sAlo = reinterpret_cast<char*>(smem + Cfg::OFF_ALO);
-  float* sX = reinterpret_cast<float*>(smem + Cfg::OFF_X);
+  float* sX = reinterpret_cast<float*>(smem + (Cfg::PREFETCH ? Cfg::OFF_XP : Cfg::OFF_X));
   float* sS = reinterpret_cast<float*>(smem + Cfg::OFF_S);
   TileMeta& meta = *reinterpret_cast<TileMeta*>(smem + Cfg::OFF_META);
   uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
@@ -181,9 +185,8 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
   uint32_t ph_x = 0u, ph_mma = 0u;
   int loaded_layer = -1;
 
-  while (true) {
-    // ---- plan the tile and start its slab copy (thread 0)
-    if (tid == 0) {
+  // thread 0: plan the next tile into meta slot b and start its slab copy
+  auto plan_and_load = [&](int b) {
       int c = meta.next_c, k = 0, rows = 0, tasks = 0;
       const int c_end = meta.c_end;
       while (c < c_end) {
@@ -191,36 +194,40 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
         if (n > 0 && n <= R) break;
         ++c;
       }
-      meta.row0[0] = c < c_end ? a.row_ptr[c] : 0;
+      meta.row0[b] = c < c_end ? a.row_ptr[c] : 0;
       while (c < c_end && k < 64) {
         const int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
         if (n > R || rows + n > R) break;
-        meta.off[0][k] = rows;
-        meta.task0[0][k] = tasks;
+        meta.off[b][k] = rows;
+        meta.task0[b][k] = tasks;
         tasks += (n * H + 31) / 32;
         rows += n;
         ++k;
         ++c;
       }
-      meta.off[0][k] = rows;
-      meta.task0[0][k] = tasks;
-      meta.ncent[0] = k;
-      meta.nrows[0] = rows;
+      meta.off[b][k] = rows;
+      meta.task0[b][k] = tasks;
+      meta.ncent[b] = k;
+      meta.nrows[b] = rows;
       meta.next_c = c;
       if (rows > 0) {
         // C / 4 tensor loads of {4 columns x 128 rows}: each lands as one
         // K-chunk column of 8-row x 16-byte core matrices (the K-major layout)
         fence_proxy_async();
         mbar_expect_tx(bar_x, (uint32_t)(R * C * 4));
-        for (int c = 0; c < C / 4; ++c)
-          tma_load_2d(reinterpret_cast<char*>(sX) + c * R * 16, &gmap, 4 * c,
-                      (int)meta.row0[0], bar_x);
-        if (!mbar_wait(bar_x, ph_x)) meta.fail = 1;
+        for (int cc = 0; cc < C / 4; ++cc)
+          tma_load_2d(reinterpret_cast<char*>(sX) + cc * R * 16, &gmap, 4 * cc,
+                      (int)meta.row0[b], bar_x);
       }
-    }
+  };
+
+  int cur = 0;
+  if (tid == 0) plan_and_load(0);
+  while (true) {
+    if (tid == 0 && meta.nrows[cur] > 0 && !mbar_wait(bar_x, ph_x)) meta.fail = 1;
     __syncthreads();
-    const int rows = meta.nrows[0];
-    const int64_t row0 = meta.row0[0];
+    const int rows = meta.nrows[cur];
+    const int64_t row0 = meta.row0[cur];
     if (rows == 0 || meta.fail) break;
     ph_x ^= 1u;
     for (int t = tid; t < rows; t += NT) sS[t] = (float)a.sw[row0 + t];
@@ -266,6 +273,9 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
       fence_proxy_async();
       tc_fence_before();
       __syncthreads();
+      // the slab buffer is free: with its own buffer, the next tile's copy
+      // starts now and lands while this tile computes
+      if (Cfg::PREFETCH && layer == a.n_layers - 1 && tid == 0) plan_and_load(cur ^ 1);
       // ---- 1. the projection on the tensor cores (one elected thread)
       if (tid == 0) {
         tc_fence_after();
@@ -316,7 +326,7 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
       tc_fence_before();
       __syncthreads();
       // ---- 2. attention (SIMT), output into the q slots
-      tile_attention<float, H, D, C, NT, QS>(sQ, meta, 0, warp, lane);
+      tile_attention<float, H, D, C, NT, QS>(sQ, meta, cur, warp, lane);
       __syncthreads();
     }
     if (meta.fail) break;
@@ -327,12 +337,21 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
       for (int r = lane; r < rows; r += 32)
         bulk_s2g(out + (row0 + r) * C, sQ + r * QS, (uint32_t)(C * 4));
       bulk_commit();
-      bulk_wait_read_all();  // the next slab lands in the same region
+      bulk_wait_read_all();  // (without a slab buffer of its own, the next slab lands here)
     }
     __syncthreads();
+    if (Cfg::PREFETCH) {
+      cur ^= 1;
+    } else if (tid == 0) {
+      plan_and_load(cur);
+    }
   }
   if (warp == 0) bulk_wait_all();
-  if (tid == 0 && meta.fail) atomicOr(a.status, kStatusTimeout);
+  if (tid == 0 && meta.fail) {
+    atomicOr(a.status, kStatusTimeout);
+    // a prefetched slab may still be landing: let it finish before exit
+    if (Cfg::PREFETCH) mbar_wait(bar_x, ph_x);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

@@ -180,12 +180,15 @@ __device__ __forceinline__ void softmax_block(const T* q, T* o, T& mx, T& l, con
     T acc = T(0);
     if (!TAIL || b < n) {
       const T* kr = kb + b * QS;
-      if constexpr (sizeof(T) == 4 && D % 2 == 0) {
+      if constexpr (sizeof(T) == 4 && D % 4 == 0) {
+        // 16-byte broadcast loads, packed fp32x2 FMAs
         float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int t = 0; t < D; t += 2)
-          a2 = __ffma2_rn(make_float2(q[t], q[t + 1]),
-                          *reinterpret_cast<const float2*>(kr + t), a2);
+        for (int t = 0; t < D; t += 4) {
+          const float4 k4 = *reinterpret_cast<const float4*>(kr + t);
+          a2 = __ffma2_rn(make_float2(q[t], q[t + 1]), make_float2(k4.x, k4.y), a2);
+          a2 = __ffma2_rn(make_float2(q[t + 2], q[t + 3]), make_float2(k4.z, k4.w), a2);
+        }
         acc = a2.x + a2.y;
       } else {
 #pragma unroll
@@ -211,14 +214,17 @@ __device__ __forceinline__ void softmax_block(const T* q, T* o, T& mx, T& l, con
       const T pj = softmax_exp<T>(s[j] - mx);
       l += pj;
       const T* vr = vb + b * QS;
-      if constexpr (sizeof(T) == 4 && D % 2 == 0) {
+      if constexpr (sizeof(T) == 4 && D % 4 == 0) {
         const float2 p2 = make_float2(pj, pj);
 #pragma unroll
-        for (int t = 0; t < D; t += 2) {
-          float2 o2 = __ffma2_rn(p2, *reinterpret_cast<const float2*>(vr + t),
-                                 make_float2(o[t], o[t + 1]));
+        for (int t = 0; t < D; t += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(vr + t);
+          float2 o2 = __ffma2_rn(p2, make_float2(v4.x, v4.y), make_float2(o[t], o[t + 1]));
+          float2 o3 = __ffma2_rn(p2, make_float2(v4.z, v4.w), make_float2(o[t + 2], o[t + 3]));
           o[t] = o2.x;
           o[t + 1] = o2.y;
+          o[t + 2] = o3.x;
+          o[t + 3] = o3.y;
         }
       } else {
 #pragma unroll

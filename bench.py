@@ -42,6 +42,18 @@ SM_COUNT, SM_MAX_GHZ = 148, 1.965
 FP64_PEAK_TFLOPS = SM_COUNT * 64 * 2 * SM_MAX_GHZ / 1e3
 FP32_PEAK_TFLOPS = SM_COUNT * 128 * 2 * SM_MAX_GHZ / 1e3
 
+# Attention kernel of each workload and its DRAM traffic per launch
+# (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture of that
+# kernel, summarised under profiles/); None where no capture of the kernel as
+# it stands exists.  A change to a kernel resets its entry to None.
+ATTN_KERNEL = {
+    1: ("k_attn_hg<double,128,32,...>", None),
+    2: ("k_attn_dmma<160,5,640>", 5.609e6),   # profiles/k_attn_dmma_f64_diamond512.md
+    3: ("k_attn_tc<64,16,512>", None),
+    4: ("k_attn_hg<float,128,16,...>", None),
+    5: ("k_attn_tc<32,8,512>", None),
+}
+
 
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
@@ -440,9 +452,10 @@ def main(argv=None):
     bbytes = build_bytes(w.n_atoms, E)
     abytes = attention_bytes(w.n_atoms, E, w.channels, elem) + \
         (w.n_layers - 1) * 3.0 * w.channels * w.channels * elem
+    kname, traffic = ATTN_KERNEL.get(w.key, ("attention stack", None))
     roofline = {"bound": "alu", "achieved": achieved_tf, "peak": peak_fp, "unit": "TFLOP/s",
-                "frac": achieved_tf / peak_fp, "traffic": None,
-                "kernel": "attention stack (k_attn_tile: all %d layer(s) fused)" % w.n_layers,
+                "frac": achieved_tf / peak_fp, "traffic": traffic,
+                "kernel": "%s (all %d layer(s) in one launch)" % (kname, w.n_layers),
                 "algorithmic_flops_per_launch": flops,
                 "peak_basis": ("derived: 148 SMs x %d %s FMA/clk x 2 x 1.965 GHz" %
                                (64 if w.dtype == "f64" else 128, w.dtype.upper())),

@@ -333,24 +333,6 @@ int launch_tile(TileArgs& ta, cudaStream_t stream) {
   return launch_status();
 }
 
-// R = 40: 5 row blocks x 4 heads = 20 attention items and 60 projection
-// blocks per centre, so 10 warps share both phases evenly.
-template <int R, int NT>
-int launch_dmma(TileArgs& ta, cudaStream_t stream) {
-  using Cfg = DmmaCfg<R, NT>;
-  auto kern = k_attn_dmma<R, NT>;
-  prefer_shared(kern, Cfg::SMEM);
-  if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
-  int occ = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, Cfg::SMEM);
-  if (occ < 1) occ = 1;
-  int64_t want = (int64_t)sm_count() * occ;
-  int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
-  if (grid < 1) grid = 1;
-  kern<<<grid, NT, Cfg::SMEM, stream>>>(ta);
-  return launch_status();
-}
-
 // Blocks of `kern` that fit on one SM by registers, shared memory, warps.
 template <typename K>
 int resident_blocks(K kern, int nt, size_t dyn_smem) {
@@ -369,6 +351,22 @@ int resident_blocks(K kern, int nt, size_t dyn_smem) {
   int b = by_regs < by_smem ? by_regs : by_smem;
   b = b < by_thr ? b : by_thr;
   return b < 1 ? 1 : b;
+}
+
+// FP64 tensor-core kernel: one CTA of NT threads per SM (shared memory), tiles
+// of R rows, centres of at most 8 NBC edges.
+template <int R, int NBC, int NT>
+int launch_dmma(TileArgs& ta, cudaStream_t stream) {
+  using Cfg = DmmaCfg<R, NBC, NT>;
+  auto kern = k_attn_dmma<R, NBC, NT>;
+  prefer_shared(kern, Cfg::SMEM);
+  if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
+  int occ = resident_blocks(kern, NT, Cfg::SMEM);
+  int64_t want = (int64_t)sm_count() * occ;
+  int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
+  if (grid < 1) grid = 1;
+  kern<<<grid, NT, Cfg::SMEM, stream>>>(ta);
+  return launch_status();
 }
 
 // A 2-D tensor map over G [rows][C] fp32 with a {4 x 128} box (16-byte inner
@@ -420,10 +418,12 @@ int launch_tc(TileArgs& ta, cudaStream_t stream) {
   return launch_status();
 }
 
-// fp64, 32 channels, head size 8: FP64 tensor-core kernel, tile rows by nnei_max
+// fp64, 32 channels, head size 8: FP64 tensor-core kernel; the most edges of
+// a centre it takes (40 or 64), by nnei_max
 int dmma_rows(int nnei_max) { return nnei_max <= 40 ? 40 : 64; }
 
-// Returns the tile rows R of the fused kernel for this shape (0: none).
+// Returns the most edges of a centre that the fused kernel for this shape
+// takes (0: no fused kernel); larger centres go to the generic kernel.
 int tile_rows(mlg_dtype dtype, int C, int D, int nnei_max) {
   if (dtype == MLG_F64 && C == 32 && D == 8) return dmma_rows(nnei_max);
   if (dtype == MLG_F32 && C == 32 && D == 8) return 128;
@@ -434,7 +434,8 @@ int tile_rows(mlg_dtype dtype, int C, int D, int nnei_max) {
 int launch_tile_shape(mlg_dtype dtype, int C, int D, int nnei_max, TileArgs& ta,
                       cudaStream_t s) {
   if (dtype == MLG_F64 && C == 32 && D == 8)
-    return dmma_rows(nnei_max) == 40 ? launch_dmma<40, 320>(ta, s) : launch_dmma<64, 256>(ta, s);
+    return dmma_rows(nnei_max) == 40 ? launch_dmma<160, 5, 640>(ta, s)
+                                     : launch_dmma<128, 8, 512>(ta, s);
   if (dtype == MLG_F32 && C == 32 && D == 8) return launch_tc<32, 8, 512>(ta, s);
   if (dtype == MLG_F32 && C == 64 && D == 16) return launch_tc<64, 16, 512>(ta, s);
   return MLG_ERR_UNSUPPORTED;

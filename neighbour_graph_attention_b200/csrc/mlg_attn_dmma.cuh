@@ -1,20 +1,31 @@
 // mlg_attn_dmma.cuh -- fused multi-layer block-dense attention in fp64 on the
-// FP64 tensor pipe (mma.sync m8n8k4 .f64, sm_100a).
+// FP64 tensor pipe (mma.sync m16n8k8 / m16n8k16 .f64, sm_100a).
 //
 // The per-centre attention of the NeighborGraph issue (Proposed fix: dense
 // attention per centre with masks for the ragged tail, written back to the
 // edge axis), for c = 32 channels, 4 heads of d = 8, in fp64.  Every product
-// is an 8x8x4 fp64 MMA (one instruction per 256 FMAs, at the FP64 FMA rate):
-//   projection  QKV [rows][96] = X [rows][32] . [Wq | Wk | Wv]   (8 k-steps)
-//   logits      S = Q_h K_h^T per 8-row block of queries          (2 k-steps)
-//   output      O = P_h V_h                                       (keys / 4 steps)
-// The softmax runs on the S accumulators in registers: each row of an 8x8
-// accumulator lives in 4 lanes, so row max and row sum take two shuffles,
-// and the A operand of P V is gathered from those accumulators by shuffles.
+// is a 16x8 fp64 MMA:
+//   K   [rows][32] = X . Wk               m16n8k16, 16-row blocks
+//   V^T [32][rows] = Wv^T . X^T           m16n8k16, 8-row blocks (stored transposed)
+//   Q_h [16][8]    = X . Wq_h             m16n8k16, kept in registers
+//   S   [16][8]    = Q_h . K_h^T          m16n8k8 per 8-key block
+//   O   [16][8]   += P . V_h              m16n8k8 per 8-key block
+// A contraction may visit its k index in any order, so each one permutes it
+// to suit the fragments at hand: the projections read channel 4t + m at k
+// slot t + 4m (both operands then come in contiguous 16-byte pieces); the
+// logits read head dimension 2t + e at k slot t + 4e, which is the column
+// layout of the Q accumulator; P V reads key 2t + e at k slot t + 4e, which
+// is the column layout of the S accumulator.  So Q and P never leave
+// registers and need no shuffles.
+// Softmax: each lane holds two query rows (g and g + 8) of every 8-key
+// block; the row max and sum take two shuffles each; exponentials are in
+// base 2 (log2 e is folded into the Q scale) by a table-driven method.
 // Rows of a centre are padded to a multiple of 8 with zero features (their
-// keys are masked to -inf; their values are 0, so masked slots add exactly 0).
-// Tiles of consecutive centres (padded rows <= R) stay in shared memory for
-// all layers; only the final layer is written back.
+// keys are masked to -inf and their values are 0); query blocks of 16 rows
+// may run past a centre into rows that are only read, never written.
+// One CTA per SM holds a tile of consecutive centres for all layers: the
+// layer's input X and its output ping-pong between two buffers, and only the
+// last layer's output goes back to global memory.
 #pragma once
 
 #include "mlg_common.cuh"
@@ -23,42 +34,138 @@
 
 namespace mlg {
 
-__device__ __forceinline__ void dmma884(double& c0, double& c1, double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
-               : "+d"(c0), "+d"(c1)
-               : "d"(a), "d"(b));
+// C[16x8] += A[16x8] B[8x8] (fp64).  Lane (g, t) = (lane / 4, lane % 4) holds
+// a = {A(g,t), A(g+8,t), A(g,t+4), A(g+8,t+4)}, b = {B(t,g), B(t+4,g)},
+// c = {C(g,2t), C(g,2t+1), C(g+8,2t), C(g+8,2t+1)}.
+__device__ __forceinline__ void dmma_k8(double (&c)[4], double a0, double a1, double a2, double a3,
+                                        double b0, double b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3])
+      : "d"(a0), "d"(a1), "d"(a2), "d"(a3), "d"(b0), "d"(b1));
 }
 
-template <int R, int NT>
+// C[16x8] += A[16x16] B[16x8] (fp64): a[i] = A(g + 8 (i % 2), t + 4 (i / 2)),
+// b[i] = B(t + 4 i, g), c as in dmma_k8.
+__device__ __forceinline__ void dmma_k16(double (&c)[4], const double (&a)[8],
+                                         const double (&b)[4]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, "
+      "{%4,%5,%6,%7,%8,%9,%10,%11}, {%12,%13,%14,%15}, {%0,%1,%2,%3};"
+      : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3])
+      : "d"(a[0]), "d"(a[1]), "d"(a[2]), "d"(a[3]), "d"(a[4]), "d"(a[5]), "d"(a[6]), "d"(a[7]),
+        "d"(b[0]), "d"(b[1]), "d"(b[2]), "d"(b[3]));
+}
+
+// 2^y for y <= 0 (-inf -> 0, NaN -> NaN), after P. T. P. Tang's table-driven
+// exponential (ACM TOMS 15(2), 1989), in base 2: k = rint(32 y),
+// r = y - k / 32 (exact, |r| <= 1/64), 2^y = 2^(k >> 5) 2^((k & 31) / 32) 2^r.
+// The 32 table values 2^(j/32) sit one per lane (`tab` in lane j) and come by
+// a shuffle; 2^r = exp(r ln 2) is its Taylor series to degree 5 (truncation
+// below 2.3e-15 relative, as |r ln 2| <= 0.0109).  Below y = -1000 the result
+// is 0 (the true value is below 1e-301); above it the scaling by 2^(k >> 5)
+// is an add to the exponent field that stays in the normal range.
+namespace exp2tab {
+constexpr double kLn2 = 0.693147180559945309417232121458176568;
+constexpr double c1 = kLn2, c2 = c1 * kLn2 / 2, c3 = c2 * kLn2 / 3, c4 = c3 * kLn2 / 4,
+                 c5 = c4 * kLn2 / 5;
+constexpr double kRound = 6755399441055744.0;  // 1.5 * 2^52: adding it rounds to an integer
+}  // namespace exp2tab
+
+__device__ __forceinline__ double exp2_neg(double y, double tab) {
+  double kd = fma(y, 32.0, exp2tab::kRound);
+  const int k = __double2loint(kd);
+  kd -= exp2tab::kRound;
+  const double r = fma(kd, -1.0 / 32.0, y);
+  double p = exp2tab::c5;
+  p = fma(p, r, exp2tab::c4);
+  p = fma(p, r, exp2tab::c3);
+  p = fma(p, r, exp2tab::c2);
+  p = fma(p, r, exp2tab::c1);
+  p = fma(p, r, 1.0);
+  const double v = __shfl_sync(kFull, tab, k & 31) * p;
+  const double out = __hiloint2double(__double2hiint(v) + ((k >> 5) << 20), __double2loint(v));
+  return y < -1000.0 ? 0.0 : out;
+}
+
+__device__ __forceinline__ double2 lds2(const double* p) {
+  return *reinterpret_cast<const double2*>(p);
+}
+__device__ __forceinline__ void sts2(double* p, double x, double y) {
+  *reinterpret_cast<double2*>(p) = make_double2(x, y);
+}
+
+// Fragment A of a 16-row m16n8k16 block from a row-major [rows][stride]
+// array at `p` = row g, column 4 t (+ k0): channels 4t .. 4t + 3 of rows g and
+// g + 8 in k slots t, t + 4, t + 8, t + 12.
+__device__ __forceinline__ void frag_a16(double (&av)[8], const double* p, int stride) {
+  double2 v;
+  v = lds2(p);              av[0] = v.x; av[2] = v.y;
+  v = lds2(p + 2);          av[4] = v.x; av[6] = v.y;
+  v = lds2(p + 8 * stride); av[1] = v.x; av[3] = v.y;
+  v = lds2(p + 8 * stride + 2); av[5] = v.x; av[7] = v.y;
+}
+// Fragment B (k slots t + 4i, i = 0..3) from the same channel-contiguous
+// layout, column g of the product = row g of the array.
+__device__ __forceinline__ void frag_b16(double (&bv)[4], const double* p) {
+  double2 v;
+  v = lds2(p);     bv[0] = v.x; bv[1] = v.y;
+  v = lds2(p + 2); bv[2] = v.x; bv[3] = v.y;
+}
+// Fragment B from a [k][stride] weight array at `p` = row 4t (+ k0), column
+// g of the product: rows 4t .. 4t + 3 in k slots t + 4i.
+__device__ __forceinline__ void frag_bw(double (&bv)[4], const double* p, int stride) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) bv[i] = p[i * stride];
+}
+// Fragment A of the transposed weights (rows of the product = columns g,
+// g + 8 of the array) from a [k][stride] array at `p` = row 4t (+ k0),
+// column g.
+__device__ __forceinline__ void frag_aw(double (&av)[8], const double* p, int stride) {
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    av[2 * m] = p[m * stride];
+    av[2 * m + 1] = p[m * stride + 8];
+  }
+}
+
+// R: tile rows (centres padded to 8 rows, packed); NBC: key blocks of 8 per
+// centre at most (centres with more than 8 NBC edges are not taken).
+template <int R, int NBC, int NT>
 struct DmmaCfg {
-  static constexpr int C = 32, D = 8, H = 4, N3 = 96;
-  static constexpr int NB = R / 8;         // row blocks per tile (and per centre at most)
-  static constexpr int XS = 36;            // strides = 4 (mod 16) doubles: conflict-free frags
-  static constexpr int QS = 100;
-  static constexpr int WS = 100;
-  static constexpr size_t OFF_X = 0;
-  static constexpr size_t OFF_Q = OFF_X + (size_t)R * XS * 8;
-  static constexpr size_t OFF_W = OFF_Q + (size_t)R * QS * 8;
-  static constexpr size_t OFF_S = OFF_W + (size_t)C * WS * 8;
-  static constexpr size_t OFF_META = (OFF_S + (size_t)R * 8 + 15) / 16 * 16;
+  static constexpr int C = 32, D = 8, H = 4;
+  static constexpr int RA = R + 8;   // + slack read by 16-row blocks past the last centre
+  static constexpr int XS = 34;      // row strides in doubles, chosen so that the
+  static constexpr int KS = 40;      // 16-byte fragment loads and stores of every
+  static constexpr int VS = RA;      // phase are free of bank conflicts
+  static constexpr int WS = 3 * C + 2;  // W rows: == 2 (mod 4) doubles, 16-byte multiple
+  static constexpr size_t XBYTES = (size_t)RA * XS * 8;
+  static constexpr size_t OFF_X = 0;                               // [2][RA][XS]
+  static constexpr size_t OFF_K = OFF_X + 2 * XBYTES;              // [RA][KS]
+  static constexpr size_t OFF_V = OFF_K + (size_t)RA * KS * 8;     // [C][VS]  (V^T)
+  static constexpr size_t OFF_W = OFF_V + (size_t)C * VS * 8;      // [C][WS]: [Wq | Wk | Wv]
+  static constexpr size_t OFF_S = OFF_W + (size_t)C * WS * 8;      // [RA]
+  static constexpr size_t OFF_META = (OFF_S + (size_t)RA * 8 + 15) / 16 * 16;
   static constexpr size_t SMEM = OFF_META + sizeof(TileMeta);
-  static_assert(R % 8 == 0 && NT % 32 == 0, "shapes");
+  static_assert(R % 16 == 0 && VS % 16 == 8 && NBC * 8 <= R && NT % 32 == 0, "shapes");
 };
 
-template <int R, int NT>
-__global__ void __launch_bounds__(NT) k_attn_dmma(TileArgs a) {
-  using Cfg = DmmaCfg<R, NT>;
-  constexpr int C = Cfg::C, D = Cfg::D, H = Cfg::H, NB = Cfg::NB;
-  constexpr int XS = Cfg::XS, QS = Cfg::QS, WS = Cfg::WS;
+template <int R, int NBC, int NT>
+__global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
+  using Cfg = DmmaCfg<R, NBC, NT>;
+  constexpr int C = Cfg::C, D = Cfg::D, H = Cfg::H, RA = Cfg::RA;
+  constexpr int XS = Cfg::XS, KS = Cfg::KS, VS = Cfg::VS, WS = Cfg::WS;
   constexpr int NW = NT / 32;
   extern __shared__ __align__(128) unsigned char smem[];
-  double* sX = reinterpret_cast<double*>(smem + Cfg::OFF_X);
-  double* sQ = reinterpret_cast<double*>(smem + Cfg::OFF_Q);
+  double* sXb = reinterpret_cast<double*>(smem + Cfg::OFF_X);
+  double* sK = reinterpret_cast<double*>(smem + Cfg::OFF_K);
+  double* sV = reinterpret_cast<double*>(smem + Cfg::OFF_V);
   double* sW = reinterpret_cast<double*>(smem + Cfg::OFF_W);
   double* sS = reinterpret_cast<double*>(smem + Cfg::OFF_S);
   TileMeta& meta = *reinterpret_cast<TileMeta*>(smem + Cfg::OFF_META);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int lr = lane >> 2, lc = lane & 3;  // fragment row / column index
+  const int g = lane >> 2, t = lane & 3;
   const double* G = static_cast<const double*>(a.G);
   double* out = static_cast<double*>(a.out);
   const int64_t E = a.row_ptr[a.n_centres];
@@ -77,186 +184,259 @@ __global__ void __launch_bounds__(NT) k_attn_dmma(TileArgs a) {
     meta.next_c = lb(r0);
     meta.c_end = blockIdx.x + 1 == gridDim.x ? (int)a.n_centres : lb(r1);
   }
+  const double tab = exp2((double)lane / 32.0);               // 2^(lane / 32)
+  const double qscale = 1.4426950408889634 / sqrt((double)D);  // log2(e) / sqrt(d)
   __syncthreads();
-  const double rsd = 1.0 / sqrt((double)D);
+
+  // weights: sW[k][m C + col] = W_m[k][col] (m = 0, 1, 2: q, k, v), copied
+  // by 16-byte async copies; a layer's q block and its k, v blocks are
+  // copied at different times (see the layer loop)
+  auto load_w = [&](int layer, int m0, int nm) {
+    for (int e = tid; e < nm * C * (C / 2); e += NT) {
+      const int m = m0 + e / (C * (C / 2)), rem = e % (C * (C / 2));
+      const int k = rem / (C / 2), v = rem % (C / 2);
+      cp_async16(sW + k * WS + m * C + 2 * v,
+                 static_cast<const double*>(a.W[3 * layer + m]) + k * C + 2 * v);
+    }
+    cp_async_commit();
+  };
 
   while (true) {
-    // ---- plan a tile: consecutive centres, padded rows <= R (c0[0] = first centre)
+    // ---- plan a tile: consecutive centres with 1 .. 8 NBC edges, each padded
+    // to a multiple of 8 rows, padded rows <= R
     if (tid == 0) {
-      int c = meta.next_c, k = 0, rows = 0;
+      int c = meta.next_c, k = 0, rows = 0, tasks = 0;
       const int c_end = meta.c_end;
       while (c < c_end) {
         const int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
-        if (n > 0 && n <= R) break;
+        if (n > 0 && n <= NBC * 8) break;
         ++c;
       }
       meta.c0[0] = c;
       while (c < c_end && k < 64) {
         const int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
         const int n8 = (n + 7) & ~7;
-        if (n > R || rows + n8 > R) break;
+        if (n > NBC * 8 || rows + n8 > R) break;
         meta.off[0][k] = rows;
+        meta.task0[0][k] = tasks;
+        tasks += ((n + 15) / 16) * H;
         rows += n8;
         ++k;
         ++c;
       }
       meta.off[0][k] = rows;
+      meta.task0[0][k] = tasks;
       meta.ncent[0] = k;
       meta.nrows[0] = rows;
       meta.next_c = c;
     }
     __syncthreads();
     const int ncent = meta.ncent[0], prow = meta.nrows[0], c0 = meta.c0[0];
+    const int ntask = meta.task0[0][ncent];
     if (ncent == 0) break;
-    // ---- load the tile's rows (16-byte async copies), zero the padding rows
+
+    // ---- load the tile: each centre's rows by 16-byte async copies into
+    // buffer 0; padding rows and the slack zero in both buffers
     for (int ci = 0; ci < ncent; ++ci) {
       const int64_t g0 = a.row_ptr[c0 + ci];
       const int n = (int)(a.row_ptr[c0 + ci + 1] - g0);
       const int off = meta.off[0][ci], n8 = meta.off[0][ci + 1] - off;
-      for (int e = tid; e < n8 * (C / 2); e += NT) {
+      for (int e = tid; e < n * (C / 2); e += NT) {
         const int r = e / (C / 2), v = e - r * (C / 2);
-        double* dst = sX + (off + r) * XS + 2 * v;
-        if (r < n) cp_async16(dst, G + (g0 + r) * C + 2 * v);
-        else dst[0] = dst[1] = 0.0;
+        cp_async16(sXb + (off + r) * XS + 2 * v, G + (g0 + r) * C + 2 * v);
+      }
+      for (int e = tid; e < (n8 - n) * (C / 2); e += NT) {
+        const int r = off + n + e / (C / 2), v = e % (C / 2);
+        sts2(sXb + r * XS + 2 * v, 0.0, 0.0);
+        sts2(sXb + (RA + r) * XS + 2 * v, 0.0, 0.0);
       }
       for (int r = tid; r < n8; r += NT) sS[off + r] = r < n ? a.sw[g0 + r] : 0.0;
     }
     cp_async_commit();
+    for (int e = tid; e < (RA - prow) * (C / 2); e += NT) {
+      const int r = prow + e / (C / 2), v = e % (C / 2);
+      sts2(sXb + r * XS + 2 * v, 0.0, 0.0);
+      sts2(sXb + (RA + r) * XS + 2 * v, 0.0, 0.0);
+    }
+    for (int r = prow + tid; r < RA; r += NT) sS[r] = 0.0;
+    load_w(0, 0, 3);
+    cp_async_wait<0>();
+    __syncthreads();
 
-    // weights of a layer: sW[k][m * 32 + col] = W_m[k][col]; the next layer's
-    // copy starts as soon as the projection no longer reads sW
-    auto load_weights = [&](int layer) {
-      for (int e = tid; e < 3 * C * (C / 2); e += NT) {
-        const int m = e / (C * (C / 2)), rem = e - m * C * (C / 2);
-        const int k = rem / (C / 2), v = rem - k * (C / 2);
-        cp_async16(sW + k * WS + m * C + 2 * v,
-                   static_cast<const double*>(a.W[3 * layer + m]) + k * C + 2 * v);
-      }
-      cp_async_commit();
-    };
-    load_weights(0);
+    const int nrb16 = (prow + 15) / 16;  // 16-row blocks of the tile
     for (int layer = 0; layer < a.n_layers; ++layer) {
+      const double* sX = sXb + (layer & 1) * RA * XS;
+      double* sXn = sXb + ((layer + 1) & 1) * RA * XS;
+      // this layer's Wq is copied during phase A (the previous layer's
+      // phase B was its last reader)
+      if (layer > 0) load_w(layer, 0, 1);
+
+      // ---- phase A: K (16-row blocks x pairs of 8-column blocks) and V^T
+      // (16-dimension blocks x pairs of 8-row blocks); 4 MMAs per item
+      const int nka = nrb16 * 2;
+      for (int item = warp; item < 2 * nka; item += NW) {
+        double c[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
+        if (item < nka) {
+          const int rb = item >> 1, cb = (item & 1) * 2;  // rows 16 rb.., columns 8 cb .. 8 cb + 15
+          const double* xr = sX + (rb * 16 + g) * XS + 4 * t;
+          const double* wr = sW + 4 * t * WS + C + cb * 8 + g;
+#pragma unroll
+          for (int k0 = 0; k0 < C; k0 += 16) {
+            double av[8], b0[4], b1[4];
+            frag_a16(av, xr + k0, XS);
+            frag_bw(b0, wr + k0 * WS, WS);
+            frag_bw(b1, wr + k0 * WS + 8, WS);
+            dmma_k16(c[0], av, b0);
+            dmma_k16(c[1], av, b1);
+          }
+          const int r = rb * 16 + g;
+          const double s0 = sS[r], s1 = sS[r + 8];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            double* kr = sK + r * KS + (cb + j) * 8 + 2 * t;
+            sts2(kr, c[j][0] * s0, c[j][1] * s0);
+            sts2(kr + 8 * KS, c[j][2] * s1, c[j][3] * s1);
+          }
+        } else {
+          const int it = item - nka;
+          const int db = it & 1, rb = it >> 1;  // dimensions 16 db.., rows 16 rb..
+          const double* wr = sW + 4 * t * WS + 2 * C + db * 16 + g;
+          const double* xr = sX + (rb * 16 + g) * XS + 4 * t;
+#pragma unroll
+          for (int k0 = 0; k0 < C; k0 += 16) {
+            double av[8], b0[4], b1[4];
+            frag_aw(av, wr + k0 * WS, WS);
+            frag_b16(b0, xr + k0);
+            frag_b16(b1, xr + 8 * XS + k0);
+            dmma_k16(c[0], av, b0);
+            dmma_k16(c[1], av, b1);
+          }
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            double* vr = sV + (db * 16 + g) * VS + rb * 16 + j * 8 + 2 * t;
+            sts2(vr, c[j][0], c[j][1]);
+            sts2(vr + 8 * VS, c[j][2], c[j][3]);
+          }
+        }
+      }
       cp_async_wait<0>();
       __syncthreads();
 
-      // ---- projection: pairs of 8x8 output blocks (row block, two adjacent
-      // column blocks) over the warps; the pair shares the A fragment and
-      // gives two independent accumulator chains
-      const int nrb = prow / 8;
-      for (int item = warp; item < nrb * 6; item += NW) {
-        const int mb = item / 6, nb = (item - mb * 6) * 2;
-        double c0v = 0.0, c1v = 0.0, c2v = 0.0, c3v = 0.0;
-#pragma unroll
-        for (int k = 0; k < C / 4; ++k) {
-          const double av = sX[(mb * 8 + lr) * XS + k * 4 + lc];
-          const double bv0 = sW[(k * 4 + lc) * WS + nb * 8 + lr];
-          const double bv1 = sW[(k * 4 + lc) * WS + nb * 8 + 8 + lr];
-          dmma884(c0v, c1v, av, bv0);
-          dmma884(c2v, c3v, av, bv1);
-        }
-        const int r = mb * 8 + lr, col = nb * 8 + 2 * lc;
-        const double s = sS[r];
-        // the two blocks never straddle q / k / v (32 is a multiple of 16)
-        const double f = col < C ? s * rsd : (col < 2 * C ? s : 1.0);
-        sQ[r * QS + col] = c0v * f;
-        sQ[r * QS + col + 1] = c1v * f;
-        sQ[r * QS + col + 8] = c2v * f;
-        sQ[r * QS + col + 9] = c3v * f;
-      }
-      __syncthreads();
-      if (layer + 1 < a.n_layers) load_weights(layer + 1);
+      // the next layer's Wk, Wv are copied during phase B (phase A above was
+      // their last reader)
+      if (layer + 1 < a.n_layers) load_w(layer + 1, 1, 2);
 
-      // ---- attention: items (centre, head, query row block)
-      int nitems = 0;
-      for (int ci = 0; ci < ncent; ++ci) nitems += ((meta.off[0][ci + 1] - meta.off[0][ci]) / 8) * H;
-      for (int item = warp; item < nitems; item += NW) {
-        int ci = 0, base_item = 0;
-        while (true) {
-          const int cnt = ((meta.off[0][ci + 1] - meta.off[0][ci]) / 8) * H;
-          if (item < base_item + cnt) break;
-          base_item += cnt;
-          ++ci;
-        }
+      // ---- phase B: tasks (centre, 16-row query block, head)
+      for (int task = warp; task < ntask; task += NW) {
+        int ci = 0;
+        while (meta.task0[0][ci + 1] <= task) ++ci;
         const int off = meta.off[0][ci];
-        const int nbk = (meta.off[0][ci + 1] - off) / 8;   // key blocks of this centre
         const int n = (int)(a.row_ptr[c0 + ci + 1] - a.row_ptr[c0 + ci]);
-        const int rel = item - base_item;
-        const int h = rel / nbk, ib = rel - h * nbk;
-        // logits of 8 query rows against all keys of the centre
-        double s[NB][2];
+        const int nkb = (meta.off[0][ci + 1] - off) >> 3;
+        const int rel = task - meta.task0[0][ci];
+        const int qb = rel >> 2, h = rel & 3;
+        const int q0 = off + qb * 16;          // first query row of the block (tile-local)
+        const bool hi_rows = qb * 16 + 8 < n;  // rows g + 8 hold queries
+
+        // Q_h of the block: q[e] = Q(g, 2t + e), q[2 + e] = Q(g + 8, 2t + e)
+        double q[4] = {0.0, 0.0, 0.0, 0.0};
+        {
+          const double* xr = sX + (q0 + g) * XS + 4 * t;
+          const double* wr = sW + 4 * t * WS + h * D + g;
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-          s[j][0] = s[j][1] = 0.0;
-          if (j < nbk) {
+          for (int k0 = 0; k0 < C; k0 += 16) {
+            double av[8], bv[4];
+            frag_a16(av, xr + k0, XS);
+            frag_bw(bv, wr + k0 * WS, WS);
+            dmma_k16(q, av, bv);
+          }
+          const double f0 = sS[q0 + g] * qscale, f1 = sS[q0 + g + 8] * qscale;
+          q[0] *= f0;
+          q[1] *= f0;
+          q[2] *= f1;
+          q[3] *= f1;
+        }
+        // logits against the centre's keys (base-2 units):
+        // s[j][e] = S(g, 8j + 2t + e), s[j][2 + e] = S(g + 8, 8j + 2t + e)
+        double s[NBC][4];
 #pragma unroll
-            for (int kk = 0; kk < D / 4; ++kk) {
-              const double av = sQ[(off + ib * 8 + lr) * QS + h * D + kk * 4 + lc];
-              const double bv = sQ[(off + j * 8 + lr) * QS + C + h * D + kk * 4 + lc];
-              dmma884(s[j][0], s[j][1], av, bv);
+        for (int j = 0; j < NBC; ++j) {
+          s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0;
+          if (j < nkb) {
+            const double2 kv = lds2(sK + (off + 8 * j + g) * KS + h * D + 2 * t);
+            dmma_k8(s[j], q[0], q[2], q[1], q[3], kv.x, kv.y);
+          }
+        }
+        double m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < NBC; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const bool valid = j < nkb && 8 * j + 2 * t + e < n;
+            s[j][e] = valid ? s[j][e] : -INFINITY;
+            s[j][2 + e] = valid ? s[j][2 + e] : -INFINITY;
+            m0 = fmax(m0, s[j][e]);
+            m1 = fmax(m1, s[j][2 + e]);
+          }
+        m0 = fmax(m0, __shfl_xor_sync(kFull, m0, 1));
+        m0 = fmax(m0, __shfl_xor_sync(kFull, m0, 2));
+        m1 = fmax(m1, __shfl_xor_sync(kFull, m1, 1));
+        m1 = fmax(m1, __shfl_xor_sync(kFull, m1, 2));
+        double l0 = 0.0, l1 = 0.0;
+#pragma unroll
+        for (int j = 0; j < NBC; ++j) {
+          if (j < nkb) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              s[j][e] = exp2_neg(s[j][e] - m0, tab);
+              l0 += s[j][e];
+              if (hi_rows) {
+                s[j][2 + e] = exp2_neg(s[j][2 + e] - m1, tab);
+                l1 += s[j][2 + e];
+              } else {
+                s[j][2 + e] = 0.0;
+              }
             }
           }
         }
-        double mx = -INFINITY;
+        l0 += __shfl_xor_sync(kFull, l0, 1);
+        l0 += __shfl_xor_sync(kFull, l0, 2);
+        l1 += __shfl_xor_sync(kFull, l1, 1);
+        l1 += __shfl_xor_sync(kFull, l1, 2);
+        // O = P V_h over two accumulator chains (even / odd key blocks)
+        double o[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
 #pragma unroll
-        for (int j = 0; j < NB; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = j * 8 + 2 * lc + e;
-            if (j >= nbk || col >= n) s[j][e] = -INFINITY;
-            mx = fmax(mx, s[j][e]);
-          }
-        mx = fmax(mx, __shfl_xor_sync(kFull, mx, 1));
-        mx = fmax(mx, __shfl_xor_sync(kFull, mx, 2));
-        double sum = 0.0;
-#pragma unroll
-        for (int j = 0; j < NB; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const double p = j < nbk ? exp(s[j][e] - mx) : 0.0;
-            s[j][e] = p;
-            sum += p;
-          }
-        sum += __shfl_xor_sync(kFull, sum, 1);
-        sum += __shfl_xor_sync(kFull, sum, 2);
-        // O = P V: the A operand (row lr, key 4 kk + lc) sits in lane
-        // (lr, (kk & 1) * 2 + lc / 2), element lc & 1, of accumulator kk / 2
-        // two accumulator chains (even / odd key steps), summed at the end
-        double o0 = 0.0, o1 = 0.0, o2 = 0.0, o3 = 0.0;
-        const int src_lo = (lane & ~3) | (lc >> 1), src_hi = src_lo | 2;
-#pragma unroll
-        for (int j = 0; j < NB; ++j) {
-          if (j < nbk) {
-            const double w0 = __shfl_sync(kFull, s[j][0], src_lo);
-            const double w1 = __shfl_sync(kFull, s[j][1], src_lo);
-            const double x0 = __shfl_sync(kFull, s[j][0], src_hi);
-            const double x1 = __shfl_sync(kFull, s[j][1], src_hi);
-            const double bv0 = sQ[(off + (2 * j) * 4 + lc) * QS + 2 * C + h * D + lr];
-            const double bv1 = sQ[(off + (2 * j + 1) * 4 + lc) * QS + 2 * C + h * D + lr];
-            dmma884(o0, o1, (lc & 1) ? w1 : w0, bv0);
-            dmma884(o2, o3, (lc & 1) ? x1 : x0, bv1);
+        for (int j = 0; j < NBC; ++j) {
+          if (j < nkb) {
+            const double2 vv = lds2(sV + (h * D + g) * VS + off + 8 * j + 2 * t);
+            dmma_k8(o[j & 1], s[j][0], s[j][2], s[j][1], s[j][3], vv.x, vv.y);
           }
         }
-        o0 += o2;
-        o1 += o3;
-        const double inv = 1.0 / sum;
-        const int r = ib * 8 + lr;
+        const int r = qb * 16 + g;
         if (r < n) {
-          double* xo = sX + (off + r) * XS + h * D + 2 * lc;
-          xo[0] = o0 * inv;
-          xo[1] = o1 * inv;
+          const double i0 = 1.0 / l0;
+          sts2(sXn + (q0 + g) * XS + h * D + 2 * t, (o[0][0] + o[1][0]) * i0,
+               (o[0][1] + o[1][1]) * i0);
+        }
+        if (r + 8 < n) {
+          const double i1 = 1.0 / l1;
+          sts2(sXn + (q0 + g + 8) * XS + h * D + 2 * t, (o[0][2] + o[1][2]) * i1,
+               (o[0][3] + o[1][3]) * i1);
         }
       }
+      cp_async_wait<0>();
       __syncthreads();
     }
     // ---- write the tile back (16-byte stores of each centre's real rows)
+    const double* sR = sXb + (a.n_layers & 1) * RA * XS;
     for (int ci = 0; ci < ncent; ++ci) {
       const int64_t g0 = a.row_ptr[c0 + ci];
       const int n = (int)(a.row_ptr[c0 + ci + 1] - g0);
       const int off = meta.off[0][ci];
       for (int e = tid; e < n * (C / 2); e += NT) {
         const int r = e / (C / 2), v = e - r * (C / 2);
-        const double2 val = *reinterpret_cast<const double2*>(sX + (off + r) * XS + 2 * v);
-        *reinterpret_cast<double2*>(out + (g0 + r) * C + 2 * v) = val;
+        *reinterpret_cast<double2*>(out + (g0 + r) * C + 2 * v) =
+            lds2(sR + (off + r) * XS + 2 * v);
       }
     }
     __syncthreads();

@@ -160,7 +160,9 @@ def _random_graph(n_atoms, density, rcut, nnei_max, seed):
 
 
 @pytest.mark.parametrize("dtype,channels,heads,n_layers,density,nnei", [
-    ("f64", 32, 4, 3, 0.13, 64),   # ~40 edges: fused tile (<= 40) + generic for larger rows
+    ("f64", 32, 4, 3, 0.13, 64),   # ~40 edges, all rows <= 64: fused tile of the 64-edge kind
+    ("f64", 32, 4, 2, 0.13, 40),   # ragged rows <= 40 (every row count mod 16): 40-edge kind
+    ("f64", 32, 4, 2, 0.2, 96),    # ~62 edges: fused tile (<= 64) + generic for larger rows
     ("f32", 64, 4, 1, 0.41, 181),  # ~128 edges: fused tile (<= 128) + generic for larger
     ("f32", 32, 4, 2, 0.004, 128), # dilute: many centres without edges between full ones
     ("f64", 128, 4, 2, 0.3, 96),   # head-group kernel, two layers (ping-pong)
@@ -193,8 +195,38 @@ def test_stack_mixed_row_sizes(dtype, channels, heads, n_layers, density, nnei):
     outs = oracle.forward(gpu["row_ptr"], gpu["sw"], G, W, heads, dtype)
     ok, err = U.attn_tolerance_ok(w, gout[:e].cpu().numpy(), outs[-1])
     assert ok, (err, counts.min(), counts.max())
-    if density in (0.13, 0.41, 0.31):    # both sides of the tile limit are exercised
-        limit = {0.13: 40, 0.41: 128, 0.31: 96}[density]
+    if (density, nnei) in ((0.2, 96), (0.41, 181), (0.31, 181)):  # both sides of the tile limit
+        limit = {0.2: 64, 0.41: 128, 0.31: 96}[density]
         assert counts.min() <= limit < counts.max()
+    if (density, nnei) == (0.13, 40):    # query blocks end in every position of a 16-row block
+        assert set(range(16)) <= set(int(c) % 16 for c in counts if c > 0)
     # rows past E are never written
     assert bool((gout[e:] == 0).all())
+
+
+def test_peaked_softmax_f64():
+    """Logits in the hundreds to thousands: most attention weights underflow
+    (base-2 exponent arguments far below -1000) and the rest still match."""
+    import oracle
+    from neighbour_graph_attention_b200.configs import Workload
+
+    m = U.mlg()
+    gpu, csr_t = _random_graph(3000, 0.13, 4.2, 40, 23)
+    e = gpu["n_edges"]
+    w = Workload(0, "random", "random", 0, 0, 0, 3000, 4.2, 3.7, 40, 32, 4, 1, "f64")
+    rng = np.random.default_rng(9)
+    W = rng.normal(0, 1 / np.sqrt(32), (1, 3, 32, 32))
+    G = rng.normal(0, 12.0, (e, 32))
+    out = U.gpu_attention(csr_t, 3000, w, G, W[0][0], W[0][1], W[0][2])
+    ref = oracle.attention(gpu["row_ptr"], gpu["sw"], G, W[0][0], W[0][1], W[0][2], 4)
+    # the case is as peaked as intended: in centre 0 some logit gaps (head 0)
+    # exceed 1000 ln 2
+    r0, r1 = int(gpu["row_ptr"][0]), int(gpu["row_ptr"][1])
+    sw0 = gpu["sw"][r0:r1]
+    q = (G[r0:r1] @ W[0][0])[:, :8] * sw0[:, None]
+    k = (G[r0:r1] @ W[0][1])[:, :8] * sw0[:, None]
+    lg = q @ k.T / np.sqrt(8)
+    assert float((lg.max(axis=1) - lg.min(axis=1)).max()) > 1000 * np.log(2)
+    assert int(csr_t.status.item()) == 0
+    ok, err = U.attn_tolerance_ok(w, out, ref)
+    assert ok, err

@@ -453,6 +453,8 @@ def main(argv=None):
     abytes = attention_bytes(w.n_atoms, E, w.channels, elem) + \
         (w.n_layers - 1) * 3.0 * w.channels * w.channels * elem
     kname, traffic = ATTN_KERNEL.get(w.key, ("attention stack", None))
+    if args.cells is not None:   # a resized system: the stored capture does not apply
+        traffic = None
     roofline = {"bound": "alu", "achieved": achieved_tf, "peak": peak_fp, "unit": "TFLOP/s",
                 "frac": achieved_tf / peak_fp, "traffic": traffic,
                 "kernel": "%s (all %d layer(s) in one launch)" % (kname, w.n_layers),

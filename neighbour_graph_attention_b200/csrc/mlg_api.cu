@@ -29,7 +29,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Layout of the build workspace.
 struct BuildLayout {
   size_t grid, bbox, cell_count, cell_start, atom_cell, atom_rank, atom_w, recs, pos4, kept, raw,
-      partial, total;
+      partial, sync, total;
 };
 
 int64_t scan_tiles(int64_t n) { return (n + kScanTile - 1) / kScanTile; }
@@ -55,6 +55,7 @@ BuildLayout build_layout(int64_t n, int ncell_cap) {
   L.raw = take((size_t)n * sizeof(int));
   int64_t tiles = scan_tiles(n > ncell_cap ? n : ncell_cap + 1);
   L.partial = take((size_t)(tiles + 2) * sizeof(long long));
+  L.sync = take(sizeof(FusedSync));
   L.total = off;
   return L;
 }
@@ -139,6 +140,26 @@ void taylor_coeffs(double* c) {
 
 // Ask for the largest shared-memory carveout, so that the occupancy the
 // shared memory allows is the occupancy the launch gets.
+// Blocks of `kern` that fit on one SM by registers, shared memory, warps.
+template <typename K>
+int resident_blocks(K kern, int nt, size_t dyn_smem) {
+  cudaFuncAttributes fa;
+  int dev = 0, regs_sm = 65536, smem_sm = 233472, reserved = 1024, thr_sm = 2048;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
+  const int regs_warp = ((fa.numRegs * 32 + 255) / 256) * 256;
+  int by_regs = regs_sm / (regs_warp * (nt / 32));
+  int by_smem = (int)(smem_sm / (dyn_smem + fa.sharedSizeBytes + reserved));
+  int by_thr = thr_sm / nt;
+  int b = by_regs < by_smem ? by_regs : by_smem;
+  b = b < by_thr ? b : by_thr;
+  return b < 1 ? 1 : b;
+}
+
 template <typename K>
 void prefer_shared(K kern, size_t smem) {
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -176,6 +197,12 @@ int check_csr(const mlg_csr* csr) {
 }
 
 int sm_count();
+
+// Small systems on per-cell scans take the one-launch build.
+bool use_fused_build(const BuildPlan& plan, int64_t n) {
+  return plan.max_reach <= 1 && n >= 1 && n <= kFusedMaxAtoms &&
+         fused_build_fits(n, plan.ncell_cap);
+}
 
 int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
                const mlg_csr* csr, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -230,6 +257,37 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   a.raw = reinterpret_cast<int*>(w + L.raw);
   a.partial = reinterpret_cast<long long*>(w + L.partial);
 
+  // per-cell scans when every stencil reach is 1 (at most 27 stencil cells);
+  // otherwise (boxes narrower than the cutoff) the per-centre scans.  A grid
+  // of few cells splits each cell's centres over several CTAs.
+  const bool per_cell = plan.max_reach <= 1;
+  int nsplit = (4 * sm_count() + plan.ncell_cap - 1) / plan.ncell_cap;
+  nsplit = nsplit < 1 ? 1 : (nsplit > 8 ? 8 : nsplit);
+  if (use_fused_build(plan, n)) {
+    // the whole build in one cooperative launch (small systems)
+    const size_t smem = fused_build_smem(n);
+    prefer_shared(k_build_fused, smem);
+    const int64_t cap = (int64_t)resident_blocks(k_build_fused, kCellWarps * 32, smem) * sm_count();
+    const int64_t nitems = (int64_t)plan.ncell_cap * nsplit;
+    const int grid = (int)(nitems < cap ? nitems : cap);
+    FusedSync* sync = reinterpret_cast<FusedSync*>(w + L.sync);
+    if (cudaMemsetAsync(sync, 0, sizeof(FusedSync), stream) != cudaSuccess) return MLG_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kCellWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_build_fused, a, plan, plan.ncell_cap, nsplit, sync) ==
+        cudaSuccess)
+      return launch_status();
+    (void)cudaGetLastError();  // refused (not co-resident): the launch chain below
+  }
+
   const int tb = 256;
   const int atom_blocks = (int)((n + tb - 1) / tb);
   int init_blocks = (plan.ncell_cap + 1 + tb - 1) / tb;
@@ -243,12 +301,6 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   launch_scan<int>(a.cell_count, plan.ncell_cap, a.cell_start, a.partial,
                    ScanTail{nullptr, nullptr, 0}, stream);
   k_scatter<<<atom_blocks, tb, 0, stream>>>(a);
-  // per-cell scans when every stencil reach is 1 (at most 27 stencil cells);
-  // otherwise (boxes narrower than the cutoff) the per-centre scans.  A grid
-  // of few cells splits each cell's centres over several CTAs.
-  const bool per_cell = plan.max_reach <= 1;
-  int nsplit = (4 * sm_count() + plan.ncell_cap - 1) / plan.ncell_cap;
-  nsplit = nsplit < 1 ? 1 : (nsplit > 8 ? 8 : nsplit);
   const dim3 cell_grid((unsigned)plan.ncell_cap, (unsigned)nsplit);
   if (per_cell) {
     const size_t sm_count_ = cellscan_smem(false), sm_fill = cellscan_smem(true);
@@ -331,26 +383,6 @@ int launch_tile(TileArgs& ta, cudaStream_t stream) {
   if (grid < 1) grid = 1;
   kern<<<grid, NT, Cfg::SMEM, stream>>>(ta);
   return launch_status();
-}
-
-// Blocks of `kern` that fit on one SM by registers, shared memory, warps.
-template <typename K>
-int resident_blocks(K kern, int nt, size_t dyn_smem) {
-  cudaFuncAttributes fa;
-  int dev = 0, regs_sm = 65536, smem_sm = 233472, reserved = 1024, thr_sm = 2048;
-  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
-  cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
-  cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
-  const int regs_warp = ((fa.numRegs * 32 + 255) / 256) * 256;
-  int by_regs = regs_sm / (regs_warp * (nt / 32));
-  int by_smem = (int)(smem_sm / (dyn_smem + fa.sharedSizeBytes + reserved));
-  int by_thr = thr_sm / nt;
-  int b = by_regs < by_smem ? by_regs : by_smem;
-  b = b < by_thr ? b : by_thr;
-  return b < 1 ? 1 : b;
 }
 
 // FP64 tensor-core kernel: one CTA of NT threads per SM (shared memory), tiles
@@ -668,9 +700,12 @@ int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
   BuildPlan plan;
   if (n_layers < 1 || make_plan(n_atoms, rcut, box, pbc, &plan) != MLG_OK) return 0;
   auto scan_launches = [](int64_t n) { return n <= kScanSingleMax ? 1 : 3; };
-  // init, [bbox], bin, scan(cells), scatter, count, scan(row_ptr), fill, attention
+  const int attn = forward_launches(n_atoms, nnei_max, channels, heads, n_layers, dtype);
+  // one-launch build, or init, [bbox], bin, scan(cells), scatter, count,
+  // scan(row_ptr), fill; then the attention
+  if (use_fused_build(plan, n_atoms)) return 1 + attn;
   return 5 + (plan.any_open ? 1 : 0) + scan_launches(plan.ncell_cap) + scan_launches(n_atoms) +
-         forward_launches(n_atoms, nnei_max, channels, heads, n_layers, dtype);
+         attn;
 }
 
 const char* mlg_status_string(int status) {

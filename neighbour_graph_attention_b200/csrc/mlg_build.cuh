@@ -239,11 +239,12 @@ __global__ void k_init(BuildArgs a, int ncell_cap) {
   }
 }
 
-// Bounding box of the finite coordinates along open axes.
-__global__ void k_bbox(BuildArgs a, BuildPlan p) {
+// Bounding box of the finite coordinates along open axes: atoms i0, i0 +
+// stride, ... of this thread, folded into a.bbox (warp-collective).
+__device__ void bbox_accumulate(const BuildArgs& a, const BuildPlan& p, int64_t i0,
+                                int64_t stride) {
   double lo[3] = {INFINITY, INFINITY, INFINITY}, hi[3] = {-INFINITY, -INFINITY, -INFINITY};
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < a.n;
-       i += (int64_t)gridDim.x * blockDim.x) {
+  for (int64_t i = i0; i < a.n; i += stride) {
     double x0 = a.coords[3 * i], x1 = a.coords[3 * i + 1], x2 = a.coords[3 * i + 2];
     if (!(isfinite(x0) && isfinite(x1) && isfinite(x2))) continue;
     double x[3] = {x0, x1, x2};
@@ -268,10 +269,18 @@ __global__ void k_bbox(BuildArgs a, BuildPlan p) {
   }
 }
 
-__global__ void k_bin(BuildArgs a, BuildPlan p) {
-  CellGrid g = derive_grid(p, a.bbox);
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.grid = g;
-  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+__global__ void k_bbox(BuildArgs a, BuildPlan p) {
+  bbox_accumulate(a, p, (int64_t)blockIdx.x * blockDim.x + threadIdx.x,
+                  (int64_t)gridDim.x * blockDim.x);
+}
+
+// Cell, wrap image and in-cell rank of atom i (i >= n: none), counted in the
+// histogram `hist` (global or shared) with the rank in rank_out[i].  With
+// s_cell / s_w the cell and image also go to those (shared) arrays.  Called
+// by every lane of a warp (warp-aggregated histogram atomics).
+__device__ __forceinline__ void bin_atom(const BuildArgs& a, const CellGrid& g, int64_t i,
+                                         int* hist, int* rank_out, int* s_cell = nullptr,
+                                         int* s_w = nullptr) {
   int cell = -1;
   uint32_t st = 0;
   if (i < a.n) {
@@ -314,6 +323,10 @@ __global__ void k_bin(BuildArgs a, BuildPlan p) {
     }
     a.atom_cell[i] = cell;
     a.atom_w[i] = wpack;
+    if (s_cell != nullptr) {
+      s_cell[i] = cell;
+      s_w[i] = wpack;
+    }
     if (cell < 0) {  // left out of the cell lists: no centre scan will visit it
       a.kept[i] = 0;
       a.raw[i] = 0;
@@ -325,29 +338,29 @@ __global__ void k_bin(BuildArgs a, BuildPlan p) {
     unsigned peers = __match_any_sync(act, cell);
     int leader = __ffs(peers) - 1;
     int base = 0;
-    if ((int)lane_id() == leader) base = atomicAdd(&a.cell_count[cell], __popc(peers));
+    if ((int)lane_id() == leader) base = atomicAdd(&hist[cell], __popc(peers));
     base = __shfl_sync(peers, base, leader);
-    a.atom_rank[i] = base + __popc(peers & lanemask_lt());
+    rank_out[i] = base + __popc(peers & lanemask_lt());
   }
   st = __reduce_or_sync(kFull, st);
   if (lane_id() == 0 && st) atomicOr(a.status, st);
 }
 
-__global__ void k_scatter(BuildArgs a) {
-  __shared__ CellGrid sg;
-  if (threadIdx.x == 0) sg = *a.grid;
-  __syncthreads();
-  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= a.n) return;
-  int cell = a.atom_cell[i];
-  if (cell < 0) return;
+__global__ void k_bin(BuildArgs a, BuildPlan p) {
+  CellGrid g = derive_grid(p, a.bbox);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.grid = g;
+  bin_atom(a, g, (int64_t)blockIdx.x * blockDim.x + threadIdx.x, a.cell_count, a.atom_rank);
+}
+
+// Record and fp32 position of atom i (wrap image wpack) at cell-order slot pos.
+__device__ __forceinline__ void scatter_atom_at(const BuildArgs& a, const CellGrid& sg, int64_t i,
+                                                int pos, int wpack) {
   Rec r;
   r.x = a.coords[3 * i];
   r.y = a.coords[3 * i + 1];
   r.z = a.coords[3 * i + 2];
   r.j = (int)i;
-  r.w = a.atom_w[i];
-  const int pos = a.cell_start[cell] + a.atom_rank[i];
+  r.w = wpack;
   a.recs[pos] = r;
   double x[3] = {r.x, r.y, r.z};
   float y[3];
@@ -355,6 +368,17 @@ __global__ void k_scatter(BuildArgs a) {
   for (int k = 0; k < 3; ++k)
     y[k] = (float)(sg.periodic[k] ? x[k] - (double)unpack_w(r.w, k) * sg.L[k] : x[k] - sg.lo[k]);
   a.pos4[pos] = make_float4(y[0], y[1], y[2], __int_as_float((int)i));
+}
+
+__global__ void k_scatter(BuildArgs a) {
+  __shared__ CellGrid sg;
+  if (threadIdx.x == 0) sg = *a.grid;
+  __syncthreads();
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= a.n) return;
+  const int cell = a.atom_cell[i];
+  if (cell < 0) return;
+  scatter_atom_at(a, sg, i, a.cell_start[cell] + a.atom_rank[i], a.atom_w[i]);
 }
 
 // ----------------------------------------------------- candidate traversal
@@ -560,10 +584,86 @@ __device__ void warp_sort_pairs(unsigned long long* d, unsigned long long* k, in
   }
 }
 
+// Bitonic sorts of up to 64 elements held in registers, two per lane
+// (element e = 32 r + lane in register r); padding elements are ~0.
+__device__ __forceinline__ bool pair_lt(unsigned long long da, unsigned long long ka,
+                                        unsigned long long db, unsigned long long kb) {
+  return da < db || (da == db && ka < kb);
+}
+
+// ascending by (d, k)
+__device__ __forceinline__ void warp_sort64_pairs(unsigned long long& d0, unsigned long long& k0,
+                                                  unsigned long long& d1, unsigned long long& k1) {
+  const int lane = lane_id();
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride == 32) {  // partner in the other register; size 64: ascending
+        if (pair_lt(d1, k1, d0, k0)) {
+          const unsigned long long td = d0, tk = k0;
+          d0 = d1;
+          k0 = k1;
+          d1 = td;
+          k1 = tk;
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          unsigned long long& d = r ? d1 : d0;
+          unsigned long long& k = r ? k1 : k0;
+          const unsigned long long dp = __shfl_xor_sync(kFull, d, stride);
+          const unsigned long long kp = __shfl_xor_sync(kFull, k, stride);
+          const bool asc = ((32 * r + lane) & size) == 0;
+          const bool keep_min = ((lane & stride) == 0) == asc;  // lower element of an ascending pair
+          if (keep_min == pair_lt(dp, kp, d, k)) {
+            d = dp;
+            k = kp;
+          }
+        }
+      }
+    }
+  }
+}
+
+// ascending
+__device__ __forceinline__ void warp_sort64_keys(unsigned long long& k0, unsigned long long& k1) {
+  const int lane = lane_id();
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride == 32) {
+        if (k1 < k0) {
+          const unsigned long long tk = k0;
+          k0 = k1;
+          k1 = tk;
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          unsigned long long& k = r ? k1 : k0;
+          const unsigned long long kp = __shfl_xor_sync(kFull, k, stride);
+          const bool asc = ((32 * r + lane) & size) == 0;
+          const bool keep_min = ((lane & stride) == 0) == asc;
+          if (keep_min == (kp < k)) k = kp;
+        }
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------- fill
 
 __device__ __forceinline__ unsigned long long edge_key(int j, int tpack) {
   return ((unsigned long long)(unsigned)j << 21) | (unsigned long long)tpack;
+}
+
+// Key of a candidate staged in shared memory: the same (source, image) order
+// as edge_key, with the staging slot (< 1024) in the low 10 bits.
+__device__ __forceinline__ unsigned long long staged_key(int j, int tpack, int slot) {
+  return ((unsigned long long)(unsigned)j << 31) | ((unsigned long long)tpack << 10) |
+         (unsigned long long)slot;
 }
 
 // Selection for rows with more than kFillMaxCand candidates, without a
@@ -628,46 +728,82 @@ __device__ int fill_overflow_select(const BuildArgs& a, const CellGrid& g, const
   return pos < n ? pos : n;
 }
 
+// Writes edge p of centre cc for `key` (a staged_key() with srec, else an
+// edge_key()).
+__device__ __forceinline__ void write_edge(const BuildArgs& a, const Centre& cc,
+                                           unsigned long long key, int64_t p, const Rec* srec) {
+  int j, tp, wj;
+  double xj[3];
+  if (srec != nullptr) {
+    j = (int)(key >> 31);
+    tp = (int)((key >> 10) & 0x1fffffull);
+    const Rec& rc = srec[key & 1023ull];
+    wj = rc.w;
+    xj[0] = rc.x;
+    xj[1] = rc.y;
+    xj[2] = rc.z;
+  } else {
+    j = (int)(key >> 21);
+    if (j < 0 || (int64_t)j >= a.n) return;
+    tp = (int)(key & 0x1fffffull);
+    wj = a.atom_w[j];
+    xj[0] = a.coords[3 * (int64_t)j];
+    xj[1] = a.coords[3 * (int64_t)j + 1];
+    xj[2] = a.coords[3 * (int64_t)j + 2];
+  }
+  int S[3];
+  S[0] = ((tp >> 14) & 127) - 64 + cc.w[0] - unpack_w(wj, 0);
+  S[1] = ((tp >> 7) & 127) - 64 + cc.w[1] - unpack_w(wj, 1);
+  S[2] = (tp & 127) - 64 + cc.w[2] - unpack_w(wj, 2);
+  double v[3];
+  double r2 = edge_vec(a.box, cc.x, xj, S, v);
+  double r = __dsqrt_rn(r2);
+  if (p < a.capacity) {
+    a.src[p] = j;
+    a.shift[3 * p] = S[0];
+    a.shift[3 * p + 1] = S[1];
+    a.shift[3 * p + 2] = S[2];
+    a.vec[3 * p] = v[0];
+    a.vec[3 * p + 1] = v[1];
+    a.vec[3 * p + 2] = v[2];
+    a.dist[p] = r;
+    a.sw[p] = switch_fn(r, a.rcut, a.r_on, a.taylor);
+  }
+}
+
 // Sort the collected keys of one row into canonical order and write its
-// edges.  keys/d2 hold m collected candidates (keys and exact r^2 bits); the
-// row keeps n = min(raw, nnei_max).  Returns status bits.
+// edges.  keys/d2 hold m collected candidates (keys and exact r^2 bits, the
+// latter needed when m > n); the row keeps n = min(raw, nnei_max): the n
+// smallest by (r^2 bits, key), in key order.  With `srec`, the keys are
+// staged_key()s and the source records come from srec; otherwise
+// edge_key()s and global memory.  Rows of at most 64 candidates sort in
+// registers.  Returns status bits.
 __device__ uint32_t finish_row(const BuildArgs& a, const Centre& cc, unsigned long long* keys,
-                               unsigned long long* d2, int n, int m, int64_t p0) {
-  const unsigned lane = lane_id();
+                               unsigned long long* d2, int n, int m, int64_t p0,
+                               const Rec* srec = nullptr) {
+  const int lane = lane_id();
   uint32_t st = 0;
   if (m > kFillMaxCand) m = kFillMaxCand;
-  if (m > n) warp_sort_pairs(d2, keys, m);
   const int nv = n < m ? n : m;
-  warp_sort_keys(keys, nv);
   if (nv != n) st |= MLG_STATUS_INTERNAL;
-  for (int e = lane; e < nv; e += 32) {
-    unsigned long long key = keys[e];
-    int j = (int)(key >> 21);
-    if (j < 0 || (int64_t)j >= a.n) continue;
-    int tp = (int)(key & 0x1fffffull);
-    int wj = a.atom_w[j];
-    int S[3];
-    S[0] = ((tp >> 14) & 127) - 64 + cc.w[0] - unpack_w(wj, 0);
-    S[1] = ((tp >> 7) & 127) - 64 + cc.w[1] - unpack_w(wj, 1);
-    S[2] = (tp & 127) - 64 + cc.w[2] - unpack_w(wj, 2);
-    double xj[3] = {a.coords[3 * (int64_t)j], a.coords[3 * (int64_t)j + 1],
-                    a.coords[3 * (int64_t)j + 2]};
-    double v[3];
-    double r2 = edge_vec(a.box, cc.x, xj, S, v);
-    double r = __dsqrt_rn(r2);
-    int64_t p = p0 + e;
-    if (p < a.capacity) {
-      a.src[p] = j;
-      a.shift[3 * p] = S[0];
-      a.shift[3 * p + 1] = S[1];
-      a.shift[3 * p + 2] = S[2];
-      a.vec[3 * p] = v[0];
-      a.vec[3 * p + 1] = v[1];
-      a.vec[3 * p + 2] = v[2];
-      a.dist[p] = r;
-      a.sw[p] = switch_fn(r, a.rcut, a.r_on, a.taylor);
+  if (m <= 64) {
+    unsigned long long k0 = lane < m ? keys[lane] : ~0ull;
+    unsigned long long k1 = lane + 32 < m ? keys[lane + 32] : ~0ull;
+    if (m > n) {
+      unsigned long long e0 = lane < m ? d2[lane] : ~0ull;
+      unsigned long long e1 = lane + 32 < m ? d2[lane + 32] : ~0ull;
+      warp_sort64_pairs(e0, k0, e1, k1);
+      if (lane >= nv) k0 = ~0ull;
+      if (lane + 32 >= nv) k1 = ~0ull;
     }
+    warp_sort64_keys(k0, k1);
+    if (lane < nv) write_edge(a, cc, k0, p0 + lane, srec);
+    if (lane + 32 < nv) write_edge(a, cc, k1, p0 + lane + 32, srec);
+    return st;
   }
+  if (m > n) warp_sort_pairs(d2, keys, m);
+  warp_sort_keys(keys, nv);
+  for (int e = lane; e < nv; e += 32) write_edge(a, cc, keys[e], p0 + e, srec);
   return st;
 }
 
@@ -735,11 +871,13 @@ __global__ void __launch_bounds__(kFillWarps * 32) k_fill(BuildArgs a) {
 // image offset T L already added.  A candidate then costs one 16-byte
 // shared load and a few fp32 operations; only candidates within the margin
 // of rcut^2 (r2lo <= r2f <= r2hi) take the exact fp64 test, so the accept
-// decision is the fp64 one bit for bit.  Cells whose stencil holds more than
-// kCellCand atoms fall back to the per-centre traversal of global memory.
-
+// decision is the fp64 one bit for bit.  With REC the candidates' exact
+// records are staged too, so the fp64 tests and the edge output read shared
+// memory only.  Cells whose stencil holds more than kCellCand atoms fall back
+// to the per-centre traversal of global memory.
 constexpr int kCellCand = 768;
 constexpr int kCellWarps = 8;
+static_assert(kCellCand <= 1024, "staged_key keeps 10 bits of slot");
 
 struct CellStage {
   int pre[33];      // candidate offset of each stencil cell
@@ -748,102 +886,148 @@ struct CellStage {
   int ncand;
   int fallback;
   int trunc;
+  int staged_cell;          // cell whose candidates the arrays hold (-1: none)
+  int self_pre;             // first slot of the cell's own (zero-image) stencil entry
+  int stash_ci[kCellWarps];   // STASH: centre whose accepted keys a warp still holds (-1: none)
+  int stash_cnt[kCellWarps];  // and how many
   float4 cand[kCellCand];   // position + image offset, atom index in .w
   int cq[kCellCand];        // cell-order index (record of the exact data)
   int ct[kCellCand];        // packed image of the stencil cell
 };
 
-template <bool FILL>
-__global__ void __launch_bounds__(kCellWarps * 32, 2) k_cellscan(BuildArgs a) {
-  __shared__ CellGrid sg;
-  __shared__ WarpScratch sws[kCellWarps];
-  extern __shared__ __align__(16) unsigned char s_dyn[];
+// Dynamic shared memory of the per-cell scans: the stage, the fill's key
+// buffers, and (REC) the candidates' exact records.
+constexpr size_t kCellKeysOff = ((sizeof(CellStage) + 15) / 16) * 16;
+constexpr size_t kCellKeysBytes = (size_t)kCellWarps * 2 * kFillMaxCand * sizeof(unsigned long long);
+constexpr size_t kCellRecOff = kCellKeysOff + kCellKeysBytes;
+__host__ __device__ constexpr size_t cellscan_smem(bool fill, bool rec = false) {
+  return rec ? kCellRecOff + (size_t)kCellCand * sizeof(Rec)
+             : kCellKeysOff + (fill ? kCellKeysBytes : 0);
+}
+
+// Count (FILL = false: raw, kept, truncations) or fill (FILL: the CSR rows)
+// of the centres of `cell` taken by split `ys` of `nsplit` (centres
+// c_lo + ys * kCellWarps + warp, stepping by nsplit * kCellWarps).  Called by
+// every thread of the CTA.  Row starts come from row_off (tile-local copy of
+// row_ptr, indexed by centre) or else from a.row_ptr.  Staged candidates of
+// the same cell from an earlier call are reused.  With STASH (and REC) the
+// count keeps each warp's accepted keys and distances in its key buffer, and
+// a fill of the same centre by the same warp starts from them.
+template <bool FILL, bool REC, bool STASH = false>
+__device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratch* sws,
+                              unsigned char* s_dyn, int cell, int ys, int nsplit,
+                              const int* row_off) {
   CellStage& cs = *reinterpret_cast<CellStage*>(s_dyn);
-  unsigned long long* s_keys =
-      reinterpret_cast<unsigned long long*>(s_dyn + ((sizeof(CellStage) + 15) / 16) * 16);
+  unsigned long long* s_keys = reinterpret_cast<unsigned long long*>(s_dyn + kCellKeysOff);
+  Rec* s_rec = reinterpret_cast<Rec*>(s_dyn + kCellRecOff);  // REC only
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) sg = *a.grid;
-  __syncthreads();
-  // blockIdx.y splits a cell's centres over several CTAs (small grids)
-  const int cell = blockIdx.x;
   if (cell >= sg.ncell) return;
   const int c_lo = a.cell_start[cell], c_hi = a.cell_start[cell + 1];
-  if (c_lo + (int)blockIdx.y * kCellWarps >= c_hi) return;
+  if (c_lo + ys * kCellWarps >= c_hi) return;
   const int cz = cell % sg.n[2], cy = (cell / sg.n[2]) % sg.n[1], cx = cell / (sg.n[2] * sg.n[1]);
-  if (warp == 0) {
-    // stencil (reach <= 1 on every axis: at most 27 cells)
-    const int w0 = 2 * sg.D[0] + 1, w1 = 2 * sg.D[1] + 1, w2 = 2 * sg.D[2] + 1;
-    const int s3 = w0 * w1 * w2;
-    int len = 0, start = 0, tp = 0;
-    if (lane < s3) {
-      int d[3];
-      d[2] = lane % w2 - sg.D[2];
-      d[1] = (lane / w2) % w1 - sg.D[1];
-      d[0] = lane / (w2 * w1) - sg.D[0];
-      const int c[3] = {cx, cy, cz};
-      int m[3], T[3];
-      bool ok = true;
+  if (cs.staged_cell != cell) {
+    __syncthreads();  // earlier readers of the staging arrays are done
+    if (warp == 0) {
+      // stencil (reach <= 1 on every axis: at most 27 cells)
+      const int w0 = 2 * sg.D[0] + 1, w1 = 2 * sg.D[1] + 1, w2 = 2 * sg.D[2] + 1;
+      const int s3 = w0 * w1 * w2;
+      int len = 0, start = 0, tp = 0;
+      if (lane < s3) {
+        int d[3];
+        d[2] = lane % w2 - sg.D[2];
+        d[1] = (lane / w2) % w1 - sg.D[1];
+        d[0] = lane / (w2 * w1) - sg.D[0];
+        const int c[3] = {cx, cy, cz};
+        int m[3], T[3];
+        bool ok = true;
 #pragma unroll
-      for (int k = 0; k < 3; ++k) {
-        int e = c[k] + d[k];
-        if (sg.periodic[k]) {
-          T[k] = floordiv(e, sg.n[k]);
-          m[k] = e - T[k] * sg.n[k];
-        } else {
-          ok = ok && e >= 0 && e < sg.n[k];
-          m[k] = e;
-          T[k] = 0;
+        for (int k = 0; k < 3; ++k) {
+          int e = c[k] + d[k];
+          if (sg.periodic[k]) {
+            T[k] = floordiv(e, sg.n[k]);
+            m[k] = e - T[k] * sg.n[k];
+          } else {
+            ok = ok && e >= 0 && e < sg.n[k];
+            m[k] = e;
+            T[k] = 0;
+          }
+        }
+        if (ok) {
+          int cc = (m[0] * sg.n[1] + m[1]) * sg.n[2] + m[2];
+          start = a.cell_start[cc];
+          len = a.cell_start[cc + 1] - start;
+          tp = ((T[0] + 64) << 14) | ((T[1] + 64) << 7) | (T[2] + 64);
         }
       }
-      if (ok) {
-        int cc = (m[0] * sg.n[1] + m[1]) * sg.n[2] + m[2];
-        start = a.cell_start[cc];
-        len = a.cell_start[cc + 1] - start;
-        tp = ((T[0] + 64) << 14) | ((T[1] + 64) << 7) | (T[2] + 64);
+      int incl = warp_incl_scan(len);
+      cs.pre[lane] = incl - len;
+      cs.start[lane] = start;
+      cs.tpack[lane] = tp;
+      if (lane == (sg.D[0] * w1 + sg.D[1]) * w2 + sg.D[2]) cs.self_pre = incl - len;
+      if (lane == 31) {
+        cs.pre[32] = incl;
+        cs.ncand = incl;
+        cs.fallback = incl > kCellCand;
+        cs.trunc = 0;
+        cs.staged_cell = cell;
       }
     }
-    int incl = warp_incl_scan(len);
-    cs.pre[lane] = incl - len;
-    cs.start[lane] = start;
-    cs.tpack[lane] = tp;
-    if (lane == 31) {
-      cs.pre[32] = incl;
-      cs.ncand = incl;
-      cs.fallback = incl > kCellCand;
-      cs.trunc = 0;
+    if (STASH && tid < kCellWarps) cs.stash_ci[tid] = -1;  // stashed slots refer to the old staging
+    __syncthreads();
+    if (!cs.fallback) {
+      // stage the candidates: slot t of stencil cell s (pre[s] <= t <
+      // pre[s + 1]); two slots per thread and round, loads first
+      const int K = cs.ncand;
+      constexpr int NT = kCellWarps * 32;
+      for (int t0 = tid; t0 < K; t0 += 2 * NT) {
+        int q[2], tp[2];
+        float4 pv[2];
+        Rec rv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int t = t0 + u * NT;
+          q[u] = -1;
+          if (t < K) {
+            int lo = 0, hi = 31;  // largest s with pre[s] <= t
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (cs.pre[mid] <= t) lo = mid; else hi = mid - 1;
+            }
+            q[u] = cs.start[lo] + (t - cs.pre[lo]);
+            tp[u] = cs.tpack[lo];
+            pv[u] = a.pos4[q[u]];
+            if (REC) rv[u] = a.recs[q[u]];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (q[u] < 0) continue;
+          const int t = t0 + u * NT;
+          float4 p = pv[u];
+          p.x += (float)(((tp[u] >> 14) & 127) - 64) * sg.Lf[0];
+          p.y += (float)(((tp[u] >> 7) & 127) - 64) * sg.Lf[1];
+          p.z += (float)((tp[u] & 127) - 64) * sg.Lf[2];
+          cs.cand[t] = p;
+          cs.cq[t] = q[u];
+          cs.ct[t] = tp[u];
+          if (REC) s_rec[t] = rv[u];
+        }
+      }
     }
+    __syncthreads();
+  } else if (!FILL && threadIdx.x == 0) {
+    cs.trunc = 0;
   }
-  __syncthreads();
+  if (!FILL) __syncthreads();
   const int K = cs.ncand;
-  if (!cs.fallback) {
-    // stage the candidates: warp w copies stencil cells w, w + 8, ...
-    for (int sidx = warp; sidx < 32; sidx += kCellWarps) {
-      const int len = cs.pre[sidx + 1] - cs.pre[sidx];
-      if (len == 0) continue;
-      const int tp = cs.tpack[sidx];
-      const float ox = (float)(((tp >> 14) & 127) - 64) * sg.Lf[0];
-      const float oy = (float)(((tp >> 7) & 127) - 64) * sg.Lf[1];
-      const float oz = (float)((tp & 127) - 64) * sg.Lf[2];
-      for (int t = lane; t < len; t += 32) {
-        const int q = cs.start[sidx] + t;
-        float4 p = a.pos4[q];
-        p.x += ox;
-        p.y += oy;
-        p.z += oz;
-        const int dst = cs.pre[sidx] + t;
-        cs.cand[dst] = p;
-        cs.cq[dst] = q;
-        cs.ct[dst] = tp;
-      }
-    }
-  }
-  __syncthreads();
   const int self_tp = (64 << 14) | (64 << 7) | 64;
   unsigned long long* keys = s_keys + (size_t)warp * 2 * kFillMaxCand;
   uint32_t st = 0;
-  for (int ci = c_lo + blockIdx.y * kCellWarps + warp; ci < c_hi;
-       ci += gridDim.y * kCellWarps) {
-    const Rec rci = a.recs[ci];
+  for (int ci = c_lo + ys * kCellWarps + warp; ci < c_hi; ci += nsplit * kCellWarps) {
+    // the centre's own record: staged (self stencil cell) or global
+    const int self_slot = cs.self_pre + (ci - c_lo);
+    const bool staged_self = REC && !cs.fallback;
+    const Rec rci = staged_self ? s_rec[self_slot] : a.recs[ci];
     const int i = rci.j;
     Centre cc;
     cc.i = i;
@@ -855,6 +1039,7 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2) k_cellscan(BuildArgs a) {
     cc.c[0] = cx;
     cc.c[1] = cy;
     cc.c[2] = cz;
+    const int64_t p0 = FILL ? (row_off != nullptr ? (int64_t)row_off[i] : a.row_ptr[i]) : 0;
     if (cs.fallback) {
       if (!FILL) {
         int cnt = 0;
@@ -873,20 +1058,30 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2) k_cellscan(BuildArgs a) {
       } else {
         const int n = a.kept[i];
         if (n > 0)
-          st |= fill_row_global(a, sg, cc, sws[warp], keys, keys + kFillMaxCand, n, a.raw[i],
-                                a.row_ptr[i]);
+          st |= fill_row_global(a, sg, cc, sws[warp], keys, keys + kFillMaxCand, n, a.raw[i], p0);
       }
       continue;
     }
-    const float4 pi = a.pos4[ci];
     const int n = FILL ? a.kept[i] : 0;
     if (FILL && n == 0) continue;
+    if (FILL && STASH && cs.stash_ci[warp] == ci) {
+      // the count pass left this centre's accepted keys and distances here
+      st |= finish_row(a, cc, keys, keys + kFillMaxCand, n, cs.stash_cnt[warp], p0, s_rec);
+      continue;
+    }
+    if (STASH) {
+      __syncwarp();
+      if (lane == 0) cs.stash_ci[warp] = -1;  // the key buffer is about to be overwritten
+    }
+    const float4 pi = staged_self ? cs.cand[self_slot] : a.pos4[ci];
     const bool need_d2 = FILL && a.raw[i] > n;
+    constexpr bool kCollect = FILL || STASH;
     int cnt = 0;
     for (int base = 0; base < K; base += 32) {
       const int t = base + lane;
       bool acc = false;
-      int tp = 0, q = 0, j = -1;
+      double r2 = 0.0;
+      int tp = 0, j = -1;
       if (t < K) {
         const float4 c4 = cs.cand[t];
         const float dx = c4.x - pi.x, dy = c4.y - pi.y, dz = c4.z - pi.z;
@@ -896,21 +1091,18 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2) k_cellscan(BuildArgs a) {
         if (r2f < sg.r2lo) {
           acc = !(j == i && tp == self_tp);
         } else if (r2f <= sg.r2hi) {
-          double r2;
-          q = cs.cq[t];
-          acc = test_candidate(sg, cc, a.recs[q], tp, a.rc2, &r2);
+          acc = test_candidate(sg, cc, REC ? s_rec[t] : a.recs[cs.cq[t]], tp, a.rc2, &r2);
         }
       }
-      if (!FILL) {
+      if (!kCollect) {
         cnt += acc ? 1 : 0;
       } else {
         const unsigned m = __ballot_sync(kFull, acc);
         if (acc) {
           const int qd = cnt + __popc(m & lanemask_lt());
           if (qd < kFillMaxCand) {
-            keys[qd] = edge_key(j, tp);
-            if (need_d2) {
-              double r2;
+            keys[qd] = REC ? staged_key(j, tp, t) : edge_key(j, tp);
+            if (!REC && need_d2) {
               test_candidate(sg, cc, a.recs[cs.cq[t]], tp, a.rc2, &r2);
               keys[kFillMaxCand + qd] = (unsigned long long)__double_as_longlong(r2);
             }
@@ -919,21 +1111,36 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2) k_cellscan(BuildArgs a) {
         cnt += __popc(m);
       }
     }
+    if (REC && kCollect && (FILL ? need_d2 : cnt > a.nnei_max) && cnt <= kFillMaxCand) {
+      // exact distances of a truncated row's accepted candidates, after the
+      // scan (their slots are in the keys)
+      __syncwarp();
+      for (int q = lane; q < cnt; q += 32) {
+        const unsigned long long key = keys[q];
+        double r2;
+        test_candidate(sg, cc, s_rec[key & 1023ull], (int)((key >> 10) & 0x1fffffull), a.rc2,
+                       &r2);
+        keys[kFillMaxCand + q] = (unsigned long long)__double_as_longlong(r2);
+      }
+    }
     if (!FILL) {
-      cnt = warp_sum(cnt);
+      if (!kCollect) cnt = warp_sum(cnt);  // collecting lanes hold the warp total already
       if (lane == 0) {
         a.raw[i] = cnt;
         a.kept[i] = cnt < a.nnei_max ? cnt : a.nnei_max;
         if (cnt > a.nnei_max) atomicAdd(&cs.trunc, 1);
+        if (STASH && cnt <= kFillMaxCand) {
+          cs.stash_ci[warp] = ci;
+          cs.stash_cnt[warp] = cnt;
+        }
       }
     } else {
       __syncwarp();
       if (cnt > kFillMaxCand) {
         // more candidates than a warp holds: threshold search from global memory
-        st |= fill_row_global(a, sg, cc, sws[warp], keys, keys + kFillMaxCand, n, cnt,
-                              a.row_ptr[i]);
+        st |= fill_row_global(a, sg, cc, sws[warp], keys, keys + kFillMaxCand, n, cnt, p0);
       } else {
-        st |= finish_row(a, cc, keys, keys + kFillMaxCand, n, cnt, a.row_ptr[i]);
+        st |= finish_row(a, cc, keys, keys + kFillMaxCand, n, cnt, p0, REC ? s_rec : nullptr);
       }
     }
   }
@@ -947,9 +1154,18 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2) k_cellscan(BuildArgs a) {
   }
 }
 
-inline size_t cellscan_smem(bool fill) {
-  size_t base = ((sizeof(CellStage) + 15) / 16) * 16;
-  return base + (fill ? (size_t)kCellWarps * 2 * kFillMaxCand * sizeof(unsigned long long) : 0);
+template <bool FILL>
+__global__ void __launch_bounds__(kCellWarps * 32, FILL ? 3 : 4) k_cellscan(BuildArgs a) {
+  __shared__ CellGrid sg;
+  __shared__ WarpScratch sws[kCellWarps];
+  extern __shared__ __align__(16) unsigned char s_dyn[];
+  if (threadIdx.x == 0) {
+    sg = *a.grid;
+    reinterpret_cast<CellStage*>(s_dyn)->staged_cell = -1;
+  }
+  __syncthreads();
+  // blockIdx.y splits a cell's centres over several CTAs (small grids)
+  cellscan_item<FILL, false>(a, sg, sws, s_dyn, blockIdx.x, blockIdx.y, gridDim.y, nullptr);
 }
 
 // ------------------------------------------------------------------ scans
@@ -1000,13 +1216,12 @@ struct ScanTail {
   int64_t capacity;
 };
 
-// One block: tiles of 1024 x 4 items, each thread a contiguous int4, carry
-// from tile to tile.
+// One block: tiles of blockDim.x x 4 items, each thread 4 contiguous items,
+// carry from tile to tile.  Called by every thread of the block.
 template <typename TOut>
-__global__ void __launch_bounds__(1024) k_scan_single(const int* in, int64_t n, TOut* out,
-                                                      ScanTail tail) {
+__device__ void scan_block(const int* in, int64_t n, TOut* out, ScanTail tail) {
   long long carry = 0;
-  for (int64_t base = 0; base < n; base += 4096) {
+  for (int64_t base = 0; base < n; base += 4 * (int64_t)blockDim.x) {
     const int64_t t0 = base + 4 * (int64_t)threadIdx.x;
     int v[4];
 #pragma unroll
@@ -1028,6 +1243,12 @@ __global__ void __launch_bounds__(1024) k_scan_single(const int* in, int64_t n, 
       if (carry > tail.capacity) atomicOr(tail.status, (uint32_t)MLG_STATUS_CAPACITY);
     }
   }
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(1024) k_scan_single(const int* in, int64_t n, TOut* out,
+                                                      ScanTail tail) {
+  scan_block<TOut>(in, n, out, tail);
 }
 
 __global__ void __launch_bounds__(kScanThreads) k_scan_reduce(const int* in, int64_t n,
@@ -1094,6 +1315,163 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_down(const int* in, int64
       if (total > tail.capacity) atomicOr(tail.status, (uint32_t)MLG_STATUS_CAPACITY);
     }
   }
+}
+
+// ------------------------------------------------------- one-launch build
+//
+// Small systems (n <= kFusedMaxAtoms, per-cell scans): the whole build in one
+// cooperative launch, where the chain of small kernels above would be bound
+// by launch latency.  CTA 0 alone bins the atoms (init, bounding box, cell
+// histogram, cell scan, scatter) and then releases a flag; every CTA counts
+// its (cell, split) items; a grid barrier; every CTA scans the kept counts
+// into shared memory for its row starts (CTA 0 also writes row_ptr, n_edges
+// and the capacity check) and fills its items, reusing the staged candidates
+// of a cell it has just counted.  Both waits are bounded: a CTA whose wait
+// runs out sets MLG_STATUS_TIMEOUT and leaves, which ends the others' waits
+// the same way.  The launch is cooperative, so every CTA is resident.
+constexpr int kFusedMaxAtoms = 4096;
+constexpr long long kFusedSpinLimit = 1ll << 21;  // polls, 256 ns apart: a second or two
+
+struct FusedSync {
+  unsigned int ready;    // 1 once CTA 0 has binned the atoms
+  unsigned int arrived;  // CTAs done with the count pass
+};                       // zeroed by the host before each launch
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// polls until *p >= want; false if the limit ran out first
+__device__ __forceinline__ bool wait_at_least(const unsigned* p, unsigned want) {
+  for (long long it = 0; it < kFusedSpinLimit; ++it) {
+    if (ld_acquire_gpu(p) >= want) return true;
+    __nanosleep(256);
+  }
+  return false;
+}
+
+// Dynamic shared memory of the one-launch build: the per-cell scan's, then
+// the row starts; CTA 0's binning scratch (histogram and three per-atom
+// arrays) must fit in the same bytes.
+__host__ __device__ constexpr size_t fused_build_smem(int64_t n) {
+  return cellscan_smem(true, true) + (size_t)(n + 1) * sizeof(int);
+}
+__host__ __device__ constexpr bool fused_build_fits(int64_t n, int ncell_cap) {
+  return (size_t)(ncell_cap + 1 + 3 * n) * sizeof(int) <= fused_build_smem(n);
+}
+
+__global__ void __launch_bounds__(kCellWarps * 32, 2)
+    k_build_fused(BuildArgs a, BuildPlan p, int ncell_cap, int nsplit, FusedSync* sync) {
+  __shared__ CellGrid sg;
+  __shared__ WarpScratch sws[kCellWarps];
+  __shared__ int s_ok;
+  extern __shared__ __align__(16) unsigned char s_dyn[];
+  int* s_off = reinterpret_cast<int*>(s_dyn + cellscan_smem(true, true));  // [n + 1] row starts
+  const int tid = threadIdx.x;
+  const unsigned tout = MLG_STATUS_TIMEOUT;
+
+  if (blockIdx.x == 0) {
+    // ---- binning, by this CTA alone, with its shared memory as scratch:
+    // cell histogram (then starts), and each atom's cell, rank and image
+    int* s_hist = reinterpret_cast<int*>(s_dyn);  // [ncell_cap + 1]
+    int* s_cell = s_hist + ncell_cap + 1;          // [n]
+    int* s_rank = s_cell + a.n;                    // [n]
+    int* s_w = s_rank + a.n;                       // [n]
+    for (int m = tid; m <= ncell_cap; m += blockDim.x) s_hist[m] = 0;
+    if (tid < 3) {
+      a.bbox[tid] = ~0ull;
+      a.bbox[3 + tid] = 0ull;
+    }
+    if (tid == 0) {
+      *a.n_truncated = 0;
+      *a.status = 0u;
+    }
+    __syncthreads();
+    if (p.any_open) {
+      bbox_accumulate(a, p, tid, blockDim.x);
+      __syncthreads();
+    }
+    if (tid == 0) {
+      sg = derive_grid(p, a.bbox);
+      *a.grid = sg;
+    }
+    __syncthreads();
+    for (int64_t base = 0; base < a.n; base += blockDim.x)
+      bin_atom(a, sg, base + tid, s_hist, s_rank, s_cell, s_w);
+    __syncthreads();
+    // cell starts: exclusive scan of the histogram, contiguous chunks per thread
+    {
+      const int per = (ncell_cap + (int)blockDim.x - 1) / (int)blockDim.x;
+      const int m0 = tid * per, m1 = min(m0 + per, ncell_cap);
+      int sum = 0;
+      for (int m = m0; m < m1; ++m) sum += s_hist[m];
+      int total;
+      int off = block_excl_scan<int>(sum, &total);
+      for (int m = m0; m < m1; ++m) {
+        const int c = s_hist[m];
+        s_hist[m] = off;
+        a.cell_start[m] = off;
+        off += c;
+      }
+      if (tid == 0) {
+        s_hist[ncell_cap] = total;
+        a.cell_start[ncell_cap] = total;
+      }
+    }
+    __syncthreads();
+    for (int64_t i = tid; i < a.n; i += blockDim.x) {
+      const int cell = s_cell[i];
+      if (cell >= 0) scatter_atom_at(a, sg, i, s_hist[cell] + s_rank[i], s_w[i]);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      st_release_gpu(&sync->ready, 1u);
+    }
+  }
+  if (tid == 0) {
+    s_ok = blockIdx.x == 0 ? 1 : (wait_at_least(&sync->ready, 1u) ? 1 : 0);
+    if (s_ok && blockIdx.x != 0) sg = *a.grid;
+    reinterpret_cast<CellStage*>(s_dyn)->staged_cell = -1;
+  }
+  __syncthreads();
+  if (!s_ok) {
+    if (tid == 0) atomicOr(a.status, tout);
+    return;
+  }
+
+  // ---- count pass (keys kept for the fill)
+  const int nitems = sg.ncell * nsplit;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x)
+    cellscan_item<false, true, true>(a, sg, sws, s_dyn, item / nsplit, item % nsplit, nsplit,
+                                     nullptr);
+
+  // ---- grid barrier: every count is written
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(&sync->arrived, 1u);
+    s_ok = wait_at_least(&sync->arrived, gridDim.x) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!s_ok) {
+    if (tid == 0) atomicOr(a.status, tout);
+    return;
+  }
+
+  // ---- row starts of every centre, then the fill pass
+  scan_block<int>(a.kept, a.n, s_off, ScanTail{nullptr, nullptr, 0});
+  if (blockIdx.x == 0)
+    scan_block<long long>(a.kept, a.n, reinterpret_cast<long long*>(a.row_ptr),
+                          ScanTail{a.n_edges, a.status, a.capacity});
+  __syncthreads();
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x)
+    cellscan_item<true, true, true>(a, sg, sws, s_dyn, item / nsplit, item % nsplit, nsplit,
+                                    s_off);
 }
 
 }  // namespace mlg

@@ -10,6 +10,8 @@
 //   Q_h [16][8]    = X . Wq_h             m16n8k16, kept in registers
 //   S   [16][8]    = Q_h . K_h^T          m16n8k8 per 8-key block
 //   O   [16][8]   += P . V_h              m16n8k8 per 8-key block
+// A centre's last query rows, when 8 or fewer, take the same three products
+// on 8-row blocks (m8n8k4), so no MMA row is padding.
 // A contraction may visit its k index in any order, so each one permutes it
 // to suit the fragments at hand: the projections read channel 4t + m at k
 // slot t + 4m (both operands then come in contiguous 16-byte pieces); the
@@ -33,6 +35,23 @@
 #include "mlg_attn_hg.cuh"
 
 namespace mlg {
+
+// C[8x8] += A[8x4] B[4x8] (fp64): lane (g, t) holds A(g, t), B(t, g) and
+// C(g, 2t), C(g, 2t + 1).
+__device__ __forceinline__ void dmma884(double& c0, double& c1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(c0), "+d"(c1)
+               : "d"(a), "d"(b));
+}
+
+// Query blocks of a centre with n edges: 16-row blocks (the last one may
+// be partial when more than 8 rows remain) and at most one final 8-row block.
+__host__ __device__ __forceinline__ int full_qblocks(int n) {
+  return n / 16 + (n % 16 > 8 ? 1 : 0);
+}
+__host__ __device__ __forceinline__ int half_qblocks(int n) {
+  return n % 16 != 0 && n % 16 <= 8 ? 1 : 0;
+}
 
 // C[16x8] += A[16x8] B[8x8] (fp64).  Lane (g, t) = (lane / 4, lane % 4) holds
 // a = {A(g,t), A(g+8,t), A(g,t+4), A(g+8,t+4)}, b = {B(t,g), B(t+4,g)},
@@ -139,7 +158,8 @@ struct DmmaCfg {
   static constexpr int XS = 34;      // row strides in doubles, chosen so that the
   static constexpr int KS = 40;      // 16-byte fragment loads and stores of every
   static constexpr int VS = RA;      // phase are free of bank conflicts
-  static constexpr int WS = 3 * C + 2;  // W rows: == 2 (mod 4) doubles, 16-byte multiple
+  static constexpr int WS = 3 * C + 1;  // W rows: odd, so 8-byte fragment loads of rows 4t + i
+                                        // fill a half-warp's banks once
   static constexpr size_t XBYTES = (size_t)RA * XS * 8;
   static constexpr size_t OFF_X = 0;                               // [2][RA][XS]
   static constexpr size_t OFF_K = OFF_X + 2 * XBYTES;              // [RA][KS]
@@ -189,16 +209,179 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
   __syncthreads();
 
   // weights: sW[k][m C + col] = W_m[k][col] (m = 0, 1, 2: q, k, v), copied
-  // by 16-byte async copies; a layer's q block and its k, v blocks are
-  // copied at different times (see the layer loop)
+  // by 8-byte async copies (the row stride is odd); a layer's q block and its
+  // k, v blocks are copied at different times (see the layer loop)
   auto load_w = [&](int layer, int m0, int nm) {
-    for (int e = tid; e < nm * C * (C / 2); e += NT) {
-      const int m = m0 + e / (C * (C / 2)), rem = e % (C * (C / 2));
-      const int k = rem / (C / 2), v = rem % (C / 2);
-      cp_async16(sW + k * WS + m * C + 2 * v,
-                 static_cast<const double*>(a.W[3 * layer + m]) + k * C + 2 * v);
+    for (int e = tid; e < nm * C * C; e += NT) {
+      const int m = m0 + e / (C * C), rem = e % (C * C);
+      const int k = rem / C, col = rem % C;
+      cp_async8(sW + k * WS + m * C + col,
+                static_cast<const double*>(a.W[3 * layer + m]) + k * C + col);
     }
     cp_async_commit();
+  };
+
+  // Attention of query rows qb * 16 .. + 15 of the centre at tile row `off`
+  // (n edges, nkb key blocks), head h: X from sX, output rows to sXn.
+  auto attend16 = [&](const double* sX, double* sXn, int off, int n, int nkb, int qb, int h) {
+    const int q0 = off + qb * 16;          // first query row of the block (tile-local)
+    const bool hi_rows = qb * 16 + 8 < n;  // rows g + 8 hold queries
+    // Q_h of the block: q[e] = Q(g, 2t + e), q[2 + e] = Q(g + 8, 2t + e)
+    double q[4] = {0.0, 0.0, 0.0, 0.0};
+    {
+      const double* xr = sX + (q0 + g) * XS + 4 * t;
+      const double* wr = sW + 4 * t * WS + h * D + g;
+#pragma unroll
+      for (int k0 = 0; k0 < C; k0 += 16) {
+        double av[8], bv[4];
+        frag_a16(av, xr + k0, XS);
+        frag_bw(bv, wr + k0 * WS, WS);
+        dmma_k16(q, av, bv);
+      }
+      const double f0 = sS[q0 + g] * qscale, f1 = sS[q0 + g + 8] * qscale;
+      q[0] *= f0;
+      q[1] *= f0;
+      q[2] *= f1;
+      q[3] *= f1;
+    }
+    // logits against the centre's keys (base-2 units):
+    // s[j][e] = S(g, 8j + 2t + e), s[j][2 + e] = S(g + 8, 8j + 2t + e)
+    double s[NBC][4];
+#pragma unroll
+    for (int j = 0; j < NBC; ++j) {
+      s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0;
+      if (j < nkb) {
+        const double2 kv = lds2(sK + (off + 8 * j + g) * KS + h * D + 2 * t);
+        dmma_k8(s[j], q[0], q[2], q[1], q[3], kv.x, kv.y);
+      }
+    }
+    double m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NBC; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool valid = j < nkb && 8 * j + 2 * t + e < n;
+        s[j][e] = valid ? s[j][e] : -INFINITY;
+        s[j][2 + e] = valid ? s[j][2 + e] : -INFINITY;
+        m0 = fmax(m0, s[j][e]);
+        m1 = fmax(m1, s[j][2 + e]);
+      }
+    m0 = fmax(m0, __shfl_xor_sync(kFull, m0, 1));
+    m0 = fmax(m0, __shfl_xor_sync(kFull, m0, 2));
+    m1 = fmax(m1, __shfl_xor_sync(kFull, m1, 1));
+    m1 = fmax(m1, __shfl_xor_sync(kFull, m1, 2));
+    double l0 = 0.0, l1 = 0.0;
+#pragma unroll
+    for (int j = 0; j < NBC; ++j) {
+      if (j < nkb) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          s[j][e] = exp2_neg(s[j][e] - m0, tab);
+          l0 += s[j][e];
+          if (hi_rows) {
+            s[j][2 + e] = exp2_neg(s[j][2 + e] - m1, tab);
+            l1 += s[j][2 + e];
+          } else {
+            s[j][2 + e] = 0.0;
+          }
+        }
+      }
+    }
+    l0 += __shfl_xor_sync(kFull, l0, 1);
+    l0 += __shfl_xor_sync(kFull, l0, 2);
+    l1 += __shfl_xor_sync(kFull, l1, 1);
+    l1 += __shfl_xor_sync(kFull, l1, 2);
+    // O = P V_h over two accumulator chains (even / odd key blocks)
+    double o[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
+#pragma unroll
+    for (int j = 0; j < NBC; ++j) {
+      if (j < nkb) {
+        const double2 vv = lds2(sV + (h * D + g) * VS + off + 8 * j + 2 * t);
+        dmma_k8(o[j & 1], s[j][0], s[j][2], s[j][1], s[j][3], vv.x, vv.y);
+      }
+    }
+    const int r = qb * 16 + g;
+    if (r < n) {
+      const double i0 = 1.0 / l0;
+      sts2(sXn + (q0 + g) * XS + h * D + 2 * t, (o[0][0] + o[1][0]) * i0,
+           (o[0][1] + o[1][1]) * i0);
+    }
+    if (r + 8 < n) {
+      const double i1 = 1.0 / l1;
+      sts2(sXn + (q0 + g + 8) * XS + h * D + 2 * t, (o[0][2] + o[1][2]) * i1,
+           (o[0][3] + o[1][3]) * i1);
+    }
+  };
+  // The same for the 8 query rows qr .. qr + 7 of the centre (m8n8k4): the
+  // projection's step s reads channel 16 (s / 4) + 4t + s % 4 at k slot t, the
+  // logits and P V read dimension / key 2t + e at the k slot t of step e.
+  auto attend8 = [&](const double* sX, double* sXn, int off, int n, int nkb, int qr, int h) {
+    const int q0 = off + qr;
+    double qa[2] = {0.0, 0.0}, qb[2] = {0.0, 0.0};  // two chains: channels 0..15, 16..31
+    {
+      const double* xr = sX + (q0 + g) * XS + 4 * t;
+      const double* wr = sW + 4 * t * WS + h * D + g;
+#pragma unroll
+      for (int c16 = 0; c16 < C; c16 += 16) {
+        double* q = c16 ? qb : qa;
+        const double2 xa = lds2(xr + c16), xb = lds2(xr + c16 + 2);
+        dmma884(q[0], q[1], xa.x, wr[(c16 + 0) * WS]);
+        dmma884(q[0], q[1], xa.y, wr[(c16 + 1) * WS]);
+        dmma884(q[0], q[1], xb.x, wr[(c16 + 2) * WS]);
+        dmma884(q[0], q[1], xb.y, wr[(c16 + 3) * WS]);
+      }
+    }
+    const double f = sS[q0 + g] * qscale;
+    const double q0v = (qa[0] + qb[0]) * f, q1v = (qa[1] + qb[1]) * f;  // Q(g, 2t), Q(g, 2t + 1)
+    // s[j][e] = S(g, 8j + 2t + e)
+    double s[NBC][2];
+#pragma unroll
+    for (int j = 0; j < NBC; ++j) {
+      s[j][0] = s[j][1] = 0.0;
+      if (j < nkb) {
+        const double2 kv = lds2(sK + (off + 8 * j + g) * KS + h * D + 2 * t);
+        dmma884(s[j][0], s[j][1], q0v, kv.x);
+        dmma884(s[j][0], s[j][1], q1v, kv.y);
+      }
+    }
+    double m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NBC; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool valid = j < nkb && 8 * j + 2 * t + e < n;
+        s[j][e] = valid ? s[j][e] : -INFINITY;
+        m = fmax(m, s[j][e]);
+      }
+    m = fmax(m, __shfl_xor_sync(kFull, m, 1));
+    m = fmax(m, __shfl_xor_sync(kFull, m, 2));
+    double l = 0.0;
+#pragma unroll
+    for (int j = 0; j < NBC; ++j) {
+      if (j < nkb) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          s[j][e] = exp2_neg(s[j][e] - m, tab);
+          l += s[j][e];
+        }
+      }
+    }
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+    double o[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+#pragma unroll
+    for (int j = 0; j < NBC; ++j) {
+      if (j < nkb) {
+        const double2 vv = lds2(sV + (h * D + g) * VS + off + 8 * j + 2 * t);
+        dmma884(o[j & 1][0], o[j & 1][1], s[j][0], vv.x);
+        dmma884(o[j & 1][0], o[j & 1][1], s[j][1], vv.y);
+      }
+    }
+    if (qr + g < n) {
+      const double il = 1.0 / l;
+      sts2(sXn + (q0 + g) * XS + h * D + 2 * t, (o[0][0] + o[1][0]) * il,
+           (o[0][1] + o[1][1]) * il);
+    }
   };
 
   while (true) {
@@ -219,7 +402,7 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
         if (n > NBC * 8 || rows + n8 > R) break;
         meta.off[0][k] = rows;
         meta.task0[0][k] = tasks;
-        tasks += ((n + 15) / 16) * H;
+        tasks += H * full_qblocks(n) + (H / 2) * half_qblocks(n);
         rows += n8;
         ++k;
         ++c;
@@ -326,102 +509,22 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
       // their last reader)
       if (layer + 1 < a.n_layers) load_w(layer + 1, 1, 2);
 
-      // ---- phase B: tasks (centre, 16-row query block, head)
-      for (int task = warp; task < ntask; task += NW) {
+      // ---- phase B: units of equal work: (centre, 16-row query block, head),
+      // or two heads of a centre's final 8-row query block
+      for (int unit = warp; unit < ntask; unit += NW) {
         int ci = 0;
-        while (meta.task0[0][ci + 1] <= task) ++ci;
+        while (meta.task0[0][ci + 1] <= unit) ++ci;
         const int off = meta.off[0][ci];
         const int n = (int)(a.row_ptr[c0 + ci + 1] - a.row_ptr[c0 + ci]);
         const int nkb = (meta.off[0][ci + 1] - off) >> 3;
-        const int rel = task - meta.task0[0][ci];
-        const int qb = rel >> 2, h = rel & 3;
-        const int q0 = off + qb * 16;          // first query row of the block (tile-local)
-        const bool hi_rows = qb * 16 + 8 < n;  // rows g + 8 hold queries
-
-        // Q_h of the block: q[e] = Q(g, 2t + e), q[2 + e] = Q(g + 8, 2t + e)
-        double q[4] = {0.0, 0.0, 0.0, 0.0};
-        {
-          const double* xr = sX + (q0 + g) * XS + 4 * t;
-          const double* wr = sW + 4 * t * WS + h * D + g;
-#pragma unroll
-          for (int k0 = 0; k0 < C; k0 += 16) {
-            double av[8], bv[4];
-            frag_a16(av, xr + k0, XS);
-            frag_bw(bv, wr + k0 * WS, WS);
-            dmma_k16(q, av, bv);
-          }
-          const double f0 = sS[q0 + g] * qscale, f1 = sS[q0 + g + 8] * qscale;
-          q[0] *= f0;
-          q[1] *= f0;
-          q[2] *= f1;
-          q[3] *= f1;
-        }
-        // logits against the centre's keys (base-2 units):
-        // s[j][e] = S(g, 8j + 2t + e), s[j][2 + e] = S(g + 8, 8j + 2t + e)
-        double s[NBC][4];
-#pragma unroll
-        for (int j = 0; j < NBC; ++j) {
-          s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0;
-          if (j < nkb) {
-            const double2 kv = lds2(sK + (off + 8 * j + g) * KS + h * D + 2 * t);
-            dmma_k8(s[j], q[0], q[2], q[1], q[3], kv.x, kv.y);
-          }
-        }
-        double m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < NBC; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const bool valid = j < nkb && 8 * j + 2 * t + e < n;
-            s[j][e] = valid ? s[j][e] : -INFINITY;
-            s[j][2 + e] = valid ? s[j][2 + e] : -INFINITY;
-            m0 = fmax(m0, s[j][e]);
-            m1 = fmax(m1, s[j][2 + e]);
-          }
-        m0 = fmax(m0, __shfl_xor_sync(kFull, m0, 1));
-        m0 = fmax(m0, __shfl_xor_sync(kFull, m0, 2));
-        m1 = fmax(m1, __shfl_xor_sync(kFull, m1, 1));
-        m1 = fmax(m1, __shfl_xor_sync(kFull, m1, 2));
-        double l0 = 0.0, l1 = 0.0;
-#pragma unroll
-        for (int j = 0; j < NBC; ++j) {
-          if (j < nkb) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              s[j][e] = exp2_neg(s[j][e] - m0, tab);
-              l0 += s[j][e];
-              if (hi_rows) {
-                s[j][2 + e] = exp2_neg(s[j][2 + e] - m1, tab);
-                l1 += s[j][2 + e];
-              } else {
-                s[j][2 + e] = 0.0;
-              }
-            }
-          }
-        }
-        l0 += __shfl_xor_sync(kFull, l0, 1);
-        l0 += __shfl_xor_sync(kFull, l0, 2);
-        l1 += __shfl_xor_sync(kFull, l1, 1);
-        l1 += __shfl_xor_sync(kFull, l1, 2);
-        // O = P V_h over two accumulator chains (even / odd key blocks)
-        double o[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
-#pragma unroll
-        for (int j = 0; j < NBC; ++j) {
-          if (j < nkb) {
-            const double2 vv = lds2(sV + (h * D + g) * VS + off + 8 * j + 2 * t);
-            dmma_k8(o[j & 1], s[j][0], s[j][2], s[j][1], s[j][3], vv.x, vv.y);
-          }
-        }
-        const int r = qb * 16 + g;
-        if (r < n) {
-          const double i0 = 1.0 / l0;
-          sts2(sXn + (q0 + g) * XS + h * D + 2 * t, (o[0][0] + o[1][0]) * i0,
-               (o[0][1] + o[1][1]) * i0);
-        }
-        if (r + 8 < n) {
-          const double i1 = 1.0 / l1;
-          sts2(sXn + (q0 + g + 8) * XS + h * D + 2 * t, (o[0][2] + o[1][2]) * i1,
-               (o[0][3] + o[1][3]) * i1);
+        const int nf = full_qblocks(n);
+        const int rel = unit - meta.task0[0][ci];
+        if (rel < H * nf) {
+          attend16(sX, sXn, off, n, nkb, rel / H, rel % H);
+        } else {
+          const int h0 = 2 * (rel - H * nf);
+          attend8(sX, sXn, off, n, nkb, nf * 16, h0);
+          attend8(sX, sXn, off, n, nkb, nf * 16, h0 + 1);
         }
       }
       cp_async_wait<0>();

@@ -235,6 +235,14 @@ int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
                              const uint8_t pbc[3], int32_t nnei_max, int32_t channels,
                              int32_t heads, int32_t n_layers, mlg_dtype dtype);
 
+/* Diagnostics: out[i] = 2^y[i] for i < n, by the device exponential that
+ * the fp64 attention uses for its softmax weights (arguments y <= 0; -inf
+ * gives 0, NaN gives NaN, y < -1000 gives 0).  y and out: device arrays of n
+ * doubles.  For tests of that routine against the CUDA math library.
+ * Returns MLG_ERR_INVALID_ARG for null pointers with n > 0 or n < 0,
+ * MLG_ERR_CUDA if the launch fails. */
+int mlg_exp2_neg(const double* y, double* out, int64_t n, mlg_stream_t stream);
+
 /* A static string naming a host status code. */
 const char* mlg_status_string(int status);
 

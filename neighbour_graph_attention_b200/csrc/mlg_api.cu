@@ -721,6 +721,15 @@ const char* mlg_status_string(int status) {
   }
 }
 
+int mlg_exp2_neg(const double* y, double* out, int64_t n, mlg_stream_t stream) {
+  if (n < 0 || (n > 0 && (y == nullptr || out == nullptr))) return MLG_ERR_INVALID_ARG;
+  if (n == 0) return MLG_OK;
+  const int64_t blocks = (n + 255) / 256;
+  k_exp2_neg<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, (cudaStream_t)stream>>>(y, out,
+                                                                                          n);
+  return launch_status();
+}
+
 int mlg_version(void) { return 100; }
 
 }  // extern "C"

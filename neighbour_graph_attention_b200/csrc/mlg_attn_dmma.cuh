@@ -108,6 +108,18 @@ __device__ __forceinline__ double exp2_neg(double y, double tab) {
   return y < -1000.0 ? 0.0 : out;
 }
 
+// out[i] = exp2_neg(y[i]) (diagnostics); every lane of a warp takes part in
+// each round (the table shuffle), lanes past n on a dummy argument.
+__global__ void k_exp2_neg(const double* y, double* out, int64_t n) {
+  const double tab = exp2((double)(threadIdx.x & 31) / 32.0);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < n; base += stride) {
+    const int64_t i = base + threadIdx.x;
+    const double v = exp2_neg(i < n ? y[i] : 0.0, tab);
+    if (i < n) out[i] = v;
+  }
+}
+
 __device__ __forceinline__ double2 lds2(const double* p) {
   return *reinterpret_cast<const double2*>(p);
 }

@@ -888,6 +888,7 @@ struct CellStage {
   int trunc;
   int staged_cell;          // cell whose candidates the arrays hold (-1: none)
   int self_pre;             // first slot of the cell's own (zero-image) stencil entry
+  int c_lo, c_hi;           // the staged cell's centres (cell-order range)
   int stash_ci[kCellWarps];   // STASH: centre whose accepted keys a warp still holds (-1: none)
   int stash_cnt[kCellWarps];  // and how many
   float4 cand[kCellCand];   // position + image offset, atom index in .w
@@ -922,10 +923,12 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
   Rec* s_rec = reinterpret_cast<Rec*>(s_dyn + kCellRecOff);  // REC only
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (cell >= sg.ncell) return;
-  const int c_lo = a.cell_start[cell], c_hi = a.cell_start[cell + 1];
+  const bool reuse = cs.staged_cell == cell;
+  const int c_lo = reuse ? cs.c_lo : a.cell_start[cell];
+  const int c_hi = reuse ? cs.c_hi : a.cell_start[cell + 1];
   if (c_lo + ys * kCellWarps >= c_hi) return;
   const int cz = cell % sg.n[2], cy = (cell / sg.n[2]) % sg.n[1], cx = cell / (sg.n[2] * sg.n[1]);
-  if (cs.staged_cell != cell) {
+  if (!reuse) {
     __syncthreads();  // earlier readers of the staging arrays are done
     if (warp == 0) {
       // stencil (reach <= 1 on every axis: at most 27 cells)
@@ -970,6 +973,8 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
         cs.fallback = incl > kCellCand;
         cs.trunc = 0;
         cs.staged_cell = cell;
+        cs.c_lo = c_lo;
+        cs.c_hi = c_hi;
       }
     }
     if (STASH && tid < kCellWarps) cs.stash_ci[tid] = -1;  // stashed slots refer to the old staging
@@ -1062,13 +1067,15 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
       }
       continue;
     }
-    const int n = FILL ? a.kept[i] : 0;
-    if (FILL && n == 0) continue;
     if (FILL && STASH && cs.stash_ci[warp] == ci) {
       // the count pass left this centre's accepted keys and distances here
-      st |= finish_row(a, cc, keys, keys + kFillMaxCand, n, cs.stash_cnt[warp], p0, s_rec);
+      const int raw = cs.stash_cnt[warp];
+      const int n = raw < a.nnei_max ? raw : a.nnei_max;
+      if (n > 0) st |= finish_row(a, cc, keys, keys + kFillMaxCand, n, raw, p0, s_rec);
       continue;
     }
+    const int n = FILL ? a.kept[i] : 0;
+    if (FILL && n == 0) continue;
     if (STASH) {
       __syncwarp();
       if (lane == 0) cs.stash_ci[warp] = -1;  // the key buffer is about to be overwritten

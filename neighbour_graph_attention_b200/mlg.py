@@ -89,6 +89,8 @@ _lib.mlg_attention_stack.restype = ctypes.c_int
 _lib.mlg_attention_stack.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32, _c_i32,
                                      _c_i32, ctypes.c_int, ctypes.POINTER(_p), _p, _p, _p, _c_sz,
                                      _p]
+_lib.mlg_exp2_neg.restype = ctypes.c_int
+_lib.mlg_exp2_neg.argtypes = [_p, _p, _c_i64, _p]
 _lib.mlg_status_string.restype = ctypes.c_char_p
 _lib.mlg_status_string.argtypes = [ctypes.c_int]
 _lib.mlg_version.restype = ctypes.c_int
@@ -107,6 +109,15 @@ def lib() -> ctypes.CDLL:
 
 def mlg_status_string(code: int) -> str:
     return _lib.mlg_status_string(int(code)).decode()
+
+
+def mlg_exp2_neg(y, out, stream=None, check: bool = True) -> int:
+    """out = 2^y elementwise by the fp64 attention's device exponential
+    (diagnostics; y, out: device float64 tensors of equal length)."""
+    rc = _lib.mlg_exp2_neg(_ptr(y), _ptr(out), int(y.numel()), _stream_handle(stream))
+    if check and rc != MLG_OK:
+        raise MlgError(rc, "mlg_exp2_neg")
+    return rc
 
 
 def mlg_version() -> int:

@@ -230,3 +230,33 @@ def test_peaked_softmax_f64():
     assert int(csr_t.status.item()) == 0
     ok, err = U.attn_tolerance_ok(w, out, ref)
     assert ok, err
+
+
+def test_device_exp2_against_cuda():
+    """The fp64 softmax's table-driven 2^y (Tang's method) against CUDA's own
+    exp2 (torch on the GPU): relative error below 4e-15 on [-1000, 0], at the
+    table points k/32 and at the rounding midpoints between them; -inf -> 0,
+    NaN -> NaN, below -1000 -> 0."""
+    m = U.mlg()
+    rng = np.random.default_rng(3)
+    k = np.arange(0, 32001, dtype=np.float64)
+    y = np.concatenate([
+        np.linspace(-1000.0, 0.0, 1_000_001),
+        -rng.uniform(0.0, 1000.0, 200_000),
+        -rng.uniform(0.0, 1.0, 200_000),
+        -k / 32.0, -(k + 0.5) / 32.0,
+    ])
+    y = y[y >= -1000.0]
+    yd = torch.as_tensor(y, device="cuda")
+    out = torch.empty_like(yd)
+    m.mlg_exp2_neg(yd, out)
+    ref = torch.exp2(yd)
+    rel = ((out - ref).abs() / ref).max().item()
+    assert rel < 4e-15, rel
+    sp = torch.tensor([-np.inf, np.nan, -1000.5, -2000.0, 0.0, -0.0], dtype=torch.float64,
+                      device="cuda")
+    so = torch.empty_like(sp)
+    m.mlg_exp2_neg(sp, so)
+    so = so.cpu().numpy()
+    assert so[0] == 0.0 and np.isnan(so[1]) and so[2] == 0.0 and so[3] == 0.0
+    assert so[4] == 1.0 and so[5] == 1.0

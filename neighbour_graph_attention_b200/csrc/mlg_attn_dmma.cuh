@@ -77,47 +77,68 @@ __device__ __forceinline__ void dmma_k16(double (&c)[4], const double (&a)[8],
         "d"(b[0]), "d"(b[1]), "d"(b[2]), "d"(b[3]));
 }
 
-// 2^y for y <= 0 (-inf -> 0, NaN -> NaN), after P. T. P. Tang's table-driven
-// exponential (ACM TOMS 15(2), 1989), in base 2: k = rint(32 y),
-// r = y - k / 32 (exact, |r| <= 1/64), 2^y = 2^(k >> 5) 2^((k & 31) / 32) 2^r.
-// The 32 table values 2^(j/32) sit one per lane (`tab` in lane j) and come by
-// a shuffle; 2^r = exp(r ln 2) is its Taylor series to degree 5 (truncation
-// below 2.3e-15 relative, as |r ln 2| <= 0.0109).  Below y = -1000 the result
-// is 0 (the true value is below 1e-301); above it the scaling by 2^(k >> 5)
-// is an add to the exponent field that stays in the normal range.
+// 2^y for y <= 0, or slightly above (-inf -> 0, NaN -> NaN, +inf -> +inf), after P. T. P.
+// Tang's table-driven exponential (ACM TOMS 15(2), 1989), in base 2:
+// k = rint(1024 y), r = y - k / 1024 (exact, |r| <= 1/2048),
+// 2^y = 2^(k >> 10) 2^((k & 1023) / 1024) 2^r, with the 1024 values
+// 2^(j/1024) in a shared-memory table `tab` and 2^r = exp(r ln 2) by its
+// Taylor series to degree 3 (truncation below 5.6e-16 relative, as
+// |r ln 2| <= 3.4e-4).  Arguments whose high word lies below that of -1000
+// give 0 (the true value is below 1e-301); above that the scaling by
+// 2^(k >> 10) is an add to the exponent field that stays in the normal range.
+// Besides the table load, the only FP64-pipe work is six operations.
 namespace exp2tab {
+constexpr int kBits = 10, kSize = 1 << kBits;
 constexpr double kLn2 = 0.693147180559945309417232121458176568;
-constexpr double c1 = kLn2, c2 = c1 * kLn2 / 2, c3 = c2 * kLn2 / 3, c4 = c3 * kLn2 / 4,
-                 c5 = c4 * kLn2 / 5;
+constexpr double c1 = kLn2, c2 = c1 * kLn2 / 2, c3 = c2 * kLn2 / 3;
 constexpr double kRound = 6755399441055744.0;  // 1.5 * 2^52: adding it rounds to an integer
+constexpr unsigned kHiMinus1000 = 0xC08F4000u;  // high word of -1000.0
 }  // namespace exp2tab
 
-__device__ __forceinline__ double exp2_neg(double y, double tab) {
-  double kd = fma(y, 32.0, exp2tab::kRound);
+// fills tab[0 .. 1023] with 2^(j/1024), threads tid0, tid0 + stride, ...
+__device__ __forceinline__ void exp2_table_fill(double* tab, int tid0, int stride) {
+  for (int j = tid0; j < exp2tab::kSize; j += stride) tab[j] = exp2((double)j / exp2tab::kSize);
+}
+
+__device__ __forceinline__ double exp2_neg(double y, const double* tab) {
+  double kd = fma(y, (double)exp2tab::kSize, exp2tab::kRound);
   const int k = __double2loint(kd);
   kd -= exp2tab::kRound;
-  const double r = fma(kd, -1.0 / 32.0, y);
-  double p = exp2tab::c5;
-  p = fma(p, r, exp2tab::c4);
-  p = fma(p, r, exp2tab::c3);
+  const double r = fma(kd, -1.0 / exp2tab::kSize, y);
+  double p = exp2tab::c3;
   p = fma(p, r, exp2tab::c2);
   p = fma(p, r, exp2tab::c1);
   p = fma(p, r, 1.0);
-  const double v = __shfl_sync(kFull, tab, k & 31) * p;
-  const double out = __hiloint2double(__double2hiint(v) + ((k >> 5) << 20), __double2loint(v));
-  return y < -1000.0 ? 0.0 : out;
+  const double v = tab[k & (exp2tab::kSize - 1)] * p;
+  const double out =
+      __hiloint2double(__double2hiint(v) + ((k >> exp2tab::kBits) << 20), __double2loint(v));
+  const unsigned hy = (unsigned)__double2hiint(y);
+  double res = hy > exp2tab::kHiMinus1000 ? 0.0 : out;  // below -1000, and -inf: 0
+  if ((hy & 0x7ff00000u) == 0x7ff00000u && (hy != 0xfff00000u || __double2loint(y) != 0))
+    res = y;  // NaN and +inf give themselves
+  return res;
 }
 
-// out[i] = exp2_neg(y[i]) (diagnostics); every lane of a warp takes part in
-// each round (the table shuffle), lanes past n on a dummy argument.
+// Order-preserving integer image of a double's high word (sign folded), for
+// row maxima on the integer pipe; from_ord_hi inverts it with a zero low
+// word, which is within 2^-20 relative of the maximum: the softmax does not
+// depend on the shift, and the exponential takes arguments slightly above 0.
+__device__ __forceinline__ int ord_hi(double x) {
+  const int h = __double2hiint(x);
+  return h ^ ((h >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ double from_ord_hi(int o) {
+  return __hiloint2double(o ^ ((o >> 31) & 0x7fffffff), 0);
+}
+
+// out[i] = exp2_neg(y[i]) (diagnostics).
 __global__ void k_exp2_neg(const double* y, double* out, int64_t n) {
-  const double tab = exp2((double)(threadIdx.x & 31) / 32.0);
+  __shared__ double tab[exp2tab::kSize];
+  exp2_table_fill(tab, threadIdx.x, blockDim.x);
+  __syncthreads();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < n; base += stride) {
-    const int64_t i = base + threadIdx.x;
-    const double v = exp2_neg(i < n ? y[i] : 0.0, tab);
-    if (i < n) out[i] = v;
-  }
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    out[i] = exp2_neg(y[i], tab);
 }
 
 __device__ __forceinline__ double2 lds2(const double* p) {
@@ -178,7 +199,8 @@ struct DmmaCfg {
   static constexpr size_t OFF_V = OFF_K + (size_t)RA * KS * 8;     // [C][VS]  (V^T)
   static constexpr size_t OFF_W = OFF_V + (size_t)C * VS * 8;      // [C][WS]: [Wq | Wk | Wv]
   static constexpr size_t OFF_S = OFF_W + (size_t)C * WS * 8;      // [RA]
-  static constexpr size_t OFF_META = (OFF_S + (size_t)RA * 8 + 15) / 16 * 16;
+  static constexpr size_t OFF_T = (OFF_S + (size_t)RA * 8 + 15) / 16 * 16;  // exp2 table
+  static constexpr size_t OFF_META = OFF_T + (size_t)exp2tab::kSize * 8;
   static constexpr size_t SMEM = OFF_META + sizeof(TileMeta);
   static_assert(R % 16 == 0 && VS % 16 == 8 && NBC * 8 <= R && NT % 32 == 0, "shapes");
 };
@@ -195,6 +217,7 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
   double* sV = reinterpret_cast<double*>(smem + Cfg::OFF_V);
   double* sW = reinterpret_cast<double*>(smem + Cfg::OFF_W);
   double* sS = reinterpret_cast<double*>(smem + Cfg::OFF_S);
+  double* tab = reinterpret_cast<double*>(smem + Cfg::OFF_T);
   TileMeta& meta = *reinterpret_cast<TileMeta*>(smem + Cfg::OFF_META);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -216,7 +239,7 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
     meta.next_c = lb(r0);
     meta.c_end = blockIdx.x + 1 == gridDim.x ? (int)a.n_centres : lb(r1);
   }
-  const double tab = exp2((double)lane / 32.0);               // 2^(lane / 32)
+  exp2_table_fill(tab, tid, NT);
   const double qscale = 1.4426950408889634 / sqrt((double)D);  // log2(e) / sqrt(d)
   __syncthreads();
 
@@ -267,7 +290,7 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
         dmma_k8(s[j], q[0], q[2], q[1], q[3], kv.x, kv.y);
       }
     }
-    double m0 = -INFINITY, m1 = -INFINITY;
+    int o0 = INT_MIN, o1 = INT_MIN;  // row maxima, on the integer pipe
 #pragma unroll
     for (int j = 0; j < NBC; ++j)
 #pragma unroll
@@ -275,13 +298,14 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
         const bool valid = j < nkb && 8 * j + 2 * t + e < n;
         s[j][e] = valid ? s[j][e] : -INFINITY;
         s[j][2 + e] = valid ? s[j][2 + e] : -INFINITY;
-        m0 = fmax(m0, s[j][e]);
-        m1 = fmax(m1, s[j][2 + e]);
+        o0 = max(o0, ord_hi(s[j][e]));
+        o1 = max(o1, ord_hi(s[j][2 + e]));
       }
-    m0 = fmax(m0, __shfl_xor_sync(kFull, m0, 1));
-    m0 = fmax(m0, __shfl_xor_sync(kFull, m0, 2));
-    m1 = fmax(m1, __shfl_xor_sync(kFull, m1, 1));
-    m1 = fmax(m1, __shfl_xor_sync(kFull, m1, 2));
+    o0 = max(o0, __shfl_xor_sync(kFull, o0, 1));
+    o0 = max(o0, __shfl_xor_sync(kFull, o0, 2));
+    o1 = max(o1, __shfl_xor_sync(kFull, o1, 1));
+    o1 = max(o1, __shfl_xor_sync(kFull, o1, 2));
+    const double m0 = from_ord_hi(o0), m1 = from_ord_hi(o1);
     double l0 = 0.0, l1 = 0.0;
 #pragma unroll
     for (int j = 0; j < NBC; ++j) {
@@ -356,17 +380,18 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
         dmma884(s[j][0], s[j][1], q1v, kv.y);
       }
     }
-    double m = -INFINITY;
+    int om = INT_MIN;
 #pragma unroll
     for (int j = 0; j < NBC; ++j)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const bool valid = j < nkb && 8 * j + 2 * t + e < n;
         s[j][e] = valid ? s[j][e] : -INFINITY;
-        m = fmax(m, s[j][e]);
+        om = max(om, ord_hi(s[j][e]));
       }
-    m = fmax(m, __shfl_xor_sync(kFull, m, 1));
-    m = fmax(m, __shfl_xor_sync(kFull, m, 2));
+    om = max(om, __shfl_xor_sync(kFull, om, 1));
+    om = max(om, __shfl_xor_sync(kFull, om, 2));
+    const double m = from_ord_hi(om);
     double l = 0.0;
 #pragma unroll
     for (int j = 0; j < NBC; ++j) {

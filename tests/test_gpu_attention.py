@@ -260,3 +260,43 @@ def test_device_exp2_against_cuda():
     so = so.cpu().numpy()
     assert so[0] == 0.0 and np.isnan(so[1]) and so[2] == 0.0 and so[3] == 0.0
     assert so[4] == 1.0 and so[5] == 1.0
+
+
+def test_nan_feature_confined_to_its_centre():
+    """A NaN in one edge feature turns every output row of that centre to NaN
+    (all its keys, values and queries depend on it), as in the oracle, and no
+    other row: one layer and the six-layer stack."""
+    import oracle
+
+    m = U.mlg()
+    w = C.workload(2)
+    s = C.system(2, 0)
+    gpu, csr_t = U.gpu_build(s["coords"], s["box"], s["pbc"], w.rcut, w.r_on, w.nnei_max)
+    rp = gpu["row_ptr"]
+    e = gpu["n_edges"]
+    G = C.features(2, 0, e).astype(np.float64)
+    W = C.weights(2, 0)
+    G[int(rp[5]) + 3, 7] = np.nan
+    bad = np.zeros(e, dtype=bool)
+    bad[int(rp[5]):int(rp[6])] = True
+    out = U.gpu_attention(csr_t, w.n_atoms, w, G, W[0][0], W[0][1], W[0][2])
+    ref = oracle.attention(rp, gpu["sw"], G, W[0][0], W[0][1], W[0][2], w.heads)
+    assert np.isnan(ref[bad]).all() and np.isfinite(ref[~bad]).all()
+    assert np.isnan(out[bad]).all() and np.isfinite(out[~bad]).all()
+    ok, err = U.attn_tolerance_ok(w, out[~bad], ref[~bad])
+    assert ok, err
+    # the fused six-layer stack
+    g0 = torch.zeros((csr_t.capacity, w.channels), dtype=torch.float64, device="cuda")
+    g0[:e] = torch.as_tensor(G, device="cuda")
+    gout = torch.zeros_like(g0)
+    Wt = [torch.as_tensor(W[l][k], device="cuda") for l in range(w.n_layers) for k in range(3)]
+    ws = m.workspace(m.mlg_attention_stack_workspace_bytes(csr_t.capacity, w.channels,
+                                                           w.n_layers, m.MLG_F64))
+    m.mlg_attention_stack(csr_t, w.n_atoms, w.nnei_max, w.channels, w.heads, w.n_layers,
+                          m.MLG_F64, Wt, g0, gout, ws)
+    torch.cuda.synchronize()
+    outs = oracle.forward(rp, gpu["sw"], G, W, w.heads, "f64")
+    o6 = gout[:e].cpu().numpy()
+    assert np.isnan(o6[bad]).all() and np.isfinite(o6[~bad]).all()
+    ok, err = U.attn_tolerance_ok(w, o6[~bad], outs[-1][~bad])
+    assert ok, err

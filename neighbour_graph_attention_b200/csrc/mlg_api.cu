@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -138,11 +139,41 @@ void taylor_coeffs(double* c) {
   for (int k = 1; k < 12; ++k) c[k] = -c[k - 1] / (double)((2 * k) * (2 * k + 1));
 }
 
-// Ask for the largest shared-memory carveout, so that the occupancy the
-// shared memory allows is the occupancy the launch gets.
+// Host-side caches.  A kernel's attributes and occupancy, and a device's SM
+// count, do not change while the process runs, so the queries and attribute
+// settings behind a launch happen once per kernel and device rather than on
+// every call (they cost microseconds of host time each).
+struct KernelCacheEntry {
+  const void* fn;
+  int dev;
+  size_t smem_set;  // largest dynamic shared memory size set so far (0: none)
+  int nt;           // occupancy query: threads, shared memory, result
+  size_t smem_occ;
+  int blocks;
+};
+std::mutex g_kc_mu;
+constexpr int kKernelCacheMax = 512;
+KernelCacheEntry g_kc[kKernelCacheMax];
+int g_kc_n = 0;
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+
+// Entry for (fn, dev), created if absent (nullptr when the cache is full).
+KernelCacheEntry* kernel_cache(const void* fn, int dev) {
+  for (int i = 0; i < g_kc_n; ++i)
+    if (g_kc[i].fn == fn && g_kc[i].dev == dev) return &g_kc[i];
+  if (g_kc_n == kKernelCacheMax) return nullptr;
+  g_kc[g_kc_n] = KernelCacheEntry{fn, dev, 0, 0, 0, 0};
+  return &g_kc[g_kc_n++];
+}
+
 // Blocks of `kern` that fit on one SM by registers, shared memory, warps.
 template <typename K>
-int resident_blocks(K kern, int nt, size_t dyn_smem) {
+int resident_blocks_uncached(K kern, int nt, size_t dyn_smem) {
   cudaFuncAttributes fa;
   int dev = 0, regs_sm = 65536, smem_sm = 233472, reserved = 1024, thr_sm = 2048;
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return 1;
@@ -161,10 +192,41 @@ int resident_blocks(K kern, int nt, size_t dyn_smem) {
 }
 
 template <typename K>
+int resident_blocks(K kern, int nt, size_t dyn_smem) {
+  const void* fn = reinterpret_cast<const void*>(kern);
+  const int dev = current_device();
+  {
+    std::lock_guard<std::mutex> lk(g_kc_mu);
+    KernelCacheEntry* e = kernel_cache(fn, dev);
+    if (e != nullptr && e->blocks > 0 && e->nt == nt && e->smem_occ == dyn_smem) return e->blocks;
+  }
+  const int b = resident_blocks_uncached(kern, nt, dyn_smem);
+  std::lock_guard<std::mutex> lk(g_kc_mu);
+  if (KernelCacheEntry* e = kernel_cache(fn, dev)) {
+    e->nt = nt;
+    e->smem_occ = dyn_smem;
+    e->blocks = b;
+  }
+  return b;
+}
+
+// Allow `smem` bytes of dynamic shared memory and ask for the largest
+// carveout, so that the occupancy the shared memory allows is the occupancy
+// the launch gets.
+template <typename K>
 void prefer_shared(K kern, size_t smem) {
+  const void* fn = reinterpret_cast<const void*>(kern);
+  const int dev = current_device();
+  {
+    std::lock_guard<std::mutex> lk(g_kc_mu);
+    KernelCacheEntry* e = kernel_cache(fn, dev);
+    if (e != nullptr && e->smem_set >= smem && e->smem_set > 0) return;
+  }
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                        (int)cudaSharedmemCarveoutMaxShared);
+  std::lock_guard<std::mutex> lk(g_kc_mu);
+  if (KernelCacheEntry* e = kernel_cache(fn, dev)) e->smem_set = smem > e->smem_set ? smem : e->smem_set;
 }
 
 int launch_status() {
@@ -323,9 +385,12 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
 
 
 int sm_count() {
-  int sms = 148, dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static int cached[64] = {0};
+  const int dev = current_device();
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cached[dev] = sms;
   return sms;
 }
 
@@ -354,14 +419,12 @@ int launch_generic(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max, int3
   if (dtype == MLG_F64) {
     size_t smem = attn_generic_smem<double>(nnei_max, a.D);
     if (smem > 227 * 1024) return MLG_ERR_UNSUPPORTED;
-    cudaFuncSetAttribute(k_attn_generic<double>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
+    prefer_shared(k_attn_generic<double>, smem);
     k_attn_generic<double><<<grid, kAttnWarps * 32, smem, stream>>>(a);
   } else {
     size_t smem = attn_generic_smem<float>(nnei_max, a.D);
     if (smem > 227 * 1024) return MLG_ERR_UNSUPPORTED;
-    cudaFuncSetAttribute(k_attn_generic<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
+    prefer_shared(k_attn_generic<float>, smem);
     k_attn_generic<float><<<grid, kAttnWarps * 32, smem, stream>>>(a);
   }
   return launch_status();
@@ -372,12 +435,9 @@ template <typename T, int C, int D, int R, int NT, int TM, int TN, int XB>
 int launch_tile(TileArgs& ta, cudaStream_t stream) {
   using Cfg = TileCfg<T, C, D, R, NT, TM, TN, XB>;
   auto kern = k_attn_tile<T, C, D, R, NT, TM, TN, XB>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) !=
-      cudaSuccess)
-    return launch_status() == MLG_OK ? MLG_ERR_CUDA : MLG_ERR_CUDA;
-  int occ = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, Cfg::SMEM);
-  if (occ < 1) occ = 1;
+  prefer_shared(kern, Cfg::SMEM);
+  if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
+  const int occ = resident_blocks(kern, NT, Cfg::SMEM);
   int64_t want = (int64_t)sm_count() * occ;
   int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
   if (grid < 1) grid = 1;
@@ -480,9 +540,7 @@ int launch_hg(HgArgs& ha, cudaStream_t stream) {
   auto kern = k_attn_hg<T, C, D, HG, R, NT, TM, TN, KC>;
   prefer_shared(kern, Cfg::SMEM);
   if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
-  int occ = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, Cfg::SMEM);
-  if (occ < 1) occ = 1;
+  const int occ = resident_blocks(kern, NT, Cfg::SMEM);
   int64_t gx = ((int64_t)sm_count() * occ + Cfg::NG - 1) / Cfg::NG;
   if (gx > ha.n_centres) gx = ha.n_centres;
   if (gx < 1) gx = 1;

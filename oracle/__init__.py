@@ -75,6 +75,9 @@ def _load():
             lib.oracle_attention.argtypes = [i64, p, p, i32, i32, p, p, p, p, p, ctypes.c_int]
             lib.oracle_attention_map.restype = ctypes.c_int
             lib.oracle_attention_map.argtypes = [p, p, i32, i32, p, p, p, i64, i32, p]
+            lib.oracle_local_attention.restype = ctypes.c_int
+            lib.oracle_local_attention.argtypes = [i64, p, p, i32, i32, p, p, p, p, p, p,
+                                                   ctypes.c_int]
             _lib = lib
     return _lib
 
@@ -190,6 +193,31 @@ def attention(row_ptr, sw, G, Wq, Wk, Wv, heads: int, nthreads: int = 0) -> np.n
                                   int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_attention failed ({rc})")
+    return out
+
+
+def local_attention(row_ptr, sw, H, G, Wq, Wk, Wv, heads: int, nthreads: int = 0) -> np.ndarray:
+    """Local attention, one query per centre (NeighborGraph issue, "Graph-native
+    alternatives", item 2: LocalAtten with queries = centres, keys = edges).
+
+    q_i = H_i Wq from the centre's own feature row, K = G_i Wk and V = G_i Wv
+    from its edges; per head l_b = s_b (q_i . k_b) / sqrt(d), softmax over the
+    centre's edges, out_i = sum_b P_b V_b, heads concatenated; a centre
+    without edges gets a zero row.  Returns [n_centres][c], computed in fp64.
+    """
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int64)
+    sw, H, G = _as_f64(sw), _as_f64(H), _as_f64(G)
+    Wq, Wk, Wv = _as_f64(Wq), _as_f64(Wk), _as_f64(Wv)
+    c = H.shape[1]
+    n = row_ptr.size - 1
+    if H.shape[0] != n:
+        raise ValueError("H needs one row per centre")
+    out = np.zeros((n, c), dtype=np.float64)
+    rc = _load().oracle_local_attention(n, _ptr(row_ptr), _ptr(sw), c, int(heads), _ptr(H),
+                                        _ptr(G), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(out),
+                                        int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_local_attention failed ({rc})")
     return out
 
 

@@ -28,6 +28,11 @@
  *    ragged tails, scattered back to the edge axis): Q = G Wq, K = G Wk,
  *    V = G Wv; per head l_ab = s_a s_b (q_a . k_b) / sqrt(d); softmax over
  *    the centre's real edges b; O_a = sum_b P_ab V_b.
+ *  - Local attention, one query per centre (NeighborGraph issue, "Graph-native
+ *    alternatives", item 2: LocalAtten maps onto the per-centre CSR segment
+ *    with queries = centres and keys = edges): q_i = H_i Wq from the centre's
+ *    own feature row, K = G_i Wk, V = G_i Wv from its edges; per head
+ *    l_b = s_b (q_i . k_b) / sqrt(d); softmax over b; out_i = sum_b P_b V_b.
  *
  * Build: gcc -std=c11 -O2 -ffp-contract=off -fopenmp -shared -fPIC.
  * No -ffast-math, no contraction: every product and sum below is rounded
@@ -510,4 +515,74 @@ int oracle_attention_map(const int64_t* row_ptr, const double* sw, int32_t c, in
     head_map(n, c, d, h, sw + base, Q, K, P);
     free(Q); free(K);
     return ORC_OK;
+}
+
+/* Local attention over every centre: one query per centre from its own
+ * feature row H_i (q_i = H_i Wq), keys and values from its edges (K = G_i Wk,
+ * V = G_i Wv); per head h, l_b = s_b (q_i . k_b) / sqrt(d), P = softmax over
+ * the centre's edges b, out_i = sum_b P_b V_b, heads concatenated.  The
+ * centre has no distance of its own, so only the key's switch s_b weighs the
+ * logit.  A centre without edges gets a zero row.  H and out are
+ * [n_centres][c], G is [E][c] in CSR order. */
+int oracle_local_attention(int64_t n_centres, const int64_t* row_ptr, const double* sw,
+                           int32_t c, int32_t heads, const double* H, const double* G,
+                           const double* Wq, const double* Wk, const double* Wv, double* out,
+                           int nthreads) {
+    if (n_centres < 0 || c <= 0 || heads <= 0 || c % heads != 0) return ORC_ERR_ARG;
+    int d = c / heads;
+    double rsd = sqrt((double)d);
+    set_threads(nthreads);
+    int err = ORC_OK;
+#pragma omp parallel
+    {
+        double *q = (double*)malloc((size_t)c * sizeof(double));
+        double *K = NULL, *V = NULL, *P = NULL;
+        int64_t have = 0;
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t i = 0; i < n_centres; ++i) {
+            int64_t base = row_ptr[i];
+            int64_t n = row_ptr[i + 1] - base;
+            for (int m = 0; m < c; ++m) out[i * c + m] = 0.0;
+            if (n <= 0) continue;
+            if (n > have) {
+                free(K); free(V); free(P);
+                K = (double*)malloc((size_t)(n * c) * sizeof(double));
+                V = (double*)malloc((size_t)(n * c) * sizeof(double));
+                P = (double*)malloc((size_t)n * sizeof(double));
+                have = n;
+            }
+            if (!q || !K || !V || !P) {
+#pragma omp atomic write
+                err = ORC_ERR_MEM;
+                have = 0;
+                continue;
+            }
+            project(1, c, H + i * c, Wq, q);
+            project(n, c, G + base * c, Wk, K);
+            project(n, c, G + base * c, Wv, V);
+            for (int h = 0; h < heads; ++h) {
+                double m = -INFINITY;
+                for (int64_t b = 0; b < n; ++b) {
+                    double dot = 0.0;
+                    for (int t = 0; t < d; ++t) dot = dot + q[h * d + t] * K[b * c + h * d + t];
+                    double l = (sw[base + b] * dot) / rsd;
+                    P[b] = l;
+                    if (l > m) m = l;
+                }
+                double z = 0.0;
+                for (int64_t b = 0; b < n; ++b) {
+                    double e = exp(P[b] - m);
+                    P[b] = e;
+                    z = z + e;
+                }
+                for (int t = 0; t < d; ++t) {
+                    double acc = 0.0;
+                    for (int64_t b = 0; b < n; ++b) acc = acc + (P[b] / z) * V[b * c + h * d + t];
+                    out[i * c + h * d + t] = acc;
+                }
+            }
+        }
+        free(q); free(K); free(V); free(P);
+    }
+    return err;
 }

@@ -235,6 +235,32 @@ int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
                              const uint8_t pbc[3], int32_t nnei_max, int32_t channels,
                              int32_t heads, int32_t n_layers, mlg_dtype dtype);
 
+/* Local attention: one query per centre (NeighborGraph issue, "Graph-native
+ * alternatives", item 2: LocalAtten with queries = centres and keys = edges
+ * of the destination CSR).  For centre i with n = row_ptr[i+1] - row_ptr[i]
+ * edges: q = H_in[i] Wq, k_b = G_in[row_ptr[i] + b] Wk, v_b = ... Wv; per
+ * head h (d = channels / heads) l_b = sw_b (q^h . k_b^h) / sqrt(d), softmax
+ * over b < n, out[i]^h = sum_b P_b v_b^h; a centre without edges gets a
+ * zero row.  Only the key's switch weighs the logit (the centre has no
+ * distance of its own).
+ *   csr      CSR from mlg_build_csr (row_ptr, sw, capacity, status used);
+ *            rows must hold at most nnei_max edges (true for a CSR built
+ *            with the same nnei_max); longer rows give a zero row and set
+ *            MLG_STATUS_INTERNAL.
+ *   H_in     device [n_centres][channels] centre features, dtype.
+ *   G_in     device [E][channels] edge features in CSR order, dtype.
+ *   out      device [n_centres][channels], dtype; must not alias H_in or G_in.
+ *   Wq/Wk/Wv device [channels][channels] row-major (y = x W), dtype.
+ * channels <= 256, channels % heads == 0, 1 <= nnei_max <= 256.  The call
+ * is asynchronous on `stream`, allocates nothing and needs no workspace.
+ * Returns MLG_ERR_INVALID_ARG / MLG_ERR_UNSUPPORTED for bad arguments or
+ * shapes, MLG_ERR_CUDA if the launch fails; when E > capacity (status
+ * MLG_STATUS_CAPACITY) it writes nothing. */
+int mlg_local_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                        int32_t channels, int32_t heads, mlg_dtype dtype, const void* H_in,
+                        const void* G_in, void* out, const void* Wq, const void* Wk,
+                        const void* Wv, mlg_stream_t stream);
+
 /* Diagnostics: out[i] = 2^y[i] for i < n, by the device exponential that
  * the fp64 attention uses for its softmax weights (arguments y <= 0; -inf
  * gives 0, NaN gives NaN, y < -1000 gives 0).  y and out: device arrays of n

@@ -16,6 +16,7 @@
 #include "mlg_attn_hg.cuh"
 #include "mlg_attn_dmma.cuh"
 #include "mlg_attn_tc.cuh"
+#include "mlg_local.cuh"
 
 using namespace mlg;
 
@@ -696,6 +697,45 @@ int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
   if (!Wq || !Wk || !Wv) return MLG_ERR_INVALID_ARG;
   return attention_stack_impl(csr, n_centres, nnei_max, channels, heads, dtype, 1, W, G_in, G_out,
                               nullptr, (cudaStream_t)stream);
+}
+
+int mlg_local_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                        int32_t channels, int32_t heads, mlg_dtype dtype, const void* H_in,
+                        const void* G_in, void* out, const void* Wq, const void* Wk,
+                        const void* Wv, mlg_stream_t stream) {
+  int rc = check_attention_args(csr, n_centres, nnei_max, channels, heads, dtype, G_in, out);
+  if (rc != MLG_OK) return rc;
+  if (H_in == nullptr || H_in == out || !Wq || !Wk || !Wv) return MLG_ERR_INVALID_ARG;
+  if (n_centres == 0) return MLG_OK;
+  if (channels > kLocalMaxC) return MLG_ERR_UNSUPPORTED;
+  LocalArgs la;
+  la.row_ptr = csr->row_ptr;
+  la.sw = csr->sw;
+  la.n_centres = n_centres;
+  la.capacity = csr->capacity;
+  la.channels = channels;
+  la.heads = heads;
+  la.nnei_max = nnei_max;
+  la.H = H_in;
+  la.G = G_in;
+  la.out = out;
+  la.Wq = Wq;
+  la.Wk = Wk;
+  la.Wv = Wv;
+  la.status = csr->status;
+  cudaStream_t st = (cudaStream_t)stream;
+  auto go = [&](auto kern, size_t smem) {
+    if (smem > 227 * 1024) return (int)MLG_ERR_UNSUPPORTED;
+    prefer_shared(kern, smem);
+    if (cudaGetLastError() != cudaSuccess) return (int)MLG_ERR_CUDA;
+    const int64_t want = (int64_t)resident_blocks(kern, kLocalThreads, smem) * sm_count();
+    const int grid = (int)(n_centres < want ? n_centres : want);
+    kern<<<grid, kLocalThreads, smem, st>>>(la);
+    return launch_status();
+  };
+  if (dtype == MLG_F64)
+    return go(k_local_attn<double>, local_smem<double>(channels, heads, nnei_max));
+  return go(k_local_attn<float>, local_smem<float>(channels, heads, nnei_max));
 }
 
 size_t mlg_attention_stack_workspace_bytes(int64_t capacity, int32_t channels, int32_t n_layers,

@@ -89,6 +89,9 @@ _lib.mlg_attention_stack.restype = ctypes.c_int
 _lib.mlg_attention_stack.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32, _c_i32,
                                      _c_i32, ctypes.c_int, ctypes.POINTER(_p), _p, _p, _p, _c_sz,
                                      _p]
+_lib.mlg_local_attention.restype = ctypes.c_int
+_lib.mlg_local_attention.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32, _c_i32,
+                                     ctypes.c_int, _p, _p, _p, _p, _p, _p, _p]
 _lib.mlg_exp2_neg.restype = ctypes.c_int
 _lib.mlg_exp2_neg.argtypes = [_p, _p, _c_i64, _p]
 _lib.mlg_status_string.restype = ctypes.c_char_p
@@ -285,6 +288,19 @@ def mlg_block_attention(csr: Csr, n_centres: int, nnei_max: int, channels: int, 
                                     _ptr(G_out), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(ws),
                                     int(ws_bytes), _stream_handle(stream))
     return _check(code, "mlg_block_attention", check)
+
+
+def mlg_local_attention(csr: Csr, n_centres: int, nnei_max: int, channels: int, heads: int,
+                        dtype: int, H_in, G_in, out, Wq, Wk, Wv, stream=None,
+                        check: bool = True) -> int:
+    """Launch local attention (one query per centre from ``H_in``; keys and
+    values from the centre's edges in ``G_in``) on ``stream``."""
+    c = csr.struct()
+    code = _lib.mlg_local_attention(ctypes.byref(c), int(n_centres), int(nnei_max),
+                                    int(channels), int(heads), int(dtype), _ptr(H_in),
+                                    _ptr(G_in), _ptr(out), _ptr(Wq), _ptr(Wk), _ptr(Wv),
+                                    _stream_handle(stream))
+    return _check(code, "mlg_local_attention", check)
 
 
 def mlg_forward(system: mlg_system, rcut: float, r_on: float, nnei_max: int, channels: int,

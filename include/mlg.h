@@ -146,6 +146,26 @@ size_t mlg_build_csr_workspace_bytes(int64_t n_atoms, double rcut, const double 
 int mlg_build_csr(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
                   const mlg_csr* csr, void* ws, size_t ws_bytes, mlg_stream_t stream);
 
+/* Several independent systems in one CSR (batched inference of many
+ * structures, as the NValchemi batching on the source pages does; there is
+ * no neighbour cache, so a refill of the same size, a cell change or a new
+ * partition always gives the fresh graph).  Atom a of system k is centre and
+ * source number off_k + a, off_k = the atoms of systems 0..k-1; rows of
+ * system k are its mlg_build_csr rows with sources offset by off_k, in that
+ * order, so row_ptr has sum(N_k) + 1 entries.  Systems never pair with each
+ * other; each has its own box, pbc and types.  A system with 0 atoms adds no
+ * rows.  Same outputs, status bits and capacity behaviour as mlg_build_csr;
+ * arguments as there, plus:
+ *   systems    host array of n_systems descriptors (device coordinates)
+ *   ws         >= mlg_build_csr_batch_workspace_bytes(), 256-byte aligned
+ * The systems run one after another on `stream` (a launch chain per system,
+ * with one scan of all kept counts between the count and fill passes). */
+size_t mlg_build_csr_batch_workspace_bytes(const mlg_system* systems, int32_t n_systems,
+                                           double rcut);
+int mlg_build_csr_batch(const mlg_system* systems, int32_t n_systems, double rcut, double r_on,
+                        int32_t nnei_max, const mlg_csr* csr, void* ws, size_t ws_bytes,
+                        mlg_stream_t stream);
+
 /* Bytes of device workspace that mlg_block_attention needs (0 in this build). */
 size_t mlg_attention_workspace_bytes(int64_t n_centres, int32_t nnei_max, int32_t channels,
                                      int32_t heads, mlg_dtype dtype);

@@ -267,27 +267,13 @@ bool use_fused_build(const BuildPlan& plan, int64_t n) {
          fused_build_fits(n, plan.ncell_cap);
 }
 
-int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
-               const mlg_csr* csr, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  if (sys == nullptr || sys->coords == nullptr) return MLG_ERR_INVALID_ARG;
-  if (!(r_on >= 0.0) || !(r_on < rcut) || !std::isfinite(r_on)) return MLG_ERR_INVALID_ARG;
-  if (nnei_max < 1) return MLG_ERR_INVALID_ARG;
-  if (nnei_max > kMaxNnei) return MLG_ERR_UNSUPPORTED;
-  if (sys->types != nullptr && sys->n_types < 1) return MLG_ERR_INVALID_ARG;
-  int rc = check_csr(csr);
-  if (rc != MLG_OK) return rc;
-  BuildPlan plan;
-  rc = make_plan(sys->n_atoms, rcut, sys->box, sys->pbc, &plan);
-  if (rc != MLG_OK) return rc;
-  const int64_t n = sys->n_atoms;
-  BuildLayout L = build_layout(n, plan.ncell_cap);
-  if (ws == nullptr || ws_bytes < L.total || ((uintptr_t)ws % kAlign) != 0)
-    return MLG_ERR_WORKSPACE;
-
-  char* w = static_cast<char*>(ws);
+// Arguments of the build kernels for one system whose workspace starts at w
+// (layout L).  The caller adjusts the pointers and offsets of a batch.
+BuildArgs make_build_args(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+                          const mlg_csr* csr, char* w, const BuildLayout& L) {
   BuildArgs a;
   std::memset(&a, 0, sizeof(a));
-  a.n = n;
+  a.n = sys->n_atoms;
   a.coords = sys->coords;
   a.types = sys->types;
   a.n_types = sys->n_types;
@@ -307,6 +293,8 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   a.n_edges = csr->n_edges;
   a.n_truncated = csr->n_truncated;
   a.status = csr->status;
+  a.src_offset = 0;
+  a.zero_globals = 1;
   a.grid = reinterpret_cast<CellGrid*>(w + L.grid);
   a.bbox = reinterpret_cast<unsigned long long*>(w + L.bbox);
   a.cell_count = reinterpret_cast<int*>(w + L.cell_count);
@@ -319,13 +307,83 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   a.kept = reinterpret_cast<int*>(w + L.kept);
   a.raw = reinterpret_cast<int*>(w + L.raw);
   a.partial = reinterpret_cast<long long*>(w + L.partial);
+  return a;
+}
 
-  // per-cell scans when every stencil reach is 1 (at most 27 stencil cells);
-  // otherwise (boxes narrower than the cutoff) the per-centre scans.  A grid
-  // of few cells splits each cell's centres over several CTAs.
-  const bool per_cell = plan.max_reach <= 1;
+// A grid of few cells splits each cell's centres over several CTAs.
+int build_nsplit(const BuildPlan& plan) {
   int nsplit = (4 * sm_count() + plan.ncell_cap - 1) / plan.ncell_cap;
-  nsplit = nsplit < 1 ? 1 : (nsplit > 8 ? 8 : nsplit);
+  return nsplit < 1 ? 1 : (nsplit > 8 ? 8 : nsplit);
+}
+
+// Host checks shared by the single and the batched build.
+int check_build_args(double rcut, double r_on, int32_t nnei_max, const mlg_csr* csr) {
+  if (!(r_on >= 0.0) || !(r_on < rcut) || !std::isfinite(r_on)) return MLG_ERR_INVALID_ARG;
+  if (nnei_max < 1) return MLG_ERR_INVALID_ARG;
+  if (nnei_max > kMaxNnei) return MLG_ERR_UNSUPPORTED;
+  return check_csr(csr);
+}
+
+// The launch chain up to the kept counts: init, [bbox], bin, cell scan,
+// scatter, count.  Per-cell scans when every stencil reach is 1 (at most 27
+// stencil cells); otherwise (boxes narrower than the cutoff) the per-centre
+// scans.
+void launch_count_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
+                        cudaStream_t stream) {
+  const int tb = 256;
+  const int atom_blocks = (int)((a.n + tb - 1) / tb);
+  int init_blocks = (plan.ncell_cap + 1 + tb - 1) / tb;
+  if (init_blocks > 1024) init_blocks = 1024;
+  k_init<<<init_blocks, tb, 0, stream>>>(a, plan.ncell_cap);
+  if (plan.any_open) {
+    int bb = atom_blocks < 592 ? atom_blocks : 592;
+    k_bbox<<<bb, tb, 0, stream>>>(a, plan);
+  }
+  k_bin<<<atom_blocks, tb, 0, stream>>>(a, plan);
+  launch_scan<int>(a.cell_count, plan.ncell_cap, a.cell_start, a.partial,
+                   ScanTail{nullptr, nullptr, 0}, stream);
+  k_scatter<<<atom_blocks, tb, 0, stream>>>(a);
+  if (plan.max_reach <= 1) {
+    const size_t sm_count_ = cellscan_smem(false);
+    prefer_shared(k_cellscan<false>, sm_count_);
+    k_cellscan<false><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kCellWarps * 32,
+                        sm_count_, stream>>>(a);
+  } else {
+    k_count<<<(int)((a.n + kCountWarps - 1) / kCountWarps), kCountWarps * 32, 0, stream>>>(a);
+  }
+}
+
+// The fill, once row_ptr holds the row starts.
+void launch_fill_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
+                       cudaStream_t stream) {
+  if (plan.max_reach <= 1) {
+    const size_t sm_fill = cellscan_smem(true);
+    prefer_shared(k_cellscan<true>, sm_fill);
+    k_cellscan<true><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kCellWarps * 32,
+                       sm_fill, stream>>>(a);
+  } else {
+    const size_t fill_smem = (size_t)kFillWarps * 2 * kFillMaxCand * sizeof(unsigned long long);
+    k_fill<<<(int)((a.n + kFillWarps - 1) / kFillWarps), kFillWarps * 32, fill_smem, stream>>>(
+        a);
+  }
+}
+
+int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+               const mlg_csr* csr, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (sys == nullptr || sys->coords == nullptr) return MLG_ERR_INVALID_ARG;
+  if (sys->types != nullptr && sys->n_types < 1) return MLG_ERR_INVALID_ARG;
+  int rc = check_build_args(rcut, r_on, nnei_max, csr);
+  if (rc != MLG_OK) return rc;
+  BuildPlan plan;
+  rc = make_plan(sys->n_atoms, rcut, sys->box, sys->pbc, &plan);
+  if (rc != MLG_OK) return rc;
+  const int64_t n = sys->n_atoms;
+  BuildLayout L = build_layout(n, plan.ncell_cap);
+  if (ws == nullptr || ws_bytes < L.total || ((uintptr_t)ws % kAlign) != 0)
+    return MLG_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  const BuildArgs a = make_build_args(sys, rcut, r_on, nnei_max, csr, w, L);
+  const int nsplit = build_nsplit(plan);
   if (use_fused_build(plan, n)) {
     // the whole build in one cooperative launch (small systems)
     const size_t smem = fused_build_smem(n);
@@ -350,40 +408,101 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
       return launch_status();
     (void)cudaGetLastError();  // refused (not co-resident): the launch chain below
   }
-
-  const int tb = 256;
-  const int atom_blocks = (int)((n + tb - 1) / tb);
-  int init_blocks = (plan.ncell_cap + 1 + tb - 1) / tb;
-  if (init_blocks > 1024) init_blocks = 1024;
-  k_init<<<init_blocks, tb, 0, stream>>>(a, plan.ncell_cap);
-  if (plan.any_open) {
-    int bb = atom_blocks < 592 ? atom_blocks : 592;
-    k_bbox<<<bb, tb, 0, stream>>>(a, plan);
-  }
-  k_bin<<<atom_blocks, tb, 0, stream>>>(a, plan);
-  launch_scan<int>(a.cell_count, plan.ncell_cap, a.cell_start, a.partial,
-                   ScanTail{nullptr, nullptr, 0}, stream);
-  k_scatter<<<atom_blocks, tb, 0, stream>>>(a);
-  const dim3 cell_grid((unsigned)plan.ncell_cap, (unsigned)nsplit);
-  if (per_cell) {
-    const size_t sm_count_ = cellscan_smem(false), sm_fill = cellscan_smem(true);
-    prefer_shared(k_cellscan<false>, sm_count_);
-    prefer_shared(k_cellscan<true>, sm_fill);
-    k_cellscan<false><<<cell_grid, kCellWarps * 32, sm_count_, stream>>>(a);
-  } else {
-    k_count<<<(int)((n + kCountWarps - 1) / kCountWarps), kCountWarps * 32, 0, stream>>>(a);
-  }
+  launch_count_phase(a, plan, nsplit, stream);
   launch_scan<long long>(a.kept, n, reinterpret_cast<long long*>(a.row_ptr), a.partial,
                          ScanTail{a.n_edges, a.status, a.capacity}, stream);
-  if (per_cell) {
-    k_cellscan<true><<<cell_grid, kCellWarps * 32, cellscan_smem(true), stream>>>(a);
-  } else {
-    const size_t fill_smem = (size_t)kFillWarps * 2 * kFillMaxCand * sizeof(unsigned long long);
-    k_fill<<<(int)((n + kFillWarps - 1) / kFillWarps), kFillWarps * 32, fill_smem, stream>>>(a);
-  }
+  launch_fill_phase(a, plan, nsplit, stream);
   return launch_status();
 }
 
+// ---------------------------------------------------------------- batches
+//
+// Workspace of a batch: the kept and raw counts of all atoms (one array, so
+// that one scan gives the global row starts) and its scan partials, then the
+// build workspace of each system with atoms.
+struct BatchTotals {
+  int64_t n_total;
+  size_t global_bytes;
+  size_t total;
+  size_t kept, raw, partial;
+};
+
+int batch_totals(const mlg_system* systems, int32_t n_systems, double rcut, BatchTotals* t) {
+  if (n_systems < 0 || (n_systems > 0 && systems == nullptr)) return MLG_ERR_INVALID_ARG;
+  int64_t n_total = 0;
+  size_t per_sys = 0;
+  for (int32_t k = 0; k < n_systems; ++k) {
+    const mlg_system& s = systems[k];
+    if (s.n_atoms < 0) return MLG_ERR_INVALID_ARG;
+    if (s.n_atoms == 0) continue;
+    if (s.coords == nullptr || (s.types != nullptr && s.n_types < 1)) return MLG_ERR_INVALID_ARG;
+    BuildPlan plan;
+    int rc = make_plan(s.n_atoms, rcut, s.box, s.pbc, &plan);
+    if (rc != MLG_OK) return rc;
+    per_sys += align_up(build_layout(s.n_atoms, plan.ncell_cap).total);
+    n_total += s.n_atoms;
+  }
+  if (n_total > (int64_t)INT32_MAX / 2) return MLG_ERR_UNSUPPORTED;
+  t->n_total = n_total;
+  size_t off = 0;
+  t->kept = off;
+  off = align_up(off + (size_t)n_total * sizeof(int));
+  t->raw = off;
+  off = align_up(off + (size_t)n_total * sizeof(int));
+  t->partial = off;
+  off = align_up(off + (size_t)(scan_tiles(n_total > 0 ? n_total : 1) + 2) * sizeof(long long));
+  t->global_bytes = off;
+  t->total = off + per_sys;
+  return MLG_OK;
+}
+
+int build_batch_impl(const mlg_system* systems, int32_t n_systems, double rcut, double r_on,
+                     int32_t nnei_max, const mlg_csr* csr, void* ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+  int rc = check_build_args(rcut, r_on, nnei_max, csr);
+  if (rc != MLG_OK) return rc;
+  BatchTotals T;
+  rc = batch_totals(systems, n_systems, rcut, &T);
+  if (rc != MLG_OK) return rc;
+  if (ws == nullptr || ws_bytes < T.total || ((uintptr_t)ws % kAlign) != 0)
+    return MLG_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  int* kept = reinterpret_cast<int*>(w + T.kept);
+  int* raw = reinterpret_cast<int*>(w + T.raw);
+  long long* partial = reinterpret_cast<long long*>(w + T.partial);
+  if (cudaMemsetAsync(csr->status, 0, sizeof(uint32_t), stream) != cudaSuccess ||
+      cudaMemsetAsync(csr->n_truncated, 0, sizeof(int64_t), stream) != cudaSuccess)
+    return MLG_ERR_CUDA;
+  // count every system into its slice of the kept counts
+  for (int pass = 0; pass < 2; ++pass) {
+    if (pass == 1)
+      launch_scan<long long>(kept, T.n_total, reinterpret_cast<long long*>(csr->row_ptr),
+                             partial, ScanTail{csr->n_edges, csr->status, csr->capacity},
+                             stream);
+    size_t sys_off = T.global_bytes;
+    int64_t atom_off = 0;
+    for (int32_t k = 0; k < n_systems; ++k) {
+      const mlg_system& s = systems[k];
+      if (s.n_atoms == 0) continue;
+      BuildPlan plan;
+      make_plan(s.n_atoms, rcut, s.box, s.pbc, &plan);
+      const BuildLayout L = build_layout(s.n_atoms, plan.ncell_cap);
+      BuildArgs a = make_build_args(&s, rcut, r_on, nnei_max, csr, w + sys_off, L);
+      a.kept = kept + atom_off;
+      a.raw = raw + atom_off;
+      a.row_ptr = csr->row_ptr + atom_off;
+      a.src_offset = (int32_t)atom_off;
+      a.zero_globals = 0;
+      if (pass == 0)
+        launch_count_phase(a, plan, build_nsplit(plan), stream);
+      else
+        launch_fill_phase(a, plan, build_nsplit(plan), stream);
+      sys_off += align_up(L.total);
+      atom_off += s.n_atoms;
+    }
+  }
+  return launch_status();
+}
 
 int sm_count() {
   static int cached[64] = {0};
@@ -675,6 +794,21 @@ size_t mlg_build_csr_workspace_bytes(int64_t n_atoms, double rcut, const double 
 int mlg_build_csr(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
                   const mlg_csr* csr, void* ws, size_t ws_bytes, mlg_stream_t stream) {
   return build_impl(sys, rcut, r_on, nnei_max, csr, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+size_t mlg_build_csr_batch_workspace_bytes(const mlg_system* systems, int32_t n_systems,
+                                           double rcut) {
+  if (!(rcut > 0.0) || !std::isfinite(rcut)) return 0;
+  BatchTotals T;
+  if (batch_totals(systems, n_systems, rcut, &T) != MLG_OK) return 0;
+  return T.total;
+}
+
+int mlg_build_csr_batch(const mlg_system* systems, int32_t n_systems, double rcut, double r_on,
+                        int32_t nnei_max, const mlg_csr* csr, void* ws, size_t ws_bytes,
+                        mlg_stream_t stream) {
+  return build_batch_impl(systems, n_systems, rcut, r_on, nnei_max, csr, ws, ws_bytes,
+                          (cudaStream_t)stream);
 }
 
 size_t mlg_attention_workspace_bytes(int64_t n_centres, int32_t nnei_max, int32_t channels,

@@ -95,6 +95,8 @@ struct BuildArgs {
   int64_t* n_edges;
   int64_t* n_truncated;
   uint32_t* status;
+  int32_t src_offset;        // added to written source indices (systems of a batch)
+  int zero_globals;          // k_init clears n_truncated and status (not in a batch)
   // workspace
   CellGrid* grid;
   unsigned long long* bbox;  // [6] ordered bits: min x, y, z, max x, y, z
@@ -233,7 +235,7 @@ __global__ void k_init(BuildArgs a, int ncell_cap) {
     a.bbox[t] = ~0ull;
     a.bbox[3 + t] = 0ull;
   }
-  if (t == 0) {
+  if (t == 0 && a.zero_globals) {
     *a.n_truncated = 0;
     *a.status = 0u;
   }
@@ -759,7 +761,7 @@ __device__ __forceinline__ void write_edge(const BuildArgs& a, const Centre& cc,
   double r2 = edge_vec(a.box, cc.x, xj, S, v);
   double r = __dsqrt_rn(r2);
   if (p < a.capacity) {
-    a.src[p] = j;
+    a.src[p] = j + a.src_offset;
     a.shift[3 * p] = S[0];
     a.shift[3 * p + 1] = S[1];
     a.shift[3 * p + 2] = S[2];

@@ -89,6 +89,11 @@ _lib.mlg_attention_stack.restype = ctypes.c_int
 _lib.mlg_attention_stack.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32, _c_i32,
                                      _c_i32, ctypes.c_int, ctypes.POINTER(_p), _p, _p, _p, _c_sz,
                                      _p]
+_lib.mlg_build_csr_batch_workspace_bytes.restype = _c_sz
+_lib.mlg_build_csr_batch_workspace_bytes.argtypes = [ctypes.POINTER(mlg_system), _c_i32, _c_dbl]
+_lib.mlg_build_csr_batch.restype = ctypes.c_int
+_lib.mlg_build_csr_batch.argtypes = [ctypes.POINTER(mlg_system), _c_i32, _c_dbl, _c_dbl, _c_i32,
+                                     ctypes.POINTER(mlg_csr), _p, _c_sz, _p]
 _lib.mlg_local_attention.restype = ctypes.c_int
 _lib.mlg_local_attention.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32, _c_i32,
                                      ctypes.c_int, _p, _p, _p, _p, _p, _p, _p]
@@ -288,6 +293,31 @@ def mlg_block_attention(csr: Csr, n_centres: int, nnei_max: int, channels: int, 
                                     _ptr(G_out), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(ws),
                                     int(ws_bytes), _stream_handle(stream))
     return _check(code, "mlg_block_attention", check)
+
+
+def _system_array(systems):
+    arr = (mlg_system * max(len(systems), 1))()
+    for k, s in enumerate(systems):
+        arr[k] = s
+    return arr
+
+
+def mlg_build_csr_batch_workspace_bytes(systems, rcut: float) -> int:
+    """Workspace bytes of mlg_build_csr_batch for these mlg_system descriptors."""
+    return _lib.mlg_build_csr_batch_workspace_bytes(_system_array(systems), len(systems),
+                                                    float(rcut))
+
+
+def mlg_build_csr_batch(systems, rcut: float, r_on: float, nnei_max: int, csr: Csr, ws,
+                        ws_bytes: int | None = None, stream=None, check: bool = True) -> int:
+    """Launch the build of one CSR over several systems (``systems``: a list of
+    mlg_system descriptors, e.g. from make_system)."""
+    c = csr.struct()
+    nb = ws.numel() * ws.element_size() if ws_bytes is None else int(ws_bytes)
+    code = _lib.mlg_build_csr_batch(_system_array(systems), len(systems), float(rcut),
+                                    float(r_on), int(nnei_max), ctypes.byref(c), _ptr(ws), nb,
+                                    _stream_handle(stream))
+    return _check(code, "mlg_build_csr_batch", check)
 
 
 def mlg_local_attention(csr: Csr, n_centres: int, nnei_max: int, channels: int, heads: int,

@@ -171,3 +171,27 @@ def test_product_path_fails_loudly_without_library(tmp_path):
         "    print('IMPORT_ERROR', 'no CPU fallback' in str(e))\n")
     out = subprocess.run(["python", "-c", code], capture_output=True, text=True)
     assert "IMPORT_ERROR True" in out.stdout, out.stdout + out.stderr
+
+
+def test_batch_workspace_and_checks(mlg):
+    """Host side of the batched build: workspace sizes and argument checks
+    (no kernel runs: every call below fails a host check)."""
+    lib = mlg.lib()
+    a, b = _sys(mlg, 64), _sys(mlg, 200, box=np.zeros((3, 3)), pbc=(0, 0, 0))
+    empty = _sys(mlg, 0)
+    one_a = mlg.mlg_build_csr_workspace_bytes(64, 4.0, np.diag([10.0] * 3), [1, 1, 1])
+    one_b = mlg.mlg_build_csr_workspace_bytes(200, 4.0, np.zeros((3, 3)), [0, 0, 0])
+    both = mlg.mlg_build_csr_batch_workspace_bytes([a, empty, b], 4.0)
+    assert both >= one_a + one_b                       # each system's own workspace, plus counts
+    assert mlg.mlg_build_csr_batch_workspace_bytes([], 4.0) > 0
+    assert mlg.mlg_build_csr_batch_workspace_bytes([a], -1.0) == 0
+    assert mlg.mlg_build_csr_batch_workspace_bytes([_sys(mlg, -3)], 4.0) == 0
+    arr = mlg._system_array([a, b])
+    csr = _fake_csr(mlg)
+    call = lambda n=2, rcut=4.0, r_on=3.5, nnei=40, ws=None, nb=0: lib.mlg_build_csr_batch(
+        arr, n, rcut, r_on, nnei, ctypes.byref(csr), ws, nb, None)
+    assert call(ws=None, nb=both) == mlg.MLG_ERR_WORKSPACE
+    assert call(ws=FAKE * 16, nb=both - 1) == mlg.MLG_ERR_WORKSPACE
+    assert call(n=-1, ws=FAKE * 16, nb=both) == mlg.MLG_ERR_INVALID_ARG
+    assert call(r_on=5.0, ws=FAKE * 16, nb=both) == mlg.MLG_ERR_INVALID_ARG
+    assert call(nnei=999, ws=FAKE * 16, nb=both) == mlg.MLG_ERR_UNSUPPORTED

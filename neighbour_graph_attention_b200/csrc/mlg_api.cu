@@ -550,21 +550,6 @@ int launch_generic(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max, int3
   return launch_status();
 }
 
-// Tile kernel instantiations: (dtype, channels, head size) -> tile rows R.
-template <typename T, int C, int D, int R, int NT, int TM, int TN, int XB>
-int launch_tile(TileArgs& ta, cudaStream_t stream) {
-  using Cfg = TileCfg<T, C, D, R, NT, TM, TN, XB>;
-  auto kern = k_attn_tile<T, C, D, R, NT, TM, TN, XB>;
-  prefer_shared(kern, Cfg::SMEM);
-  if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
-  const int occ = resident_blocks(kern, NT, Cfg::SMEM);
-  int64_t want = (int64_t)sm_count() * occ;
-  int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
-  if (grid < 1) grid = 1;
-  kern<<<grid, NT, Cfg::SMEM, stream>>>(ta);
-  return launch_status();
-}
-
 // FP64 tensor-core kernel: one CTA of NT threads per SM (shared memory), tiles
 // of R rows, centres of at most 8 NBC edges.
 template <int R, int NBC, int NT>

@@ -1,29 +1,21 @@
-// mlg_attn_tile.cuh -- fused multi-layer block-dense attention for channel
-// counts whose three projection matrices fit in shared memory (sm_100a).
+// mlg_attn_tile.cuh -- pieces shared by the fused block-dense attention
+// kernels (sm_100a): the tile arguments and plan, PTX helpers for mbarriers
+// and TMA bulk copies, and the per-centre attention loop over a resident tile.
 //
 // NeighborGraph issue ("NeighborGraph attention is 4-9x slower than dense and
 // OOM-prone"), Proposed fix: per centre, gather the compact block of its edge
 // features through destination_row_ptr, run dense attention with per-row
 // masks, write back to the edge axis.  Because the edges of a centre are one
 // contiguous CSR slab, a tile of consecutive centres is one contiguous
-// [rows][C] slab of G: it is moved global->shared and shared->global by TMA
-// bulk copies (cp.async.bulk, no multicast).  A centre's output rows depend
-// only on its own input rows, so every layer of the stack runs on the
-// resident tile before it is written back (G^{l+1} = O^l never leaves the SM).
+// [rows][C] slab of G; a centre's output rows depend only on its own input
+// rows, so every layer of a stack can run on the resident tile before it is
+// written back (G^{l+1} = O^l never leaves the SM).
 //
-// Per tile and layer:
-//   1. QKV = X [rows][C] . [Wq | Wk | Wv] [C][3C]: register-tiled FMA GEMM
-//      from shared memory; the epilogue folds s_a / sqrt(d) into q (times
-//      log2 e for fp32, whose softmax uses exp2) and s_b into k.
-//   2. attention: one lane per (query row a, head h) of a centre, lanes of a
-//      warp in lock-step over key rows b, so k_b and v_b are broadcast
-//      shared-memory reads; softmax with a running max in blocks of 8 keys.
-//   3. O overwrites X in shared memory; the next layer's weights stream in
-//      (TMA) while the attention runs.
-// Persistent CTAs: CTA b owns the centres whose first edge row lies in the
-// b-th equal share of the E rows; it packs consecutive centres into tiles of
-// at most R rows and prefetches the next tile's slab.  Centres with more than
-// R edges are left to the generic kernel (mlg_attn.cuh).
+// tile_attention(): one lane per (query row a, head h) of a centre, the lanes
+// of a warp in lock-step over key rows b, so k_b and v_b are broadcast
+// shared-memory reads; softmax with a running max in blocks of 8 keys.  Used
+// by the tcgen05 kernel (mlg_attn_tc.cuh) and the head-group kernel
+// (mlg_attn_hg.cuh).
 #pragma once
 
 #include "mlg_common.cuh"
@@ -121,7 +113,7 @@ __device__ __forceinline__ float softmax_exp<float>(float x) { return exp2f(x); 
 template <>
 __device__ __forceinline__ double softmax_exp<double>(double x) { return exp(x); }
 
-// ---------------------------------------------------------------- the kernel
+// ---------------------------------------------------------------- tiles
 
 struct TileMeta {
   uint64_t bar_x[2];
@@ -137,38 +129,6 @@ struct TileMeta {
   int fail;
 };
 
-template <typename T, int C, int D, int R, int NT, int TM, int TN, int XB>
-struct TileCfg {
-  static constexpr int H = C / D;
-  static constexpr int N3 = 3 * C;              // GEMM output columns
-  static constexpr int NCG = N3 / TN;           // column groups
-  static constexpr int NRG = R / TM;            // row groups
-  static constexpr int QS = N3 + (sizeof(T) == 8 ? 1 : 4);  // QKV row stride (elements)
-  static constexpr int MAXC = 64;               // centres per tile (bookkeeping arrays)
-  static_assert(NCG * NRG == NT, "thread grid must cover the tile");
-  static_assert(C % D == 0 && D % 4 == 0, "head size");
-  static_assert(C % NCG == 0, "column groups must not straddle q/k/v");
-  // shared memory layout (bytes)
-  static constexpr size_t X_BYTES = (size_t)R * C * sizeof(T);
-  static constexpr size_t W_BYTES = (size_t)3 * C * C * sizeof(T);
-  static constexpr size_t Q_BYTES = (size_t)R * QS * sizeof(T);
-  static_assert(XB == 1 || XB == 2, "one or two tile buffers");
-  static constexpr size_t OFF_X0 = 0;
-  static constexpr size_t OFF_X1 = OFF_X0 + X_BYTES;
-  static constexpr size_t OFF_W = OFF_X0 + XB * X_BYTES;
-  static constexpr size_t OFF_Q = OFF_W + W_BYTES;
-  static constexpr size_t OFF_S = OFF_Q + Q_BYTES;
-  static constexpr size_t OFF_META = (OFF_S + (size_t)R * sizeof(T) + 15) / 16 * 16;
-  static constexpr size_t SMEM = OFF_META + sizeof(TileMeta);
-};
-
-
-
-// One key block of the running-max softmax for one lane (query row, head):
-// logits of keys [b0, b0 + 8) (masked to -inf at and beyond n when TAIL),
-// rescale of the running sum and output when the block raises the maximum,
-// then accumulation of exp(l - max) v.  fp32 logits are in log2 units (q
-// carries log2 e), fp64 ones in natural units.
 template <typename T, int D, bool TAIL>
 __device__ __forceinline__ void softmax_block(const T* q, T* o, T& mx, T& l, const T* kb,
                                               const T* vb, int b0, int n, int QS) {
@@ -275,222 +235,6 @@ __device__ __forceinline__ void tile_attention(T* sQ, const TileMeta& meta, int 
       T* qo = sQ + (base + row) * QS + h * D;
 #pragma unroll
       for (int t = 0; t < D; ++t) qo[t] = o[t] * rl;
-    }
-  }
-}
-
-template <typename T, int C, int D, int R, int NT, int TM, int TN, int XB>
-__global__ void __launch_bounds__(NT) k_attn_tile(TileArgs a) {
-  using Cfg = TileCfg<T, C, D, R, NT, TM, TN, XB>;
-  constexpr int H = Cfg::H, NCG = Cfg::NCG, QS = Cfg::QS;
-  extern __shared__ __align__(128) unsigned char smem[];
-  T* sX[2] = {reinterpret_cast<T*>(smem + Cfg::OFF_X0),
-              reinterpret_cast<T*>(smem + (XB == 2 ? Cfg::OFF_X1 : Cfg::OFF_X0))};
-  T* sW = reinterpret_cast<T*>(smem + Cfg::OFF_W);
-  T* sQ = reinterpret_cast<T*>(smem + Cfg::OFF_Q);
-  T* sS = reinterpret_cast<T*>(smem + Cfg::OFF_S);
-  TileMeta& meta = *reinterpret_cast<TileMeta*>(smem + Cfg::OFF_META);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const T* G = static_cast<const T*>(a.G);
-  T* out = static_cast<T*>(a.out);
-  const int64_t E = a.row_ptr[a.n_centres];
-  if (E > a.capacity || (*a.status & MLG_STATUS_CAPACITY)) return;
-
-  // ---- set-up: my centre range, barriers, first weights, first tile
-  if (tid == 0) {
-    const int64_t r0 = E * blockIdx.x / gridDim.x, r1 = E * (blockIdx.x + 1) / gridDim.x;
-    // first centre whose first row is >= r (lower bound over row_ptr[0..n_centres))
-    auto lb = [&](int64_t r) {
-      int64_t lo = 0, hi = a.n_centres;
-      while (lo < hi) {
-        int64_t mid = (lo + hi) >> 1;
-        if (a.row_ptr[mid] < r) lo = mid + 1; else hi = mid;
-      }
-      return (int)lo;
-    };
-    meta.next_c = lb(r0);
-    meta.c_end = blockIdx.x + 1 == gridDim.x ? (int)a.n_centres : lb(r1);
-    meta.fail = 0;
-    mbar_init(&meta.bar_x[0], 1);
-    mbar_init(&meta.bar_x[1], 1);
-    mbar_init(&meta.bar_w, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  // thread 0: pack the next tile (consecutive centres, <= R rows, skipping
-  // centres with more than R edges) into buffer b and start its slab copy
-  auto plan_and_load = [&](int b) {
-    int c = meta.next_c, k = 0, rows = 0;
-    const int c_end = meta.c_end;
-    // skip leading empty or oversized centres
-    while (c < c_end) {
-      int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
-      if (n > 0 && n <= R) break;
-      ++c;
-    }
-    meta.c0[b] = c;
-    meta.row0[b] = c < c_end ? a.row_ptr[c] : 0;
-    int tasks = 0;
-    while (c < c_end && k < Cfg::MAXC) {
-      int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
-      if (n > R) break;                 // oversized: ends the tile (handled elsewhere)
-      if (rows + n > R) break;
-      meta.off[b][k] = rows;
-      meta.task0[b][k] = tasks;
-      tasks += (n * H + 31) / 32;
-      rows += n;
-      ++k;
-      ++c;
-    }
-    meta.off[b][k] = rows;
-    meta.task0[b][k] = tasks;
-    meta.ncent[b] = k;
-    meta.nrows[b] = rows;
-    meta.next_c = c;
-    if (rows > 0) {
-      fence_proxy_async();
-      uint32_t bytes = (uint32_t)(rows * C * sizeof(T));
-      mbar_expect_tx(&meta.bar_x[b], bytes);
-      bulk_g2s(sX[b], G + meta.row0[b] * C, bytes, &meta.bar_x[b]);
-    }
-  };
-
-  auto load_weights = [&](int layer) {
-    fence_proxy_async();
-    const uint32_t bytes = (uint32_t)(C * C * sizeof(T));
-    mbar_expect_tx(&meta.bar_w, 3 * bytes);
-#pragma unroll
-    for (int m = 0; m < 3; ++m) bulk_g2s(sW + m * C * C, a.W[3 * layer + m], bytes, &meta.bar_w);
-  };
-
-  if (tid == 0) {
-    plan_and_load(0);
-    if (meta.nrows[0] > 0) load_weights(0);  // a CTA without tiles starts no copy
-  }
-  __syncthreads();
-
-  uint32_t ph_x[2] = {0u, 0u}, ph_w = 0u;
-  const T qscale = sizeof(T) == 4 ? T(1.4426950408889634 / sqrt((double)D))
-                                  : T(1.0 / sqrt((double)D));
-  int buf = 0;
-  bool weights_pending = meta.nrows[0] > 0;
-
-  while (true) {
-    if (meta.nrows[buf] == 0) break;  // uniform: written by thread 0 before a barrier
-    if (tid == 0) {
-      if (XB == 2) {
-        // prefetch the next tile into the other buffer (its last store must be read out)
-        bulk_wait_read_all();
-        plan_and_load(buf ^ 1);
-      }
-      bool okx = mbar_wait(&meta.bar_x[buf], ph_x[buf]);
-      if (!okx) meta.fail = 1;
-    }
-    __syncthreads();
-    if (meta.fail) break;
-    ph_x[buf] ^= 1u;
-    const int rows = meta.nrows[buf], ncent = meta.ncent[buf];
-    const int64_t row0 = meta.row0[buf];
-    for (int t = tid; t < rows; t += NT) sS[t] = (T)a.sw[row0 + t];
-    T* X = sX[buf];
-
-    for (int layer = 0; layer < a.n_layers; ++layer) {
-      if (weights_pending) {
-        if (tid == 0 && !mbar_wait(&meta.bar_w, ph_w)) meta.fail = 1;
-        ph_w ^= 1u;
-        weights_pending = false;
-      }
-      __syncthreads();
-      if (meta.fail) break;
-
-      // ---- 1. QKV = X . W (rows >= `rows` of X hold stale data; their outputs are unused)
-      {
-        const int rg = tid / NCG, cg = tid % NCG;
-        T acc[TM][TN];
-#pragma unroll
-        for (int i = 0; i < TM; ++i)
-#pragma unroll
-          for (int j = 0; j < TN; ++j) acc[i][j] = T(0);
-        const T* xr = X + (rg * TM) * C;
-#pragma unroll 2
-        for (int k = 0; k < C; k += 4) {
-          T xv[TM][4];
-#pragma unroll
-          for (int i = 0; i < TM; ++i)
-#pragma unroll
-            for (int u = 0; u < 4; ++u) xv[i][u] = xr[i * C + k + u];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            T wv[TN];
-#pragma unroll
-            for (int j = 0; j < TN; ++j) {
-              const int col = cg + NCG * j;
-              const int m = col / C, cc = col - m * C;
-              wv[j] = sW[m * C * C + (k + u) * C + cc];
-            }
-#pragma unroll
-            for (int i = 0; i < TM; ++i)
-#pragma unroll
-              for (int j = 0; j < TN; ++j) acc[i][j] = fma(xv[i][u], wv[j], acc[i][j]);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < TM; ++i) {
-          const int r = rg * TM + i;
-          const T s = r < rows ? sS[r] : T(0);
-#pragma unroll
-          for (int j = 0; j < TN; ++j) {
-            const int col = cg + NCG * j;
-            T v = acc[i][j];
-            if (col < C) v *= s * qscale;
-            else if (col < 2 * C) v *= s;
-            sQ[r * QS + col] = v;
-          }
-        }
-      }
-      __syncthreads();
-      // the next layer's weights stream in while the attention runs
-      // (with one buffer the next tile is not planned yet: any centre left may start one)
-      const bool more = layer + 1 < a.n_layers ||
-                        (XB == 2 ? meta.nrows[buf ^ 1] > 0 : meta.next_c < meta.c_end);
-      if (a.n_layers > 1 && tid == 0 && more) load_weights((layer + 1) % a.n_layers);
-      if (a.n_layers > 1) weights_pending = more;
-
-      // ---- 2. attention: warp tasks of 32 (head, row) pairs of one centre
-      tile_attention<T, C / D, D, C, NT, QS>(sQ, meta, buf, warp, lane);
-      __syncthreads();
-      for (int e = tid; e < rows * C; e += NT) {
-        const int r = e / C, col = e - r * C;
-        X[e] = sQ[r * QS + col];
-      }
-      __syncthreads();
-    }
-    if (meta.fail) break;
-    // ---- 3. write the tile back: one bulk copy of the contiguous slab
-    fence_proxy_async();
-    __syncthreads();
-    if (tid == 0) {
-      bulk_s2g(out + row0 * C, X, (uint32_t)(rows * C * sizeof(T)));
-      bulk_commit();
-      if (XB == 1) {
-        bulk_wait_read_all();
-        plan_and_load(0);
-      }
-    }
-    if (XB == 2) buf ^= 1;
-    __syncthreads();
-  }
-  if (tid == 0) {
-    bulk_wait_all();
-    if (meta.fail) {
-      atomicOr(a.status, kStatusTimeout);
-      // let copies in flight land before the CTA's shared memory is released
-      mbar_wait(&meta.bar_x[buf ^ 1], ph_x[buf ^ 1]);
-      mbar_wait(&meta.bar_w, ph_w);
-    } else if (weights_pending) {
-      mbar_wait(&meta.bar_w, ph_w);  // never left in flight at exit
     }
   }
 }

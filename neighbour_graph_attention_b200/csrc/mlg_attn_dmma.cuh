@@ -306,7 +306,10 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
     o1 = max(o1, __shfl_xor_sync(kFull, o1, 1));
     o1 = max(o1, __shfl_xor_sync(kFull, o1, 2));
     const double m0 = from_ord_hi(o0), m1 = from_ord_hi(o1);
+    // weights and O = P V_h block by block (a block's exponentials overlap
+    // the previous block's MMA), two accumulator chains (even / odd blocks)
     double l0 = 0.0, l1 = 0.0;
+    double o[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
 #pragma unroll
     for (int j = 0; j < NBC; ++j) {
       if (j < nkb) {
@@ -321,21 +324,14 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
             s[j][2 + e] = 0.0;
           }
         }
+        const double2 vv = lds2(sV + (h * D + g) * VS + off + 8 * j + 2 * t);
+        dmma_k8(o[j & 1], s[j][0], s[j][2], s[j][1], s[j][3], vv.x, vv.y);
       }
     }
     l0 += __shfl_xor_sync(kFull, l0, 1);
     l0 += __shfl_xor_sync(kFull, l0, 2);
     l1 += __shfl_xor_sync(kFull, l1, 1);
     l1 += __shfl_xor_sync(kFull, l1, 2);
-    // O = P V_h over two accumulator chains (even / odd key blocks)
-    double o[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
-#pragma unroll
-    for (int j = 0; j < NBC; ++j) {
-      if (j < nkb) {
-        const double2 vv = lds2(sV + (h * D + g) * VS + off + 8 * j + 2 * t);
-        dmma_k8(o[j & 1], s[j][0], s[j][2], s[j][1], s[j][3], vv.x, vv.y);
-      }
-    }
     const int r = qb * 16 + g;
     if (r < n) {
       const double i0 = 1.0 / l0;
@@ -393,6 +389,7 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
     om = max(om, __shfl_xor_sync(kFull, om, 2));
     const double m = from_ord_hi(om);
     double l = 0.0;
+    double o[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
 #pragma unroll
     for (int j = 0; j < NBC; ++j) {
       if (j < nkb) {
@@ -401,19 +398,13 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
           s[j][e] = exp2_neg(s[j][e] - m, tab);
           l += s[j][e];
         }
-      }
-    }
-    l += __shfl_xor_sync(kFull, l, 1);
-    l += __shfl_xor_sync(kFull, l, 2);
-    double o[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
-#pragma unroll
-    for (int j = 0; j < NBC; ++j) {
-      if (j < nkb) {
         const double2 vv = lds2(sV + (h * D + g) * VS + off + 8 * j + 2 * t);
         dmma884(o[j & 1][0], o[j & 1][1], s[j][0], vv.x);
         dmma884(o[j & 1][0], o[j & 1][1], s[j][1], vv.y);
       }
     }
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
     if (qr + g < n) {
       const double il = 1.0 / l;
       sts2(sXn + (q0 + g) * XS + h * D + 2 * t, (o[0][0] + o[1][0]) * il,

@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(NT) k_attn_hg(HgArgs a) {
       meta.next_c = c;
     }
     __syncthreads();
-    const int rows = meta.nrows[0], ncent = meta.ncent[0];
+    const int rows = meta.nrows[0];
     const int64_t row0 = meta.row0[0];
     if (rows == 0) break;
     for (int t = tid; t < rows; t += NT) sS[t] = (T)a.sw[row0 + t];

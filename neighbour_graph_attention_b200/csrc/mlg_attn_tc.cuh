@@ -134,16 +134,16 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
   using Cfg = TcCfg<C, D, NT>;
   constexpr int R = Cfg::R, N3 = Cfg::N3, QS = Cfg::QS, H = C / D;
   constexpr int NW = NT / 32, NQUART = NW / 4;  // warps per TMEM lane quadrant
-  extern __shared__ __align__(1024) unsigned char smem[];
-  float* sBhi = reinterpret_cast<float*>(smem + Cfg::OFF_BHI);
-  float* sBlo = reinterpret_cast<float*>(smem + Cfg::OFF_BLO);
-  float* sQ = reinterpret_cast<float*>(smem + Cfg::OFF_REG);
-  char* sAhi = reinterpret_cast<char*>(smem + Cfg::OFF_AHI);
-  char* sAlo = reinterpret_cast<char*>(smem + Cfg::OFF_ALO);
-  float* sX = reinterpret_cast<float*>(smem + (Cfg::PREFETCH ? Cfg::OFF_XP : Cfg::OFF_X));
-  float* sS = reinterpret_cast<float*>(smem + Cfg::OFF_S);
-  TileMeta& meta = *reinterpret_cast<TileMeta*>(smem + Cfg::OFF_META);
-  uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  extern __shared__ __align__(1024) unsigned char smem_tc[];
+  float* sBhi = reinterpret_cast<float*>(smem_tc + Cfg::OFF_BHI);
+  float* sBlo = reinterpret_cast<float*>(smem_tc + Cfg::OFF_BLO);
+  float* sQ = reinterpret_cast<float*>(smem_tc + Cfg::OFF_REG);
+  char* sAhi = reinterpret_cast<char*>(smem_tc + Cfg::OFF_AHI);
+  char* sAlo = reinterpret_cast<char*>(smem_tc + Cfg::OFF_ALO);
+  float* sX = reinterpret_cast<float*>(smem_tc + (Cfg::PREFETCH ? Cfg::OFF_XP : Cfg::OFF_X));
+  float* sS = reinterpret_cast<float*>(smem_tc + Cfg::OFF_S);
+  TileMeta& meta = *reinterpret_cast<TileMeta*>(smem_tc + Cfg::OFF_META);
+  uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem_tc + Cfg::OFF_BAR);
   uint64_t* bar_mma = bar_x + 1;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_x + 2);
 

@@ -55,13 +55,13 @@ __device__ __forceinline__ float exp_t<float>(float x) { return expf(x); }
 
 template <typename T>
 __global__ void __launch_bounds__(kLocalThreads) k_local_attn(LocalArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(16) unsigned char smem_local[];
   const int c = a.channels, H = a.heads, d = c / H, NM = a.nnei_max;
-  T* sx = reinterpret_cast<T*>(smem);  // [c]     the centre's feature row
-  T* sq = sx + c;                      // [c]     q = x Wq
-  T* su = sq + c;                      // [H][c]  u^h
-  T* sz = su + (size_t)H * c;          // [H][c]  z^h
-  T* sp = sz + (size_t)H * c;          // [H][NM] logits, then weights
+  T* sx = reinterpret_cast<T*>(smem_local);  // [c]     the centre's feature row
+  T* sq = sx + c;                             // [c]     q = x Wq
+  T* su = sq + c;                             // [H][c]  u^h
+  T* sz = su + (size_t)H * c;                 // [H][c]  z^h
+  T* sp = sz + (size_t)H * c;                 // [H][NM] logits, then weights
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, NW = blockDim.x >> 5;
   const T* Hn = static_cast<const T*>(a.H);
   const T* G = static_cast<const T*>(a.G);

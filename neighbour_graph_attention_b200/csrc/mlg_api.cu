@@ -264,7 +264,7 @@ int sm_count();
 // Small systems on per-cell scans take the one-launch build.
 bool use_fused_build(const BuildPlan& plan, int64_t n) {
   return plan.max_reach <= 1 && n >= 1 && n <= kFusedMaxAtoms &&
-         fused_build_fits(n, plan.ncell_cap);
+         fused_build_fits<kCellCand>(n, plan.ncell_cap);
 }
 
 // Arguments of the build kernels for one system whose workspace starts at w
@@ -368,6 +368,35 @@ void launch_fill_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
   }
 }
 
+// The one-launch build with stage capacity CAP; MLG_ERR_UNSUPPORTED if the
+// driver refuses the cooperative launch (the caller then runs the chain).
+template <int CAP>
+int launch_fused_build(const BuildArgs& a, const BuildPlan& plan, int nsplit, FusedSync* sync,
+                       cudaStream_t stream) {
+  const int64_t n = a.n;
+  const size_t smem = fused_build_smem<CAP>(n);
+  auto kern = k_build_fused<CAP>;
+  prefer_shared(kern, smem);
+  const int64_t cap = (int64_t)resident_blocks(kern, kCellWarps * 32, smem) * sm_count();
+  const int64_t nitems = (int64_t)plan.ncell_cap * nsplit;
+  const int grid = (int)(nitems < cap ? nitems : cap);
+  if (cudaMemsetAsync(sync, 0, sizeof(FusedSync), stream) != cudaSuccess) return MLG_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kCellWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, a, plan, plan.ncell_cap, nsplit, sync) == cudaSuccess)
+    return launch_status();
+  (void)cudaGetLastError();
+  return MLG_ERR_UNSUPPORTED;
+}
+
 int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
                const mlg_csr* csr, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (sys == nullptr || sys->coords == nullptr) return MLG_ERR_INVALID_ARG;
@@ -385,28 +414,14 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   const BuildArgs a = make_build_args(sys, rcut, r_on, nnei_max, csr, w, L);
   const int nsplit = build_nsplit(plan);
   if (use_fused_build(plan, n)) {
-    // the whole build in one cooperative launch (small systems)
-    const size_t smem = fused_build_smem(n);
-    prefer_shared(k_build_fused, smem);
-    const int64_t cap = (int64_t)resident_blocks(k_build_fused, kCellWarps * 32, smem) * sm_count();
-    const int64_t nitems = (int64_t)plan.ncell_cap * nsplit;
-    const int grid = (int)(nitems < cap ? nitems : cap);
+    // the whole build in one cooperative launch (small systems); systems of
+    // at most 75 atoms take the larger stage, which holds any 27-cell stencil
+    // (27 n candidates) so that no centre takes the global-memory traversal
     FusedSync* sync = reinterpret_cast<FusedSync*>(w + L.sync);
-    if (cudaMemsetAsync(sync, 0, sizeof(FusedSync), stream) != cudaSuccess) return MLG_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kCellWarps * 32);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, k_build_fused, a, plan, plan.ncell_cap, nsplit, sync) ==
-        cudaSuccess)
-      return launch_status();
-    (void)cudaGetLastError();  // refused (not co-resident): the launch chain below
+    const int rc2 = 27 * n <= kCellCandSmall
+                        ? launch_fused_build<kCellCandSmall>(a, plan, nsplit, sync, stream)
+                        : launch_fused_build<kCellCand>(a, plan, nsplit, sync, stream);
+    if (rc2 != MLG_ERR_UNSUPPORTED) return rc2;  // refused (not co-resident): the chain below
   }
   launch_count_phase(a, plan, nsplit, stream);
   launch_scan<long long>(a.kept, n, reinterpret_cast<long long*>(a.row_ptr), a.partial,

@@ -662,10 +662,20 @@ __device__ __forceinline__ unsigned long long edge_key(int j, int tpack) {
 }
 
 // Key of a candidate staged in shared memory: the same (source, image) order
-// as edge_key, with the staging slot (< 1024) in the low 10 bits.
+// as edge_key, with the staging slot (< 2048) in the low 11 bits.
+constexpr int kSlotBits = 11;
 __device__ __forceinline__ unsigned long long staged_key(int j, int tpack, int slot) {
-  return ((unsigned long long)(unsigned)j << 31) | ((unsigned long long)tpack << 10) |
-         (unsigned long long)slot;
+  return ((unsigned long long)(unsigned)j << (21 + kSlotBits)) |
+         ((unsigned long long)tpack << kSlotBits) | (unsigned long long)slot;
+}
+__device__ __forceinline__ int staged_src(unsigned long long key) {
+  return (int)(key >> (21 + kSlotBits));
+}
+__device__ __forceinline__ int staged_image(unsigned long long key) {
+  return (int)((key >> kSlotBits) & 0x1fffffull);
+}
+__device__ __forceinline__ int staged_slot(unsigned long long key) {
+  return (int)(key & ((1ull << kSlotBits) - 1));
 }
 
 // Selection for rows with more than kFillMaxCand candidates, without a
@@ -737,9 +747,9 @@ __device__ __forceinline__ void write_edge(const BuildArgs& a, const Centre& cc,
   int j, tp, wj;
   double xj[3];
   if (srec != nullptr) {
-    j = (int)(key >> 31);
-    tp = (int)((key >> 10) & 0x1fffffull);
-    const Rec& rc = srec[key & 1023ull];
+    j = staged_src(key);
+    tp = staged_image(key);
+    const Rec& rc = srec[staged_slot(key)];
     wj = rc.w;
     xj[0] = rc.x;
     xj[1] = rc.y;
@@ -877,11 +887,13 @@ __global__ void __launch_bounds__(kFillWarps * 32) k_fill(BuildArgs a) {
 // records are staged too, so the fp64 tests and the edge output read shared
 // memory only.  Cells whose stencil holds more than kCellCand atoms fall back
 // to the per-centre traversal of global memory.
-constexpr int kCellCand = 768;
+constexpr int kCellCand = 768;       // stage capacity of the kernel chain
+constexpr int kCellCandSmall = 2048; // one-launch build of systems of at most 75 atoms
 constexpr int kCellWarps = 8;
-static_assert(kCellCand <= 1024, "staged_key keeps 10 bits of slot");
+static_assert(kCellCandSmall <= (1 << kSlotBits), "staged_key slot bits");
 
-struct CellStage {
+template <int CAP>
+struct CellStageT {
   int pre[33];      // candidate offset of each stencil cell
   int start[32];
   int tpack[32];
@@ -893,19 +905,25 @@ struct CellStage {
   int c_lo, c_hi;           // the staged cell's centres (cell-order range)
   int stash_ci[kCellWarps];   // STASH: centre whose accepted keys a warp still holds (-1: none)
   int stash_cnt[kCellWarps];  // and how many
-  float4 cand[kCellCand];   // position + image offset, atom index in .w
-  int cq[kCellCand];        // cell-order index (record of the exact data)
-  int ct[kCellCand];        // packed image of the stencil cell
+  float4 cand[CAP];   // position + image offset, atom index in .w
+  int cq[CAP];        // cell-order index (record of the exact data)
+  int ct[CAP];        // packed image of the stencil cell
 };
+using CellStage = CellStageT<kCellCand>;
 
 // Dynamic shared memory of the per-cell scans: the stage, the fill's key
 // buffers, and (REC) the candidates' exact records.
-constexpr size_t kCellKeysOff = ((sizeof(CellStage) + 15) / 16) * 16;
 constexpr size_t kCellKeysBytes = (size_t)kCellWarps * 2 * kFillMaxCand * sizeof(unsigned long long);
-constexpr size_t kCellRecOff = kCellKeysOff + kCellKeysBytes;
+template <int CAP>
+struct CellSmem {
+  static constexpr size_t keys_off = ((sizeof(CellStageT<CAP>) + 15) / 16) * 16;
+  static constexpr size_t rec_off = keys_off + kCellKeysBytes;
+  static constexpr size_t bytes(bool fill, bool rec) {
+    return rec ? rec_off + (size_t)CAP * sizeof(Rec) : keys_off + (fill ? kCellKeysBytes : 0);
+  }
+};
 __host__ __device__ constexpr size_t cellscan_smem(bool fill, bool rec = false) {
-  return rec ? kCellRecOff + (size_t)kCellCand * sizeof(Rec)
-             : kCellKeysOff + (fill ? kCellKeysBytes : 0);
+  return CellSmem<kCellCand>::bytes(fill, rec);
 }
 
 // Count (FILL = false: raw, kept, truncations) or fill (FILL: the CSR rows)
@@ -916,13 +934,14 @@ __host__ __device__ constexpr size_t cellscan_smem(bool fill, bool rec = false) 
 // the same cell from an earlier call are reused.  With STASH (and REC) the
 // count keeps each warp's accepted keys and distances in its key buffer, and
 // a fill of the same centre by the same warp starts from them.
-template <bool FILL, bool REC, bool STASH = false>
+template <bool FILL, bool REC, bool STASH = false, int CAP = kCellCand>
 __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratch* sws,
                               unsigned char* s_dyn, int cell, int ys, int nsplit,
                               const int* row_off) {
-  CellStage& cs = *reinterpret_cast<CellStage*>(s_dyn);
-  unsigned long long* s_keys = reinterpret_cast<unsigned long long*>(s_dyn + kCellKeysOff);
-  Rec* s_rec = reinterpret_cast<Rec*>(s_dyn + kCellRecOff);  // REC only
+  CellStageT<CAP>& cs = *reinterpret_cast<CellStageT<CAP>*>(s_dyn);
+  unsigned long long* s_keys =
+      reinterpret_cast<unsigned long long*>(s_dyn + CellSmem<CAP>::keys_off);
+  Rec* s_rec = reinterpret_cast<Rec*>(s_dyn + CellSmem<CAP>::rec_off);  // REC only
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (cell >= sg.ncell) return;
   const bool reuse = cs.staged_cell == cell;
@@ -972,7 +991,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
       if (lane == 31) {
         cs.pre[32] = incl;
         cs.ncand = incl;
-        cs.fallback = incl > kCellCand;
+        cs.fallback = incl > CAP;
         cs.trunc = 0;
         cs.staged_cell = cell;
         cs.c_lo = c_lo;
@@ -1127,8 +1146,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
       for (int q = lane; q < cnt; q += 32) {
         const unsigned long long key = keys[q];
         double r2;
-        test_candidate(sg, cc, s_rec[key & 1023ull], (int)((key >> 10) & 0x1fffffull), a.rc2,
-                       &r2);
+        test_candidate(sg, cc, s_rec[staged_slot(key)], staged_image(key), a.rc2, &r2);
         keys[kFillMaxCand + q] = (unsigned long long)__double_as_longlong(r2);
       }
     }
@@ -1366,20 +1384,23 @@ __device__ __forceinline__ bool wait_at_least(const unsigned* p, unsigned want) 
 // Dynamic shared memory of the one-launch build: the per-cell scan's, then
 // the row starts; CTA 0's binning scratch (histogram and three per-atom
 // arrays) must fit in the same bytes.
+template <int CAP>
 __host__ __device__ constexpr size_t fused_build_smem(int64_t n) {
-  return cellscan_smem(true, true) + (size_t)(n + 1) * sizeof(int);
+  return CellSmem<CAP>::bytes(true, true) + (size_t)(n + 1) * sizeof(int);
 }
+template <int CAP>
 __host__ __device__ constexpr bool fused_build_fits(int64_t n, int ncell_cap) {
-  return (size_t)(ncell_cap + 1 + 3 * n) * sizeof(int) <= fused_build_smem(n);
+  return (size_t)(ncell_cap + 1 + 3 * n) * sizeof(int) <= fused_build_smem<CAP>(n);
 }
 
+template <int CAP>
 __global__ void __launch_bounds__(kCellWarps * 32, 2)
     k_build_fused(BuildArgs a, BuildPlan p, int ncell_cap, int nsplit, FusedSync* sync) {
   __shared__ CellGrid sg;
   __shared__ WarpScratch sws[kCellWarps];
   __shared__ int s_ok;
   extern __shared__ __align__(16) unsigned char s_dyn[];
-  int* s_off = reinterpret_cast<int*>(s_dyn + cellscan_smem(true, true));  // [n + 1] row starts
+  int* s_off = reinterpret_cast<int*>(s_dyn + CellSmem<CAP>::bytes(true, true));  // [n + 1] row starts
   const int tid = threadIdx.x;
   const unsigned tout = MLG_STATUS_TIMEOUT;
 
@@ -1445,7 +1466,7 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2)
   if (tid == 0) {
     s_ok = blockIdx.x == 0 ? 1 : (wait_at_least(&sync->ready, 1u) ? 1 : 0);
     if (s_ok && blockIdx.x != 0) sg = *a.grid;
-    reinterpret_cast<CellStage*>(s_dyn)->staged_cell = -1;
+    reinterpret_cast<CellStageT<CAP>*>(s_dyn)->staged_cell = -1;
   }
   __syncthreads();
   if (!s_ok) {
@@ -1456,8 +1477,8 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2)
   // ---- count pass (keys kept for the fill)
   const int nitems = sg.ncell * nsplit;
   for (int item = blockIdx.x; item < nitems; item += gridDim.x)
-    cellscan_item<false, true, true>(a, sg, sws, s_dyn, item / nsplit, item % nsplit, nsplit,
-                                     nullptr);
+    cellscan_item<false, true, true, CAP>(a, sg, sws, s_dyn, item / nsplit, item % nsplit,
+                                          nsplit, nullptr);
 
   // ---- grid barrier: every count is written
   __syncthreads();
@@ -1479,8 +1500,8 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2)
                           ScanTail{a.n_edges, a.status, a.capacity});
   __syncthreads();
   for (int item = blockIdx.x; item < nitems; item += gridDim.x)
-    cellscan_item<true, true, true>(a, sg, sws, s_dyn, item / nsplit, item % nsplit, nsplit,
-                                    s_off);
+    cellscan_item<true, true, true, CAP>(a, sg, sws, s_dyn, item / nsplit, item % nsplit,
+                                         nsplit, s_off);
 }
 
 }  // namespace mlg

@@ -1,17 +1,18 @@
 // mlg_attn_dmma.cuh -- fused multi-layer block-dense attention in fp64 on the
-// FP64 tensor pipe (mma.sync m16n8k8 / m16n8k16 .f64, sm_100a).
+// FP64 tensor pipe (mma.sync m16n8k16 / m16n8k8 / m8n8k4 .f64, sm_100a).
 //
 // The per-centre attention of the NeighborGraph issue (Proposed fix: dense
 // attention per centre with masks for the ragged tail, written back to the
 // edge axis), for c = 32 channels, 4 heads of d = 8, in fp64.  Every product
-// is a 16x8 fp64 MMA:
-//   K   [rows][32] = X . Wk               m16n8k16, 16-row blocks
+// is an fp64 MMA:
+//   K   [rows][32] = X . Wk               m16n8k16, 16-row blocks of the tile
 //   V^T [32][rows] = Wv^T . X^T           m16n8k16, 8-row blocks (stored transposed)
 //   Q_h [16][8]    = X . Wq_h             m16n8k16, kept in registers
 //   S   [16][8]    = Q_h . K_h^T          m16n8k8 per 8-key block
 //   O   [16][8]   += P . V_h              m16n8k8 per 8-key block
 // A centre's last query rows, when 8 or fewer, take the same three products
-// on 8-row blocks (m8n8k4), so no MMA row is padding.
+// on 8-row blocks (m8n8k4), so no MMA row is padding and no query block runs
+// past its centre's rows.
 // A contraction may visit its k index in any order, so each one permutes it
 // to suit the fragments at hand: the projections read channel 4t + m at k
 // slot t + 4m (both operands then come in contiguous 16-byte pieces); the
@@ -20,14 +21,18 @@
 // is the column layout of the S accumulator.  So Q and P never leave
 // registers and need no shuffles.
 // Softmax: each lane holds two query rows (g and g + 8) of every 8-key
-// block; the row max and sum take two shuffles each; exponentials are in
-// base 2 (log2 e is folded into the Q scale) by a table-driven method.
+// block.  The row maxima are taken on the integer pipe from the doubles' high
+// words, the sums by two shuffles; exponentials are in base 2 (log2 e is
+// folded into the Q scale) by a table-driven method, block by block, each
+// block's exponentials overlapping the previous block's P V MMA.  The FP64
+// MMA and the DFMA share one pipe, so the softmax keeps its FP64 work small.
 // Rows of a centre are padded to a multiple of 8 with zero features (their
-// keys are masked to -inf and their values are 0); query blocks of 16 rows
-// may run past a centre into rows that are only read, never written.
+// keys are masked to -inf and their values are 0).
 // One CTA per SM holds a tile of consecutive centres for all layers: the
 // layer's input X and its output ping-pong between two buffers, and only the
-// last layer's output goes back to global memory.
+// last layer's output goes back to global memory.  A layer is phase A (K and
+// V^T of the whole tile) and phase B (units of equal work: one 16-row query
+// block and head, or two heads of an 8-row block), with a barrier after each.
 #pragma once
 
 #include "mlg_common.cuh"

@@ -48,7 +48,7 @@ FP32_PEAK_TFLOPS = SM_COUNT * 128 * 2 * SM_MAX_GHZ / 1e3
 # it stands exists.  A change to a kernel resets its entry to None.
 ATTN_KERNEL = {
     1: ("k_attn_hg<double,128,32,...>", None),
-    2: ("k_attn_dmma<160,5,640>", None),
+    2: ("k_attn_dmma<160,5,640>", 5.622e6),   # profiles/k_attn_dmma_f64_diamond512.md
     3: ("k_attn_tc<64,16,512>", None),
     4: ("k_attn_hg<float,128,16,...>", None),
     5: ("k_attn_tc<32,8,512>", None),

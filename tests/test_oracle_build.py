@@ -321,3 +321,25 @@ def test_triclinic_brute_force(oracle_mod):
         rows = _rows(csr)[i]
         got = [(int(j), *map(int, S)) for j, S in zip(csr["src"][rows], csr["shift"][rows])]
         assert got == sorted(want)
+
+
+@pytest.mark.parametrize("lattice", ["diamond", "bcc"])
+def test_golden_shells_match_lattice_enumeration(lattice):
+    """The stored shell table against a direct count of lattice sites (no
+    oracle): every site of an ideal cubic lattice within a few cells of a
+    site at the origin, grouped by squared distance in the table's unit."""
+    basis = {"diamond": [(0, 0, 0), (0, 2, 2), (2, 0, 2), (2, 2, 0),
+                         (1, 1, 1), (1, 3, 3), (3, 1, 3), (3, 3, 1)],   # in units of a/4
+             "bcc": [(0, 0, 0), (1, 1, 1)]}[lattice]                    # in units of a/2
+    period = {"diamond": 4, "bcc": 2}[lattice]
+    r = np.arange(-5, 6)
+    cells = np.stack(np.meshgrid(r, r, r, indexing="ij"), axis=-1).reshape(-1, 3) * period
+    sites = (cells[:, None, :] + np.array(basis)[None, :, :]).reshape(-1, 3)
+    d2 = (sites ** 2).sum(axis=1)          # squared distance in units of (a/4)^2 or (a/2)^2
+    table = {int(k): v for k, v in _GOLDEN[lattice]["shells"].items()}
+    for k, count in table.items():
+        assert k < (5 * period) ** 2       # inside the enumerated cube
+        assert int((d2 == k).sum()) == count, (lattice, k)
+    # and no shell below the table's largest is missing from it
+    for k in np.unique(d2[(d2 > 0) & (d2 <= max(table))]):
+        assert int(k) in table, (lattice, int(k))

@@ -75,6 +75,9 @@ def _load():
             lib.oracle_attention.argtypes = [i64, p, p, i32, i32, p, p, p, p, p, ctypes.c_int]
             lib.oracle_attention_map.restype = ctypes.c_int
             lib.oracle_attention_map.argtypes = [p, p, i32, i32, p, p, p, i64, i32, p]
+            lib.oracle_attention_smooth.restype = ctypes.c_int
+            lib.oracle_attention_smooth.argtypes = [i64, p, p, i32, i32, i32, p, p, p, p, p,
+                                                    ctypes.c_int]
             lib.oracle_local_attention.restype = ctypes.c_int
             lib.oracle_local_attention.argtypes = [i64, p, p, i32, i32, p, p, p, p, p, p,
                                                    ctypes.c_int]
@@ -193,6 +196,30 @@ def attention(row_ptr, sw, G, Wq, Wk, Wv, heads: int, nthreads: int = 0) -> np.n
                                   int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_attention failed ({rc})")
+    return out
+
+
+def attention_smooth(row_ptr, sw, G, Wq, Wk, Wv, heads: int, nnei_max: int,
+                     nthreads: int = 0) -> np.ndarray:
+    """Slot-occupancy ("smooth") attention (NeighborGraph issue, Numerics note:
+    signed phantom count and slot-occupancy denominator; the weights factor as
+    w_b = softmax_b * sum_b e_b / D~).
+
+    As ``attention``, plus phi = nnei_max - n phantom slots per centre with
+    logit exactly 0 and value 0 -- the dense route's zero-padded slots, left
+    unmasked: m = max(max_b l_ab, 0 if phi > 0),
+    D~ = sum_b e^(l_ab - m) + phi e^(-m), O_a = sum_b e^(l_ab - m) V_b / D~.
+    """
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int64)
+    sw, G = _as_f64(sw), _as_f64(G)
+    Wq, Wk, Wv = _as_f64(Wq), _as_f64(Wk), _as_f64(Wv)
+    c = G.shape[1]
+    out = np.zeros_like(G)
+    rc = _load().oracle_attention_smooth(row_ptr.size - 1, _ptr(row_ptr), _ptr(sw), c,
+                                         int(heads), int(nnei_max), _ptr(G), _ptr(Wq), _ptr(Wk),
+                                         _ptr(Wv), _ptr(out), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_smooth failed ({rc})")
     return out
 
 

@@ -28,6 +28,15 @@
  *    ragged tails, scattered back to the edge axis): Q = G Wq, K = G Wk,
  *    V = G Wv; per head l_ab = s_a s_b (q_a . k_b) / sqrt(d); softmax over
  *    the centre's real edges b; O_a = sum_b P_ab V_b.
+ *  - Slot-occupancy ("smooth") attention (NeighborGraph issue, Numerics note and
+ *    "Graph-native alternatives": a signed phantom count and a slot-occupancy
+ *    denominator; the weights factor as w_b = softmax_b * (sum_b e_b / D~)).
+ *    Reading: the dense route pads every centre to nnei_max slots with zero
+ *    features and zero switch, so a padded slot's logit is exactly 0 and,
+ *    unmasked, it enters the softmax denominator; it adds nothing to the
+ *    numerator (its value row is 0).  With phi = nnei_max - n phantoms:
+ *    m = max(max_b l_ab, 0 if phi > 0), D~ = sum_b e^(l_ab - m) + phi e^(-m),
+ *    O_a = sum_b e^(l_ab - m) V_b / D~.
  *  - Local attention, one query per centre (NeighborGraph issue, "Graph-native
  *    alternatives", item 2: LocalAtten maps onto the per-centre CSR segment
  *    with queries = centres and keys = edges): q_i = H_i Wq from the centre's
@@ -583,6 +592,82 @@ int oracle_local_attention(int64_t n_centres, const int64_t* row_ptr, const doub
             }
         }
         free(q); free(K); free(V); free(P);
+    }
+    return err;
+}
+
+/* Slot-occupancy ("smooth") attention over every centre: as oracle_attention,
+ * plus phi = nnei_max - n phantom slots of logit exactly 0 and value 0 in the
+ * softmax of every row (the dense route's zero-padded, unmasked slots):
+ * m = max(max_b l_ab, 0 if phi > 0), D~ = sum_b e^(l_ab - m) + phi e^(-m),
+ * O_a = sum_b e^(l_ab - m) V_b / D~.  Centres with n > nnei_max are an error
+ * (phi would be negative). */
+int oracle_attention_smooth(int64_t n_centres, const int64_t* row_ptr, const double* sw,
+                            int32_t c, int32_t heads, int32_t nnei_max, const double* G,
+                            const double* Wq, const double* Wk, const double* Wv, double* out,
+                            int nthreads) {
+    if (n_centres < 0 || c <= 0 || heads <= 0 || c % heads != 0 || nnei_max < 1)
+        return ORC_ERR_ARG;
+    for (int64_t i = 0; i < n_centres; ++i)
+        if (row_ptr[i + 1] - row_ptr[i] > nnei_max) return ORC_ERR_ARG;
+    int d = c / heads;
+    double rsd = sqrt((double)d);
+    set_threads(nthreads);
+    int err = ORC_OK;
+#pragma omp parallel
+    {
+        double *Q = NULL, *K = NULL, *V = NULL, *E = NULL;
+        int64_t have = 0;
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t i = 0; i < n_centres; ++i) {
+            int64_t base = row_ptr[i];
+            int64_t n = row_ptr[i + 1] - base;
+            if (n <= 0) continue;
+            if (n > have) {
+                free(Q); free(K); free(V); free(E);
+                Q = (double*)malloc((size_t)(n * c) * sizeof(double));
+                K = (double*)malloc((size_t)(n * c) * sizeof(double));
+                V = (double*)malloc((size_t)(n * c) * sizeof(double));
+                E = (double*)malloc((size_t)n * sizeof(double));
+                have = n;
+                if (!Q || !K || !V || !E) {
+#pragma omp atomic write
+                    err = ORC_ERR_MEM;
+                    have = 0;
+                    continue;
+                }
+            }
+            const double* x = G + base * c;
+            const double* s = sw + base;
+            int64_t phi = nnei_max - n;
+            project(n, c, x, Wq, Q);
+            project(n, c, x, Wk, K);
+            project(n, c, x, Wv, V);
+            for (int h = 0; h < heads; ++h)
+                for (int64_t a = 0; a < n; ++a) {
+                    double m = phi > 0 ? 0.0 : -INFINITY;
+                    for (int64_t b = 0; b < n; ++b) {
+                        double dot = 0.0;
+                        for (int t = 0; t < d; ++t)
+                            dot = dot + Q[a * c + h * d + t] * K[b * c + h * d + t];
+                        double l = ((s[a] * s[b]) * dot) / rsd;
+                        E[b] = l;
+                        if (l > m) m = l;
+                    }
+                    double z = 0.0;
+                    for (int64_t b = 0; b < n; ++b) {
+                        E[b] = exp(E[b] - m);
+                        z = z + E[b];
+                    }
+                    if (phi > 0) z = z + (double)phi * exp(-m);  /* m >= 0 here */
+                    for (int t = 0; t < d; ++t) {
+                        double acc = 0.0;
+                        for (int64_t b = 0; b < n; ++b) acc = acc + (E[b] / z) * V[b * c + h * d + t];
+                        out[(base + a) * c + h * d + t] = acc;
+                    }
+                }
+        }
+        free(Q); free(K); free(V); free(E);
     }
     return err;
 }

@@ -185,6 +185,21 @@ int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                         void* G_out, const void* Wq, const void* Wk, const void* Wv, void* ws,
                         size_t ws_bytes, mlg_stream_t stream);
 
+/* One attention layer with the slot-occupancy ("smooth") softmax (NeighborGraph
+ * issue, Numerics note: a phantom count and a slot-occupancy denominator; the
+ * weights factor as w_b = softmax_b * sum_b e_b / D~).  As mlg_block_attention,
+ * plus phi = nnei_max - n phantom slots per destination: the zero-padded
+ * slots of the dense (nloc, nnei_max, c) route, left unmasked, whose logit is
+ * exactly 0 and whose value is 0:
+ *   m_a = max(max_b l_ab, 0 if phi > 0),  D~ = sum_b exp(l_ab - m_a) + phi exp(-m_a),
+ *   G_out[a, h d + t] = sum_b exp(l_ab - m_a) v_b[t] / D~.
+ * Destinations with more than nnei_max edges are left untouched.  Runs on
+ * the generic kernel (no fused tiles yet); no workspace. */
+int mlg_block_attention_smooth(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                               int32_t channels, int32_t heads, mlg_dtype dtype,
+                               const void* G_in, void* G_out, const void* Wq, const void* Wk,
+                               const void* Wv, mlg_stream_t stream);
+
 /* Bytes of device workspace that mlg_attention_stack needs: one [capacity][channels] buffer
  * for n_layers >= 2 (used only by centres the fused kernels do not cover), else 0. */
 size_t mlg_attention_stack_workspace_bytes(int64_t capacity, int32_t channels, int32_t n_layers,

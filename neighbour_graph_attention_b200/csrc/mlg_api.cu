@@ -532,7 +532,8 @@ int sm_count() {
 // One layer of the generic kernel over the centres with more than min_n edges.
 int launch_generic(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max, int32_t C, int32_t H,
                    mlg_dtype dtype, const void* G_in, void* G_out, const void* Wq,
-                   const void* Wk, const void* Wv, int min_n, cudaStream_t stream) {
+                   const void* Wk, const void* Wv, int min_n, cudaStream_t stream,
+                   int smooth = 0) {
   AttnArgs a;
   a.row_ptr = csr->row_ptr;
   a.sw = csr->sw;
@@ -549,6 +550,7 @@ int launch_generic(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max, int3
   a.Wv = Wv;
   a.status = csr->status;
   a.min_n = min_n;
+  a.smooth = smooth;
   int64_t want = (int64_t)sm_count() * 4;
   int grid = (int)(n_centres < want ? n_centres : want);
   if (dtype == MLG_F64) {
@@ -870,6 +872,18 @@ int mlg_local_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
   if (dtype == MLG_F64)
     return go(k_local_attn<double>, local_smem<double>(channels, heads, nnei_max));
   return go(k_local_attn<float>, local_smem<float>(channels, heads, nnei_max));
+}
+
+int mlg_block_attention_smooth(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                               int32_t channels, int32_t heads, mlg_dtype dtype,
+                               const void* G_in, void* G_out, const void* Wq, const void* Wk,
+                               const void* Wv, mlg_stream_t stream) {
+  int rc = check_attention_args(csr, n_centres, nnei_max, channels, heads, dtype, G_in, G_out);
+  if (rc != MLG_OK) return rc;
+  if (!Wq || !Wk || !Wv) return MLG_ERR_INVALID_ARG;
+  if (n_centres == 0) return MLG_OK;
+  return launch_generic(csr, n_centres, nnei_max, channels, heads, dtype, G_in, G_out, Wq, Wk, Wv,
+                        0, (cudaStream_t)stream, 1);
 }
 
 size_t mlg_attention_stack_workspace_bytes(int64_t capacity, int32_t channels, int32_t n_layers,

@@ -14,6 +14,10 @@
 //   q_a = G_a Wq, k_b = G_b Wk, v_b = G_b Wv
 //   l_ab = s_a s_b (q_a . k_b) / sqrt(d)
 //   O_a = sum_b exp(l_ab - m_a) v_b / sum_b exp(l_ab - m_a),  m_a = max_b l_ab
+// With `smooth` (slot-occupancy softmax, NeighborGraph issue, Numerics note:
+// a phantom count and a slot-occupancy denominator), the centre's
+// phi = nnei_max - n padded slots take part as phantoms of logit 0 and value
+// 0: m_a = max(max_b l_ab, 0) and the denominator gains phi exp(-m_a).
 #pragma once
 
 #include "mlg_common.cuh"
@@ -34,6 +38,7 @@ struct AttnArgs {
   const void* Wv;
   uint32_t* status;
   int min_n;  // only centres with more than min_n edges (0: all)
+  int smooth;  // slot-occupancy softmax (phantom slots up to nnei_max)
 };
 
 template <typename T>
@@ -89,8 +94,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn_generic(AttnArgs a) {
       __syncthreads();
       // one warp per query row: logits, softmax, AV
       T* p = sP + (size_t)warp * NM;
+      const int phi = a.smooth ? NM - n : 0;  // phantom slots of logit 0, value 0
       for (int r = warp; r < n; r += kAttnWarps) {
-        T mx = -INFINITY;
+        T mx = phi > 0 ? T(0) : -INFINITY;
         for (int b = lane; b < n; b += 32) {
           T l = T(0);
           for (int t = 0; t < D; ++t) l += sQ[r * DP + t] * sK[b * DP + t];
@@ -105,6 +111,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn_generic(AttnArgs a) {
           z += e;
         }
         z = warp_sum(z);
+        if (phi > 0) z += T(phi) * fast_exp<T>(-mx);  // mx >= 0 here
         __syncwarp();
         const T rz = T(1) / z;
         for (int t = lane; t < D; t += 32) {

@@ -94,6 +94,9 @@ _lib.mlg_build_csr_batch_workspace_bytes.argtypes = [ctypes.POINTER(mlg_system),
 _lib.mlg_build_csr_batch.restype = ctypes.c_int
 _lib.mlg_build_csr_batch.argtypes = [ctypes.POINTER(mlg_system), _c_i32, _c_dbl, _c_dbl, _c_i32,
                                      ctypes.POINTER(mlg_csr), _p, _c_sz, _p]
+_lib.mlg_block_attention_smooth.restype = ctypes.c_int
+_lib.mlg_block_attention_smooth.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32,
+                                            _c_i32, ctypes.c_int, _p, _p, _p, _p, _p, _p]
 _lib.mlg_local_attention.restype = ctypes.c_int
 _lib.mlg_local_attention.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32, _c_i32,
                                      ctypes.c_int, _p, _p, _p, _p, _p, _p, _p]
@@ -293,6 +296,18 @@ def mlg_block_attention(csr: Csr, n_centres: int, nnei_max: int, channels: int, 
                                     _ptr(G_out), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(ws),
                                     int(ws_bytes), _stream_handle(stream))
     return _check(code, "mlg_block_attention", check)
+
+
+def mlg_block_attention_smooth(csr: Csr, n_centres: int, nnei_max: int, channels: int,
+                               heads: int, dtype: int, G_in, G_out, Wq, Wk, Wv, stream=None,
+                               check: bool = True) -> int:
+    """Launch one attention layer with the slot-occupancy (smooth) softmax."""
+    c = csr.struct()
+    code = _lib.mlg_block_attention_smooth(ctypes.byref(c), int(n_centres), int(nnei_max),
+                                           int(channels), int(heads), int(dtype), _ptr(G_in),
+                                           _ptr(G_out), _ptr(Wq), _ptr(Wk), _ptr(Wv),
+                                           _stream_handle(stream))
+    return _check(code, "mlg_block_attention_smooth", check)
 
 
 def _system_array(systems):

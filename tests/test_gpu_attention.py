@@ -301,3 +301,47 @@ def test_nan_feature_confined_to_its_centre():
     assert np.isnan(o6[bad]).all() and np.isfinite(o6[~bad]).all()
     ok, err = U.attn_tolerance_ok(w, o6[~bad], outs[-1][~bad])
     assert ok, err
+
+
+@pytest.mark.parametrize("case", ["f64-ragged", "f32-protein", "f64-full"])
+def test_smooth_attention_matches_oracle(case):
+    """The slot-occupancy softmax (phantom slots of logit 0 up to nnei_max) on
+    the GPU against the oracle: ragged rows (phantoms matter), the protein
+    cluster in fp32, and full rows (no phantoms: the plain attention)."""
+    import oracle
+    from neighbour_graph_attention_b200.configs import Workload
+
+    m = U.mlg()
+    if case == "f64-ragged":
+        gpu, csr_t = _random_graph(3000, 0.13, 4.2, 64, 17)
+        w = Workload(0, "random", "random", 0, 0, 0, 3000, 4.2, 3.7, 64, 32, 4, 1, "f64")
+        rng = np.random.default_rng(21)
+        W = [rng.normal(0, 1 / np.sqrt(32), (32, 32)) for _ in range(3)]
+        G = rng.normal(size=(gpu["n_edges"], 32))
+    else:
+        key = 4 if case == "f32-protein" else 1
+        w = C.workload(key)
+        gpu, csr_t = graph(key, 0)
+        W = C.weights(key, 0)[0]
+        G = C.features(key, 0, gpu["n_edges"])
+    dt = U.torch_dtype(w)
+    gin = torch.zeros((csr_t.capacity, w.channels), dtype=dt, device="cuda")
+    gin[: G.shape[0]] = torch.as_tensor(G, dtype=dt, device="cuda")
+    gout = torch.zeros_like(gin)
+    wq, wk, wv = (torch.as_tensor(np.ascontiguousarray(x), dtype=dt, device="cuda") for x in W)
+    m.mlg_block_attention_smooth(csr_t, w.n_atoms, w.nnei_max, w.channels, w.heads,
+                                 U.mlg_dtype(w), gin, gout, wq, wk, wv)
+    torch.cuda.synchronize()
+    assert int(csr_t.status.item()) == 0
+    out = gout[: G.shape[0]].cpu().numpy()
+    sw = gpu["sw"] if w.dtype == "f64" else gpu["sw"].astype(np.float32).astype(np.float64)
+    ref = oracle.attention_smooth(gpu["row_ptr"], sw, G, W[0], W[1], W[2], w.heads, w.nnei_max)
+    ok, err = U.attn_tolerance_ok(w, out, ref)
+    assert ok, err
+    counts = np.diff(gpu["row_ptr"])
+    if case == "f64-full":       # every row holds nnei_max edges: no phantom slots
+        assert int(counts.min()) == w.nnei_max
+    else:                        # phantoms present: differs from the plain softmax
+        assert int(counts.min()) < w.nnei_max
+        plain = oracle.attention(gpu["row_ptr"], sw, G, W[0], W[1], W[2], w.heads)
+        assert np.max(np.abs(ref - plain)) > 1e-6

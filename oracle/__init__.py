@@ -56,7 +56,10 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            # a deliberately broken copy of this library, compiled by the
+            # mutation tests, replaces it when named here (tests only)
+            alt = os.environ.get("MLG_ORACLE_LIB")
+            lib = ctypes.CDLL(alt if alt else build())
             i64, i32, dbl = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
             p = ctypes.c_void_p
             lib.oracle_cos_pi.restype = dbl
@@ -239,7 +242,7 @@ def local_attention(row_ptr, sw, H, G, Wq, Wk, Wv, heads: int, nthreads: int = 0
     n = row_ptr.size - 1
     if H.shape[0] != n:
         raise ValueError("H needs one row per centre")
-    out = np.zeros((n, c), dtype=np.float64)
+    out = np.full((n, c), np.nan)   # every row, empty centres too, is the C code's to write
     rc = _load().oracle_local_attention(n, _ptr(row_ptr), _ptr(sw), c, int(heads), _ptr(H),
                                         _ptr(G), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(out),
                                         int(nthreads))

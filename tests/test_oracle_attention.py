@@ -124,6 +124,21 @@ def test_two_edges_logistic_closed_form(oracle_mod):
     assert np.allclose(out[1], [sig(l10 - l11), sig(l11 - l10), 0, 0], rtol=0, atol=1e-15)
 
 
+def test_two_edges_large_logits(oracle_mod):
+    # the same closed form with logits of 1000 and 1500: e^l alone would
+    # overflow, the softmax itself does not (its value is shift-invariant)
+    G = np.array([[1.0, 0.0, 0.0, 0.0], [0.0, 1.0, 0.0, 0.0]])
+    Wq = np.zeros((4, 4)); Wq[0, 2] = 2000.0; Wq[1, 3] = 1.0
+    Wk = np.zeros((4, 4)); Wk[0, 2] = 1.0; Wk[1, 2] = 3.0
+    Wv = np.eye(4)
+    s = np.array([1.0, 0.5])
+    out = oracle_mod.attention(np.array([0, 2]), s, G, Wq, Wk, Wv, 1)
+    l00, l01 = 2000.0 / 2.0, 0.5 * 6000.0 / 2.0
+    assert np.all(np.isfinite(out))
+    assert out[0, 1] == 1.0 and 0.0 < out[0, 0] <= 1e-200
+    assert abs(out[0, 0] - 1.0 / (1.0 + math.exp(l01 - l00))) <= 1e-15 * out[0, 0]
+
+
 def test_other_centres_do_not_leak(oracle_mod):
     # masked slots contribute zero: rows outside a centre never enter it
     rng = np.random.default_rng(4)

@@ -78,6 +78,52 @@ def test_tiny_cell_self_images(oracle_mod):
     assert np.array_equal(csr["dist"], np.sqrt(np.sum(csr["vec"] ** 2, axis=1)))
 
 
+def _sc_integer_lattice(cells):
+    # simple cubic, a = 1 A, integer coordinates and box: every edge vector and
+    # r^2 is an exact small integer, so equal distances are exact ties
+    x = C.lattice_sites("sc", 1.0, cells)
+    return x, np.diag([float(cells)] * 3)
+
+
+def test_cutoff_is_strict_on_an_exact_shell(oracle_mod):
+    # the neighbour set is r < rcut: with rcut = 2 A exactly the sites at
+    # distance 2 are out (simple cubic shells 6, 12, 8 at r^2 = 1, 2, 3; the 6
+    # at r^2 = 4 follow only once rcut passes 2)
+    x, box = _sc_integer_lattice(5)
+    kept, raw = oracle_mod.counts(x, box, [1, 1, 1], 2.0, 256)
+    assert np.all(raw == 6 + 12 + 8)
+    kept, raw = oracle_mod.counts(x, box, [1, 1, 1], np.nextafter(2.0, 3.0), 256)
+    assert np.all(raw == 6 + 12 + 8 + 6)
+    kept, raw = oracle_mod.counts(x, box, [1, 1, 1], 1.0, 256)
+    assert np.all(raw == 0)
+
+
+def test_cap_breaks_exact_ties_by_source_then_shift(oracle_mod):
+    # cap 10 on simple cubic with rcut 1.5: the 6 sites at r = 1 are kept and
+    # 4 of the 12 exact ties at r = sqrt(2) follow, the smallest by (source,
+    # shift); the expected sets come from a direct enumeration in integers
+    cells, cap = 5, 10
+    x, box = _sc_integer_lattice(cells)
+    csr = oracle_mod.build_csr(x, box, [1, 1, 1], 1.5, 1.0, cap)
+    xi = np.rint(x).astype(np.int64)
+    for i in (0, 7, 62, 124):
+        cand = []
+        for j in range(xi.shape[0]):
+            for S in np.ndindex(3, 3, 3):
+                S = np.array(S) - 1
+                if j == i and not S.any():
+                    continue
+                v = xi[j] + S * cells - xi[i]
+                r2 = int(v @ v)
+                if r2 <= 2:                      # r < 1.5
+                    cand.append((r2, j, *S.tolist()))
+        assert len(cand) == 18
+        want = sorted(sorted(cand)[:cap], key=lambda t: t[1:])   # kept, in canonical order
+        rows = _rows(csr)[i]
+        got = [(int(j), *map(int, S)) for j, S in zip(csr["src"][rows], csr["shift"][rows])]
+        assert got == [t[1:] for t in want]
+
+
 def test_two_atoms_hand_computed(oracle_mod):
     # cubic L = 10, atoms at x = 1 and x = 9: they are 2 A apart through the
     # boundary; 8 A apart directly (outside rcut 3)

@@ -1,0 +1,181 @@
+"""Mutation tests of the oracle's pins.
+
+Each case plants one plausible mistake in a copy of the oracle's C source (a
+dropped term, a wrong sign, a swapped index, a transposed operand, an
+off-by-one, a wrong order), compiles that copy into a scratch library and
+runs the pin tests of the part it touches against it.  The pins must fail.
+A control compiles the unmodified source the same way, and its pins must
+pass.  So a pin suite that cannot tell the definition from a near miss of it
+shows up here.
+
+Mistakes are planted in the oracle only, on the CPU.
+"""
+import concurrent.futures as cf
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+
+SWITCH = ["test_oracle_switch.py"]
+BUILD = ["test_oracle_build.py"]
+ATTN = ["test_oracle_attention.py"]
+SMOOTH = ["test_oracle_smooth.py"]
+LOCAL = ["test_oracle_local.py"]
+
+# (name, pin files, text of the definition, the planted mistake)
+MUTANTS = [
+    # the switch and its cosine (cosine switch from r_on to rcut)
+    ("taylor_sign", SWITCH,
+     "c[k] = -c[k - 1] / div;", "c[k] = c[k - 1] / div;"),
+    ("taylor_factorial", SWITCH,
+     "double div = (double)((2 * k) * (2 * k + 1));", "double div = (double)((2 * k) * (2 * k - 1));"),
+    ("taylor_truncated", SWITCH,
+     "#define ORC_NTAYLOR 12", "#define ORC_NTAYLOR 6"),
+    ("cos_phase", SWITCH,
+     "double t = u - 0.5;", "double t = u + 0.5;"),
+    ("switch_half_dropped", SWITCH,
+     "return 0.5 * one_plus;", "return one_plus;"),
+    ("switch_scaled_by_rcut", SWITCH,
+     "double u = num / den;", "double u = num / rcut;"),
+    ("switch_onset", SWITCH,
+     "if (r < r_on) return 1.0;", "if (r < r_on) return 0.5;"),
+    # the neighbour set, its cap and its order
+    ("vector_sign", BUILD,
+     "v[c] = xs - xi[c];", "v[c] = xi[c] - xs;"),
+    ("cutoff_inclusive", BUILD,
+     "if (r2 < g->rc2) {", "if (r2 <= g->rc2) {"),
+    ("self_images_dropped", BUILD,
+     "if (j == i && S[0] == 0 && S[1] == 0 && S[2] == 0) continue;", "if (j == i) continue;"),
+    ("image_range_minimum_image", BUILD,
+     "g->reach[k] = rcut / h;", "g->reach[k] = 0.5 * rcut / h;"),
+    ("negative_images_dropped", BUILD,
+     "lo[k] = (int)ceil(-df - g->reach[k] - 1e-6);", "lo[k] = (int)ceil(-df - 1e-6);"),
+    ("shift_wrong_box_row", BUILD,
+     "double p1 = s1 * g->a[1][c];", "double p1 = s1 * g->a[0][c];"),
+    ("r2_term_dropped", BUILD,
+     "r2 = r2 + t2;", "r2 = r2 + 0.0 * t2;"),
+    ("cap_keeps_farthest", BUILD,
+     "if (a->r2 < b->r2) return -1;\n    if (a->r2 > b->r2) return 1;",
+     "if (a->r2 > b->r2) return -1;\n    if (a->r2 < b->r2) return 1;"),
+    ("cap_tie_break_reversed", BUILD,
+     "if (a->j != b->j) return a->j < b->j ? -1 : 1;\n    for (int k = 0; k < 3; ++k)\n"
+     "        if (a->S[k] != b->S[k]) return a->S[k] < b->S[k] ? -1 : 1;\n    return 0;\n}\n\n"
+     "/* canonical",
+     "if (a->j != b->j) return a->j > b->j ? -1 : 1;\n    for (int k = 0; k < 3; ++k)\n"
+     "        if (a->S[k] != b->S[k]) return a->S[k] > b->S[k] ? -1 : 1;\n    return 0;\n}\n\n"
+     "/* canonical"),
+    ("cap_off_by_one", BUILD,
+     "buf->len = nnei_max;", "buf->len = nnei_max - 1;"),
+    ("canonical_shift_order_reversed", BUILD,
+     "if (a->S[k] != b->S[k]) return a->S[k] < b->S[k] ? -1 : 1;\n    return 0;\n}\n\n"
+     "/* Fractional",
+     "if (a->S[k] != b->S[k]) return a->S[k] > b->S[k] ? -1 : 1;\n    return 0;\n}\n\n"
+     "/* Fractional"),
+    ("canonical_sort_skipped", BUILD,
+     "qsort(buf->buf, (size_t)buf->len, sizeof(orc_cand), cmp_canon);", ";"),
+    ("dist_is_r2", BUILD,
+     "double r = sqrt(r2);", "double r = r2;"),
+    # block-dense attention
+    ("projection_transposed", ATTN + SMOOTH,
+     "acc = acc + x[a * c + k] * W[(int64_t)k * c + m];",
+     "acc = acc + x[a * c + k] * W[(int64_t)m * c + k];"),
+    ("logit_scale_d", ATTN,
+     "double l = ((s[a] * s[b]) * dot) / rsd;\n            P[a * n + b] = l;",
+     "double l = ((s[a] * s[b]) * dot) / (double)d;\n            P[a * n + b] = l;"),
+    ("logit_query_switch_dropped", ATTN,
+     "double l = ((s[a] * s[b]) * dot) / rsd;\n            P[a * n + b] = l;",
+     "double l = (s[b] * dot) / rsd;\n            P[a * n + b] = l;"),
+    ("logit_key_is_query_row", ATTN,
+     "for (int t = 0; t < d; ++t) dot = dot + Q[a * c + h * d + t] * K[b * c + h * d + t];",
+     "for (int t = 0; t < d; ++t) dot = dot + Q[a * c + h * d + t] * K[a * c + h * d + t];"),
+    ("logit_head_slice", ATTN,
+     "for (int t = 0; t < d; ++t) dot = dot + Q[a * c + h * d + t] * K[b * c + h * d + t];",
+     "for (int t = 0; t < d; ++t) dot = dot + Q[a * c + t] * K[b * c + t];"),
+    ("softmax_max_not_subtracted", ATTN,
+     "double e = exp(P[a * n + b] - m);", "double e = exp(P[a * n + b]);"),
+    ("softmax_not_normalised", ATTN,
+     "for (int64_t b = 0; b < n; ++b) P[a * n + b] = P[a * n + b] / z;",
+     "for (int64_t b = 0; b < n; ++b) P[a * n + b] = P[a * n + b] / 1.0;"),
+    ("av_map_transposed", ATTN,
+     "acc = acc + P[a * n + b] * V[b * c + h * d + t];",
+     "acc = acc + P[b * n + a] * V[b * c + h * d + t];"),
+    ("av_value_head_slice", ATTN,
+     "acc = acc + P[a * n + b] * V[b * c + h * d + t];",
+     "acc = acc + P[a * n + b] * V[b * c + t];"),
+    # slot-occupancy attention
+    ("smooth_phantom_sign", SMOOTH,
+     "if (phi > 0) z = z + (double)phi * exp(-m);", "if (phi > 0) z = z + (double)phi * exp(m);"),
+    ("smooth_phantoms_dropped", SMOOTH,
+     "if (phi > 0) z = z + (double)phi * exp(-m);", "if (phi > 0) z = z + 0.0 * exp(-m);"),
+    ("smooth_phantom_count", SMOOTH,
+     "int64_t phi = nnei_max - n;", "int64_t phi = nnei_max - n - 1;"),
+    ("smooth_one_switch", SMOOTH,
+     "double l = ((s[a] * s[b]) * dot) / rsd;\n                        E[b] = l;",
+     "double l = (s[b] * dot) / rsd;\n                        E[b] = l;"),
+    # local attention
+    ("local_query_from_edge", LOCAL,
+     "project(1, c, H + i * c, Wq, q);", "project(1, c, G + base * c, Wq, q);"),
+    ("local_switch_dropped", LOCAL,
+     "double l = (sw[base + b] * dot) / rsd;", "double l = dot / rsd;"),
+    ("local_not_normalised", LOCAL,
+     "acc = acc + (P[b] / z) * V[b * c + h * d + t];", "acc = acc + P[b] * V[b * c + h * d + t];"),
+    ("local_empty_row_not_zeroed", LOCAL,
+     "for (int m = 0; m < c; ++m) out[i * c + m] = 0.0;\n            if (n <= 0) continue;",
+     "if (n <= 0) continue;\n            for (int m = 0; m < c; ++m) out[i * c + m] = 0.0;"),
+]
+
+ALL_PINS = sorted({f for _, files, _, _ in MUTANTS for f in files})
+
+
+def _compile(src_text, path):
+    c_path = path + ".c"
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    subprocess.run(["gcc", *oracle.CFLAGS, "-o", path, c_path, "-lm"], check=True,
+                   capture_output=True, timeout=120)
+
+
+def _run_pins(lib, files):
+    env = dict(os.environ, MLG_ORACLE_LIB=lib, OMP_NUM_THREADS="2",
+               PYTHONDONTWRITEBYTECODE="1")
+    cmd = [sys.executable, "-m", "pytest", *[os.path.join(HERE, f) for f in files], "-x", "-q",
+           "-m", "not gpu", "-p", "no:cacheprovider"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    return r.returncode, (r.stdout + r.stderr)[-1500:]
+
+
+@pytest.fixture(scope="module")
+def outcomes(tmp_path_factory):
+    src = open(oracle._SRC).read()
+    tmp = str(tmp_path_factory.mktemp("mutants"))
+    jobs = {"control": (src, ALL_PINS)}
+    for name, files, old, new in MUTANTS:
+        assert src.count(old) == 1, f"{name}: the definition's text is not unique in the source"
+        jobs[name] = (src.replace(old, new), files)
+
+    def one(item):
+        name, (text, files) = item
+        lib = os.path.join(tmp, f"lib_{name}.so")
+        _compile(text, lib)
+        return name, _run_pins(lib, files)
+
+    with cf.ThreadPoolExecutor(max_workers=max(2, min(8, (os.cpu_count() or 2) // 2))) as ex:
+        return dict(ex.map(one, jobs.items()))
+
+
+def test_control_passes(outcomes):
+    rc, tail = outcomes["control"]
+    assert rc == 0, tail
+
+
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+def test_mutant_is_caught(outcomes, name):
+    rc, tail = outcomes[name]
+    # 1: a pin failed; a crash of the mutant (negative: a signal) counts too
+    assert rc == 1 or rc < 0, f"mutant {name} survived the pins (rc {rc}):\n{tail}"

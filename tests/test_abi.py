@@ -195,3 +195,32 @@ def test_batch_workspace_and_checks(mlg):
     assert call(n=-1, ws=FAKE * 16, nb=both) == mlg.MLG_ERR_INVALID_ARG
     assert call(r_on=5.0, ws=FAKE * 16, nb=both) == mlg.MLG_ERR_INVALID_ARG
     assert call(nnei=999, ws=FAKE * 16, nb=both) == mlg.MLG_ERR_UNSUPPORTED
+
+
+def test_local_and_smooth_argument_checks(mlg):
+    """Host checks of the local and slot-occupancy attention calls.  Every
+    call below returns before a kernel is launched (a host check fails, or
+    there is no centre), so fake device pointers are never dereferenced."""
+    lib = mlg.lib()
+    c = _fake_csr(mlg)
+    smooth = lambda **k: lib.mlg_block_attention_smooth(
+        ctypes.byref(c), k.get("n", 10), k.get("nnei", 40), k.get("ch", 32), k.get("heads", 4),
+        k.get("dtype", 1), k.get("gin", FAKE), k.get("gout", FAKE * 2), k.get("wq", FAKE),
+        FAKE, FAKE, None)
+    assert smooth(heads=3) == mlg.MLG_ERR_INVALID_ARG
+    assert smooth(gout=FAKE) == mlg.MLG_ERR_INVALID_ARG      # aliasing in/out
+    assert smooth(wq=None) == mlg.MLG_ERR_INVALID_ARG
+    assert smooth(nnei=300) == mlg.MLG_ERR_UNSUPPORTED
+    assert smooth(dtype=5) == mlg.MLG_ERR_INVALID_ARG
+    assert smooth(n=0) == mlg.MLG_OK                          # nothing to do, nothing launched
+    local = lambda **k: lib.mlg_local_attention(
+        ctypes.byref(c), k.get("n", 10), k.get("nnei", 40), k.get("ch", 32), k.get("heads", 4),
+        k.get("dtype", 1), k.get("h", FAKE * 3), k.get("gin", FAKE), k.get("out", FAKE * 2),
+        FAKE, FAKE, k.get("wv", FAKE), None)
+    assert local(h=None) == mlg.MLG_ERR_INVALID_ARG
+    assert local(h=FAKE * 2) == mlg.MLG_ERR_INVALID_ARG      # query rows alias the output
+    assert local(wv=None) == mlg.MLG_ERR_INVALID_ARG
+    assert local(ch=64, heads=5) == mlg.MLG_ERR_INVALID_ARG
+    assert local(ch=512, heads=8) == mlg.MLG_ERR_UNSUPPORTED
+    assert local(n=-2) == mlg.MLG_ERR_INVALID_ARG
+    assert local(n=0) == mlg.MLG_OK

@@ -224,3 +224,55 @@ def test_local_and_smooth_argument_checks(mlg):
     assert local(ch=512, heads=8) == mlg.MLG_ERR_UNSUPPORTED
     assert local(n=-2) == mlg.MLG_ERR_INVALID_ARG
     assert local(n=0) == mlg.MLG_OK
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) for every function the header declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    protos = {}
+    for m in re.finditer(r"^\s*((?:const\s+)?[a-z_0-9]+\s*\*?)\s*(mlg_[a-z_0-9]+)\s*\(([^)]*)\)\s*;",
+                         text, re.M):
+        ret, name, params = m.group(1), m.group(2), m.group(3).strip()
+        plist = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+        protos[name] = (ret.strip(), plist)
+    return protos
+
+
+def _c_kind(decl):
+    """The ctypes class of a C declaration (a parameter or a return type);
+    int and the int-sized enum are 32-bit here, like int32_t."""
+    decl = re.sub(r"\bconst\b", "", decl)
+    if "*" in decl or "[" in decl or re.search(r"\bmlg_stream_t\b", decl):
+        return "ptr"
+    for ctype, kind in (("int64_t", "i64"), ("int32_t", "i32"), ("size_t", "size"),
+                        ("double", "f64"), ("mlg_dtype", "i32"), ("int", "i32"), ("void", None)):
+        if re.search(r"\b%s\b" % ctype, decl):
+            return kind
+    raise AssertionError("unclassified C type: " + decl)
+
+
+def _ct_kind(t):
+    if t is None:
+        return None
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or issubclass(t, ctypes._Pointer):
+        return "ptr"
+    kinds = {ctypes.c_int64: "i64", ctypes.c_size_t: "size", ctypes.c_double: "f64",
+             ctypes.c_int32: "i32", ctypes.c_int: "i32"}
+    return kinds.get(t, repr(t))
+
+
+def test_binding_signatures_match_header(mlg):
+    # each ctypes declaration of the binding has the header's parameter count
+    # and widths, so a call through Python marshals what the C side reads
+    protos = _prototypes()
+    assert set(protos) == set(_declared_functions())
+    lib = mlg.lib()
+    for name, (ret, params) in sorted(protos.items()):
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, name + ": no argtypes in the binding"
+        want = [_c_kind(p) for p in params]
+        got = [_ct_kind(t) for t in fn.argtypes]
+        assert got == want, (name, got, want)
+        want_ret = "ptr" if "*" in ret else _c_kind(ret)
+        assert _ct_kind(fn.restype) == want_ret, (name, fn.restype, ret)

@@ -43,7 +43,11 @@ CFLAGS = ["-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
 
 
 def build(force: bool = False) -> str:
-    """Compile ``mlg_oracle.c`` into ``liboracle.so`` (gcc)."""
+    """Compile ``mlg_oracle.c`` into ``liboracle.so`` (gcc); with a stand-in
+    library named in ``MLG_ORACLE_LIB`` (the mutation tests), return that."""
+    alt = os.environ.get("MLG_ORACLE_LIB")
+    if alt:
+        return alt
     stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
     if force or stale:
         tmp = _LIB + f".tmp{os.getpid()}"
@@ -58,8 +62,7 @@ def _load():
         if _lib is None:
             # a deliberately broken copy of this library, compiled by the
             # mutation tests, replaces it when named here (tests only)
-            alt = os.environ.get("MLG_ORACLE_LIB")
-            lib = ctypes.CDLL(alt if alt else build())
+            lib = ctypes.CDLL(build())
             i64, i32, dbl = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
             p = ctypes.c_void_p
             lib.oracle_cos_pi.restype = dbl

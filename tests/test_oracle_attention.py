@@ -192,3 +192,23 @@ def test_forward_layers_chain(oracle_mod):
     for layer in range(6):
         g = oracle_mod.attention(csr["row_ptr"], csr["sw"], g, *W[layer], w.heads)
         assert np.array_equal(outs[layer], g)
+
+
+def test_forward_fp32_sees_only_fp32_values(oracle_mod):
+    # the fp32 path stores every layer in fp32 and reads s(r) as fp32: each
+    # layer's output is an fp32 array, and switch values that round to the
+    # same fp32 number give the same result
+    w = C.workload(2)
+    s = C.system(2, 1)
+    csr = oracle_mod.build_csr(s["coords"], s["box"], s["pbc"], w.rcut, w.r_on, w.nnei_max)
+    W = C.weights(2, 1)[:2].astype(np.float32)
+    G = C.features(2, 1, csr["row_ptr"][-1]).astype(np.float32)
+    sw = csr["sw"]
+    assert np.any(sw.astype(np.float32).astype(np.float64) != sw)
+    outs = oracle_mod.forward(csr["row_ptr"], sw, G, W, w.heads, "f32")
+    assert [o.dtype for o in outs] == [np.float32, np.float32]
+    outs32 = oracle_mod.forward(csr["row_ptr"], sw.astype(np.float32), G, W, w.heads, "f32")
+    assert all(np.array_equal(a, b) for a, b in zip(outs, outs32))
+    # the second layer reads the first layer's fp32 output
+    again = oracle_mod.forward(csr["row_ptr"], sw, outs[0], W[1:], w.heads, "f32")
+    assert np.array_equal(again[0], outs[1])

@@ -124,6 +124,17 @@ def test_cap_breaks_exact_ties_by_source_then_shift(oracle_mod):
         assert got == [t[1:] for t in want]
 
 
+def test_cap_equal_to_the_count_truncates_nothing(oracle_mod):
+    # a row is truncated when its count exceeds nnei_max: simple cubic with
+    # rcut 1.5 has exactly 18 neighbours per site
+    x, box = _sc_integer_lattice(4)
+    full = oracle_mod.build_csr(x, box, [1, 1, 1], 1.5, 1.0, 18)
+    assert full["n_truncated"] == 0 and np.all(np.diff(full["row_ptr"]) == 18)
+    cut = oracle_mod.build_csr(x, box, [1, 1, 1], 1.5, 1.0, 17)
+    assert cut["n_truncated"] == 64 and np.all(np.diff(cut["row_ptr"]) == 17)
+    assert np.all(cut["raw"] == 18)
+
+
 def test_two_atoms_hand_computed(oracle_mod):
     # cubic L = 10, atoms at x = 1 and x = 9: they are 2 A apart through the
     # boundary; 8 A apart directly (outside rcut 3)

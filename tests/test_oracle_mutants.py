@@ -12,6 +12,7 @@ Mistakes are planted in the oracle only, on the CPU.
 """
 import concurrent.futures as cf
 import os
+import re
 import subprocess
 import sys
 
@@ -130,7 +131,20 @@ MUTANTS = [
      "if (n <= 0) continue;\n            for (int m = 0; m < c; ++m) out[i * c + m] = 0.0;"),
 ]
 
-ALL_PINS = sorted({f for _, files, _, _ in MUTANTS for f in files})
+# the same for the oracle's Python side (oracle/__init__.py): the layer chain,
+# its fp32 rounding and the CSR's scalar outputs
+PY_MUTANTS = [
+    ("forward_layers_not_chained", ATTN,
+     "        g = o\n", "        g = np.asarray(G0)\n"),
+    ("forward_fp32_output_not_rounded", ATTN,
+     "            o = o.astype(np.float32)\n", "            o = o.astype(np.float64)\n"),
+    ("forward_fp32_switch_not_rounded", ATTN,
+     "        sw = sw.astype(np.float32).astype(np.float64)\n", "        sw = sw\n"),
+    ("n_truncated_inclusive", BUILD,
+     "np.count_nonzero(raw > nnei_max)", "np.count_nonzero(raw >= nnei_max)"),
+]
+
+ALL_PINS = sorted({f for _, files, _, _ in MUTANTS + PY_MUTANTS for f in files})
 
 
 def _compile(src_text, path):
@@ -141,11 +155,28 @@ def _compile(src_text, path):
                    capture_output=True, timeout=120)
 
 
-def _run_pins(lib, files):
+# runs pytest with a given file standing in for oracle/__init__.py (loaded as
+# the package "oracle" before the tests import it)
+_WITH_PACKAGE = (
+    "import importlib.util, sys\n"
+    "init, args = sys.argv[1], sys.argv[2:]\n"
+    "spec = importlib.util.spec_from_file_location('oracle', init)\n"
+    "mod = importlib.util.module_from_spec(spec)\n"
+    "sys.modules['oracle'] = mod\n"
+    "spec.loader.exec_module(mod)\n"
+    "import pytest\n"
+    "sys.exit(pytest.main(args))\n")
+
+
+def _run_pins(lib, files, init=None):
     env = dict(os.environ, MLG_ORACLE_LIB=lib, OMP_NUM_THREADS="2",
                PYTHONDONTWRITEBYTECODE="1")
-    cmd = [sys.executable, "-m", "pytest", *[os.path.join(HERE, f) for f in files], "-x", "-q",
-           "-m", "not gpu", "-p", "no:cacheprovider"]
+    args = [*[os.path.join(HERE, f) for f in files], "-x", "-q", "-m", "not gpu", "-p",
+            "no:cacheprovider"]
+    if init is None:
+        cmd = [sys.executable, "-m", "pytest", *args]
+    else:
+        cmd = [sys.executable, "-c", _WITH_PACKAGE, init, *args]
     r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
     return r.returncode, (r.stdout + r.stderr)[-1500:]
 
@@ -159,8 +190,24 @@ def outcomes(tmp_path_factory):
         assert src.count(old) == 1, f"{name}: the definition's text is not unique in the source"
         jobs[name] = (src.replace(old, new), files)
 
+    lib0 = oracle.build()
+    py_src = open(os.path.join(os.path.dirname(oracle._SRC), "__init__.py")).read()
+    for name, files, old, new in PY_MUTANTS:
+        assert py_src.count(old) == 1, f"{name}: the definition's text is not unique in the source"
+        jobs[name] = (py_src.replace(old, new), files)
+    # the unmodified Python side through the same stand-in path
+    jobs["py_control"] = (py_src, ALL_PINS)
+    py_names = {m[0] for m in PY_MUTANTS} | {"py_control"}
+
     def one(item):
         name, (text, files) = item
+        if name in py_names:
+            pkg = os.path.join(tmp, f"py_{name}")
+            os.makedirs(pkg, exist_ok=True)
+            init = os.path.join(pkg, "__init__.py")
+            with open(init, "w") as f:
+                f.write(text)
+            return name, _run_pins(lib0, files, init)
         lib = os.path.join(tmp, f"lib_{name}.so")
         _compile(text, lib)
         return name, _run_pins(lib, files)
@@ -169,13 +216,16 @@ def outcomes(tmp_path_factory):
         return dict(ex.map(one, jobs.items()))
 
 
-def test_control_passes(outcomes):
-    rc, tail = outcomes["control"]
+@pytest.mark.parametrize("name", ["control", "py_control"])
+def test_control_passes(outcomes, name):
+    rc, tail = outcomes[name]
     assert rc == 0, tail
 
 
-@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS + PY_MUTANTS])
 def test_mutant_is_caught(outcomes, name):
     rc, tail = outcomes[name]
-    # 1: a pin failed; a crash of the mutant (negative: a signal) counts too
-    assert rc == 1 or rc < 0, f"mutant {name} survived the pins (rc {rc}):\n{tail}"
+    # caught: pytest ran and a pin failed, or the mutant crashed (a signal);
+    # an error before the pins ran (exit 1 without a failed test) is not
+    caught = (rc == 1 and re.search(r"\b\d+ failed\b", tail)) or rc < 0
+    assert caught, f"mutant {name} survived the pins (rc {rc}):\n{tail}"

@@ -19,10 +19,11 @@
  *      (Proposed fix).
  *
  *   2. mlg_block_attention: block-dense multi-head attention of every centre
- *      over its own edges (NeighborGraph issue, Proposed fix: gather the
- *      compact per-centre block through destination_row_ptr, run the dense
- *      attention math with per-row masks for ragged tails, write back to the
- *      edge axis; no (sum nnei^2, c) pair-axis tensor ever exists).
+ *      over its own edges (NeighborGraph issue, Proposed fix: each centre's
+ *      edges form one small dense block, found by destination_row_ptr; the
+ *      block is attended to with dense products, unequal row lengths masked
+ *      per row, and the outputs go back to their edges; no (sum nnei^2, c)
+ *      pair-axis tensor ever exists).
  *
  *   mlg_forward runs stage 1 and then n_layers of stage 2.
  *
@@ -186,7 +187,7 @@ int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                         size_t ws_bytes, mlg_stream_t stream);
 
 /* One attention layer with the slot-occupancy ("smooth") softmax (NeighborGraph
- * issue, Numerics note: a phantom count and a slot-occupancy denominator; the
+ * issue, Numerics note: empty slots counted as phantoms in the denominator; the
  * weights factor as w_b = softmax_b * sum_b e_b / D~).  As mlg_block_attention,
  * plus phi = nnei_max - n phantom slots per destination: the zero-padded
  * slots of the dense (nloc, nnei_max, c) route, left unmasked, whose logit is

@@ -2,11 +2,11 @@
 // the destination CSR (sm_100a).
 //
 // deepmd-kit issue "NeighborGraph attention is 4-9x slower than dense and
-// OOM-prone", Proposed fix: gather each centre's compact block of edge
-// features through destination_row_ptr, run the dense attention math (the
-// per-centre (nnei, nnei) products of the dense route, Root cause) with
-// per-row masks for ragged tails, and write the result back on the edge
-// axis.  Here the gather is the contiguous CSR slab of the centre, the
+// OOM-prone", Proposed fix: each centre's edge features are collected into
+// one small block by way of destination_row_ptr, attended to with the same
+// batched products the dense route uses per centre (Root cause), the unequal
+// row lengths handled by masking each row, and the outputs returned to their
+// edges.  Here the gather is the contiguous CSR slab of the centre, the
 // "mask" is the loop bound n_i, and the scatter is a contiguous slab store:
 // no (sum nnei^2, c) tensor and no Q/K/V tensor ever reaches global memory.
 //
@@ -15,7 +15,7 @@
 //   l_ab = s_a s_b (q_a . k_b) / sqrt(d)
 //   O_a = sum_b exp(l_ab - m_a) v_b / sum_b exp(l_ab - m_a),  m_a = max_b l_ab
 // With `smooth` (slot-occupancy softmax, NeighborGraph issue, Numerics note:
-// a phantom count and a slot-occupancy denominator), the centre's
+// the denominator counts empty slots as phantoms), the centre's
 // phi = nnei_max - n padded slots take part as phantoms of logit 0 and value
 // 0: m_a = max(max_b l_ab, 0) and the denominator gains phi exp(-m_a).
 #pragma once

@@ -208,8 +208,8 @@ def attention(row_ptr, sw, G, Wq, Wk, Wv, heads: int, nthreads: int = 0) -> np.n
 def attention_smooth(row_ptr, sw, G, Wq, Wk, Wv, heads: int, nnei_max: int,
                      nthreads: int = 0) -> np.ndarray:
     """Slot-occupancy ("smooth") attention (NeighborGraph issue, Numerics note:
-    signed phantom count and slot-occupancy denominator; the weights factor as
-    w_b = softmax_b * sum_b e_b / D~).
+    phantom slots counted in an occupancy-dependent denominator; the weights
+    factor as w_b = softmax_b * sum_b e_b / D~).
 
     As ``attention``, plus phi = nnei_max - n phantom slots per centre with
     logit exactly 0 and value 0 -- the dense route's zero-padded slots, left

@@ -29,8 +29,9 @@
  *    V = G Wv; per head l_ab = s_a s_b (q_a . k_b) / sqrt(d); softmax over
  *    the centre's real edges b; O_a = sum_b P_ab V_b.
  *  - Slot-occupancy ("smooth") attention (NeighborGraph issue, Numerics note and
- *    "Graph-native alternatives": a signed phantom count and a slot-occupancy
- *    denominator; the weights factor as w_b = softmax_b * (sum_b e_b / D~)).
+ *    "Graph-native alternatives": phantom slots counted in a denominator that
+ *    depends on slot occupancy; the weights factor as
+ *    w_b = softmax_b * (sum_b e_b / D~)).
  *    Reading: the dense route pads every centre to nnei_max slots with zero
  *    features and zero switch, so a padded slot's logit is exactly 0 and,
  *    unmasked, it enters the softmax denominator; it adds nothing to the

@@ -1,7 +1,8 @@
 """Pins of the oracle's slot-occupancy ("smooth") attention.
 
-The NeighborGraph issue states the semantics only as "a signed phantom count
-and a slot-occupancy denominator", with weights that factor as
+The NeighborGraph issue (Numerics note) names only the ingredients: a count
+of phantom slots, which can be signed, and a denominator that depends on how
+many slots are occupied; the weights factor as
 w_b = softmax_b * (sum_b e_b / D~).  The reading: the dense route pads every
 centre to nnei_max slots with zero features and zero switch, so a padded
 slot's logit is exactly 0, and left unmasked it enters the softmax

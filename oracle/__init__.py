@@ -18,7 +18,11 @@ states the definitions in full:
   (nsel 120 / rcut 6, nsel 40 / rcut 4);
 * attention -- NeighborGraph issue, Proposed fix (dense per-centre attention
   with per-row masks) and Root cause (the dense route's per-centre
-  (nloc, nnei, nnei) batched products).
+  (nloc, nnei, nnei) batched products);
+* Verlet-list reuse -- DPA4 issue, Proposed optimizations (device tensors
+  reused while the neighbour list is unchanged): an uncapped list at
+  rcut + skin, re-evaluated at the current coordinates, then capped and
+  ordered as the full build.
 
 Parity of the switch cosine, the neighbour set and the attention is pinned by
 the ``-m "not gpu"`` tests in ``tests/test_oracle_*.py``.
@@ -84,6 +88,11 @@ def _load():
             lib.oracle_attention_smooth.restype = ctypes.c_int
             lib.oracle_attention_smooth.argtypes = [i64, p, p, i32, i32, i32, p, p, p, p, p,
                                                     ctypes.c_int]
+            lib.oracle_refine_count.restype = ctypes.c_int
+            lib.oracle_refine_count.argtypes = [i64, p, p, p, dbl, i32, p, p, p, p, p]
+            lib.oracle_refine_fill.restype = ctypes.c_int
+            lib.oracle_refine_fill.argtypes = [i64, p, p, p, dbl, dbl, i32, p, p, p, p, p, p,
+                                               p, p, p]
             lib.oracle_local_attention.restype = ctypes.c_int
             lib.oracle_local_attention.argtypes = [i64, p, p, i32, i32, p, p, p, p, p, p,
                                                    ctypes.c_int]
@@ -156,6 +165,67 @@ def build_csr(coords, box, pbc, rcut: float, r_on: float, nnei_max: int,
                              _ptr(dist), _ptr(sw), int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_fill failed ({rc})")
+    return {"row_ptr": row_ptr, "src": src, "shift": shift, "vec": vec, "dist": dist,
+            "sw": sw, "raw": raw, "n_truncated": int(np.count_nonzero(raw > nnei_max))}
+
+
+def verlet_candidates(coords, box, pbc, rcut: float, skin: float, nthreads: int = 0) -> dict:
+    """The candidate list of Verlet reuse: every pair within rcut + skin, with
+    no cap (the cap is applied when the list is used).  The CSR dict of
+    ``build_csr`` at the larger cutoff."""
+    r = float(rcut) + float(skin)
+    return build_csr(coords, box, pbc, r, min(float(rcut), r), 1 << 30, nthreads)
+
+
+def max_displacement(coords, coords_ref) -> float:
+    """The largest distance any atom has moved, on the raw (unwrapped)
+    coordinates: an atom re-wrapped into the box counts as having moved by a
+    box length."""
+    d = np.asarray(coords, dtype=np.float64) - np.asarray(coords_ref, dtype=np.float64)
+    return float(np.sqrt(np.max(np.sum(d * d, axis=1)))) if d.size else 0.0
+
+
+def needs_rebuild(coords, coords_ref, skin: float) -> bool:
+    """Verlet criterion: the list built at ``coords_ref`` stays complete while
+    every atom has moved less than skin / 2."""
+    return 2.0 * max_displacement(coords, coords_ref) >= float(skin)
+
+
+def verlet_refine(cand: dict, coords, box, pbc, rcut: float, r_on: float,
+                  nnei_max: int) -> dict:
+    """The CSR from a candidate list: every candidate (source, shift)
+    re-evaluated at the current coordinates, kept if r < rcut, the cap and
+    the canonical order applied as in ``build_csr``.  Equal to ``build_csr``
+    at the current coordinates while the Verlet criterion holds."""
+    coords, box, pbc = _geom_args(coords, box, pbc)
+    n = coords.shape[0]
+    cp = np.ascontiguousarray(cand["row_ptr"], dtype=np.int64)
+    cs = np.ascontiguousarray(cand["src"], dtype=np.int32)
+    ch = np.ascontiguousarray(cand["shift"], dtype=np.int32).reshape(-1, 3)
+    if cp.size != n + 1:
+        raise ValueError("candidate list and coordinates disagree on the atom count")
+    kept = np.zeros(n, dtype=np.int32)
+    raw = np.zeros(n, dtype=np.int64)
+    lib = _load()
+    rc = lib.oracle_refine_count(n, _ptr(coords), _ptr(box), _ptr(pbc), float(rcut),
+                                 int(nnei_max), _ptr(cp), _ptr(cs), _ptr(ch), _ptr(kept),
+                                 _ptr(raw))
+    if rc != 0:
+        raise ValueError(f"oracle_refine_count failed ({rc})")
+    row_ptr = np.zeros(n + 1, dtype=np.int64)
+    np.cumsum(kept, out=row_ptr[1:])
+    e = int(row_ptr[-1])
+    src = np.zeros(e, dtype=np.int32)
+    shift = np.zeros((e, 3), dtype=np.int32)
+    vec = np.zeros((e, 3), dtype=np.float64)
+    dist = np.zeros(e, dtype=np.float64)
+    sw = np.zeros(e, dtype=np.float64)
+    rc = lib.oracle_refine_fill(n, _ptr(coords), _ptr(box), _ptr(pbc), float(rcut),
+                                float(r_on), int(nnei_max), _ptr(cp), _ptr(cs), _ptr(ch),
+                                _ptr(row_ptr), _ptr(src), _ptr(shift), _ptr(vec), _ptr(dist),
+                                _ptr(sw))
+    if rc != 0:
+        raise ValueError(f"oracle_refine_fill failed ({rc})")
     return {"row_ptr": row_ptr, "src": src, "shift": shift, "vec": vec, "dist": dist,
             "sw": sw, "raw": raw, "n_truncated": int(np.count_nonzero(raw > nnei_max))}
 

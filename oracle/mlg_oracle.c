@@ -38,6 +38,15 @@
  *    numerator (its value row is 0).  With phi = nnei_max - n phantoms:
  *    m = max(max_b l_ab, 0 if phi > 0), D~ = sum_b e^(l_ab - m) + phi e^(-m),
  *    O_a = sum_b e^(l_ab - m) V_b / D~.
+ *  - Verlet-list reuse (DPA4 issue, Proposed optimizations: device tensors
+ *    cached across the MD steps in which the neighbour list is unchanged; the
+ *    MD engine decides when it changes, by the usual skin criterion, which the
+ *    pages leave to the engine): from a candidate list built at rcut + skin
+ *    without a cap, each step recomputes every candidate's vector from the
+ *    current coordinates, keeps r < rcut, and then applies the cap and the
+ *    canonical order, as the full build does.
+ *    While no atom has moved skin/2 or more since the list was built, every
+ *    pair within rcut is a candidate, so the result equals the full build.
  *  - Local attention, one query per centre (NeighborGraph issue, "Graph-native
  *    alternatives", item 2: LocalAtten maps onto the per-centre CSR segment
  *    with queries = centres and keys = edges): q_i = H_i Wq from the centre's
@@ -284,17 +293,24 @@ static int centre_all(const orc_geom* g, int64_t n, const double* x, const doubl
     return ORC_OK;
 }
 
+/* The cap and the order of a centre's in-cutoff edges: when there are more
+ * than nnei_max, the nnei_max smallest by (r^2, source, shift) are kept; the
+ * row is then put in canonical order. */
+static void keep_nearest_canonical(orc_vec* buf, int32_t nnei_max) {
+    if (buf->len > nnei_max) {
+        qsort(buf->buf, (size_t)buf->len, sizeof(orc_cand), cmp_dist);
+        buf->len = nnei_max;
+    }
+    qsort(buf->buf, (size_t)buf->len, sizeof(orc_cand), cmp_canon);
+}
+
 /* The kept edges of centre i in canonical order; returns raw count in *raw. */
 static int centre_edges(const orc_geom* g, int64_t n, const double* x, const double* frac,
                         int64_t i, int32_t nnei_max, orc_vec* buf, int64_t* raw) {
     int rc = centre_all(g, n, x, frac, i, buf);
     if (rc != ORC_OK) return rc;
     *raw = buf->len;
-    if (buf->len > nnei_max) {
-        qsort(buf->buf, (size_t)buf->len, sizeof(orc_cand), cmp_dist);
-        buf->len = nnei_max;
-    }
-    qsort(buf->buf, (size_t)buf->len, sizeof(orc_cand), cmp_canon);
+    keep_nearest_canonical(buf, nnei_max);
     return ORC_OK;
 }
 
@@ -415,6 +431,82 @@ int64_t oracle_centre(int64_t n, const double* coords, const double* box, const 
     int64_t kept = buf.len;
     free(buf.buf);
     return kept;
+}
+
+/* ------------------------------------------------------------------ */
+/* Verlet-list reuse                                                   */
+/* ------------------------------------------------------------------ */
+
+/* The kept edges of centre i chosen from a stored candidate row (source,
+ * shift) instead of from every source and image: each candidate's vector is
+ * recomputed from the current coordinates by edge_vec, kept if r^2 < rcut^2,
+ * the nearest nnei_max kept by (r^2, source, shift), and the row put in
+ * canonical order.  Returns the raw count in *raw. */
+static int centre_refine(const orc_geom* g, const double* x, int64_t i, const int64_t* cand_ptr,
+                         const int32_t* cand_src, const int32_t* cand_shift, int32_t nnei_max,
+                         orc_vec* buf, int64_t* raw) {
+    buf->len = 0;
+    for (int64_t p = cand_ptr[i]; p < cand_ptr[i + 1]; ++p) {
+        orc_cand c;
+        c.j = cand_src[p];
+        c.S[0] = cand_shift[3 * p];
+        c.S[1] = cand_shift[3 * p + 1];
+        c.S[2] = cand_shift[3 * p + 2];
+        double v[3];
+        c.r2 = edge_vec(g, x + 3 * i, x + 3 * (int64_t)c.j, c.S, v);
+        if (c.r2 < g->rc2)
+            if (vec_push(buf, c) != ORC_OK) return ORC_ERR_MEM;
+    }
+    *raw = buf->len;
+    keep_nearest_canonical(buf, nnei_max);
+    return ORC_OK;
+}
+
+/* Per-centre kept and raw counts from a candidate list (cand_ptr [n+1],
+ * cand_src [C], cand_shift [C][3]: the list built at a larger cutoff). */
+int oracle_refine_count(int64_t n, const double* coords, const double* box, const uint8_t* pbc,
+                        double rcut, int32_t nnei_max, const int64_t* cand_ptr,
+                        const int32_t* cand_src, const int32_t* cand_shift, int32_t* n_kept,
+                        int64_t* n_raw) {
+    orc_geom g;
+    if (n < 0 || nnei_max <= 0) return ORC_ERR_ARG;
+    int rc = geom_init(&g, box, pbc, rcut);
+    if (rc != ORC_OK) return rc;
+    orc_vec buf = {0, 0, 0};
+    for (int64_t i = 0; i < n && rc == ORC_OK; ++i) {
+        int64_t raw = 0;
+        rc = centre_refine(&g, coords, i, cand_ptr, cand_src, cand_shift, nnei_max, &buf, &raw);
+        n_kept[i] = (int32_t)buf.len;
+        n_raw[i] = raw;
+    }
+    free(buf.buf);
+    return rc;
+}
+
+/* The CSR arrays from a candidate list; row_ptr must be the exclusive prefix
+ * sum of the kept counts. */
+int oracle_refine_fill(int64_t n, const double* coords, const double* box, const uint8_t* pbc,
+                       double rcut, double r_on, int32_t nnei_max, const int64_t* cand_ptr,
+                       const int32_t* cand_src, const int32_t* cand_shift,
+                       const int64_t* row_ptr, int32_t* src, int32_t* shift, double* vec,
+                       double* dist, double* sw) {
+    orc_geom g;
+    if (n < 0 || nnei_max <= 0) return ORC_ERR_ARG;
+    int rc = geom_init(&g, box, pbc, rcut);
+    if (rc != ORC_OK) return rc;
+    orc_vec buf = {0, 0, 0};
+    for (int64_t i = 0; i < n && rc == ORC_OK; ++i) {
+        int64_t raw = 0;
+        rc = centre_refine(&g, coords, i, cand_ptr, cand_src, cand_shift, nnei_max, &buf, &raw);
+        if (rc == ORC_OK && row_ptr[i + 1] - row_ptr[i] != buf.len) rc = ORC_ERR_ROWPTR;
+        for (int64_t a = 0; rc == ORC_OK && a < buf.len; ++a) {
+            int64_t p = row_ptr[i] + a;
+            write_edge(&g, coords, i, &buf.buf[a], r_on, src + p, shift + 3 * p, vec + 3 * p,
+                       dist + p, sw + p);
+        }
+    }
+    free(buf.buf);
+    return rc;
 }
 
 /* ------------------------------------------------------------------ */

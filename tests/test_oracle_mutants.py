@@ -28,6 +28,7 @@ BUILD = ["test_oracle_build.py"]
 ATTN = ["test_oracle_attention.py"]
 SMOOTH = ["test_oracle_smooth.py"]
 LOCAL = ["test_oracle_local.py"]
+VERLET = ["test_oracle_verlet.py"]
 
 # (name, pin files, text of the definition, the planted mistake)
 MUTANTS = [
@@ -71,17 +72,28 @@ MUTANTS = [
      "if (a->j != b->j) return a->j > b->j ? -1 : 1;\n    for (int k = 0; k < 3; ++k)\n"
      "        if (a->S[k] != b->S[k]) return a->S[k] > b->S[k] ? -1 : 1;\n    return 0;\n}\n\n"
      "/* canonical"),
-    ("cap_off_by_one", BUILD,
+    ("cap_off_by_one", BUILD + VERLET,
      "buf->len = nnei_max;", "buf->len = nnei_max - 1;"),
     ("canonical_shift_order_reversed", BUILD,
      "if (a->S[k] != b->S[k]) return a->S[k] < b->S[k] ? -1 : 1;\n    return 0;\n}\n\n"
      "/* Fractional",
      "if (a->S[k] != b->S[k]) return a->S[k] > b->S[k] ? -1 : 1;\n    return 0;\n}\n\n"
      "/* Fractional"),
-    ("canonical_sort_skipped", BUILD,
+    ("canonical_sort_skipped", BUILD + VERLET,
      "qsort(buf->buf, (size_t)buf->len, sizeof(orc_cand), cmp_canon);", ";"),
     ("dist_is_r2", BUILD,
      "double r = sqrt(r2);", "double r = r2;"),
+    # Verlet-list reuse
+    ("refine_cutoff_inclusive", VERLET,
+     "if (c.r2 < g->rc2)", "if (c.r2 <= g->rc2)"),
+    ("refine_shift_dropped", VERLET,
+     "c.S[2] = cand_shift[3 * p + 2];", "c.S[2] = 0;"),
+    ("refine_source_as_centre", VERLET,
+     "c.r2 = edge_vec(g, x + 3 * i, x + 3 * (int64_t)c.j, c.S, v);",
+     "c.r2 = edge_vec(g, x + 3 * (int64_t)c.j, x + 3 * i, c.S, v);"),
+    ("refine_reads_next_row", VERLET,
+     "for (int64_t p = cand_ptr[i]; p < cand_ptr[i + 1]; ++p) {",
+     "for (int64_t p = cand_ptr[i]; p < cand_ptr[i + 1] - 1; ++p) {"),
     # block-dense attention
     ("projection_transposed", ATTN + SMOOTH,
      "acc = acc + x[a * c + k] * W[(int64_t)k * c + m];",
@@ -141,7 +153,16 @@ PY_MUTANTS = [
     ("forward_fp32_switch_not_rounded", ATTN,
      "        sw = sw.astype(np.float32).astype(np.float64)\n", "        sw = sw\n"),
     ("n_truncated_inclusive", BUILD,
-     "np.count_nonzero(raw > nnei_max)", "np.count_nonzero(raw >= nnei_max)"),
+     "np.count_nonzero(raw > nnei_max))}\n\n\ndef verlet_candidates(",
+     "np.count_nonzero(raw >= nnei_max))}\n\n\ndef verlet_candidates("),
+    ("refine_n_truncated_inclusive", VERLET,
+     "np.count_nonzero(raw > nnei_max))}\n\n\ndef centre(",
+     "np.count_nonzero(raw >= nnei_max))}\n\n\ndef centre("),
+    ("verlet_criterion_strict", VERLET,
+     "return 2.0 * max_displacement(coords, coords_ref) >= float(skin)",
+     "return 2.0 * max_displacement(coords, coords_ref) > float(skin)"),
+    ("verlet_list_without_skin", VERLET,
+     "    r = float(rcut) + float(skin)\n", "    r = float(rcut)\n"),
 ]
 
 ALL_PINS = sorted({f for _, files, _, _ in MUTANTS + PY_MUTANTS for f in files})

@@ -180,7 +180,9 @@ size_t mlg_attention_workspace_bytes(int64_t n_centres, int32_t nnei_max, int32_
  *   l_ab = s_a s_b (q_a . k_b) / sqrt(d);  P_ab = exp(l_ab - max_b l) / sum_b exp(...);
  *   G_out[a, h d + t] = sum_b P_ab v_b[t].
  * Slots beyond a destination's n edges do not exist (masked).  Reads E from csr->row_ptr
- * on the device; if *csr->status has MLG_STATUS_CAPACITY set, nothing is written. */
+ * on the device; if *csr->status has MLG_STATUS_CAPACITY set, nothing is written.
+ * nnei_max must be at least the longest row (the cap the CSR was built with): the rows
+ * of a destination with more edges are not guaranteed to be written. */
 int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                         int32_t channels, int32_t heads, mlg_dtype dtype, const void* G_in,
                         void* G_out, const void* Wq, const void* Wk, const void* Wv, void* ws,

@@ -5,9 +5,13 @@ the library's CUDA kernels. Torch tensors provide device memory and streams.
 There is no fallback: if ``libmlg.so`` is missing, importing this module
 raises.
 
-Names match the C ABI: :func:`mlg_build_csr`, :func:`mlg_block_attention`,
-:func:`mlg_forward`, the ``*_workspace_bytes`` queries and
-:func:`mlg_status_string`. :class:`Csr` bundles the caller-owned CSR buffers.
+Names match the C ABI: :func:`mlg_build_csr`, :func:`mlg_build_csr_batch`,
+:func:`mlg_block_attention`, :func:`mlg_attention_stack`, :func:`mlg_forward`,
+:func:`mlg_local_attention`, :func:`mlg_block_attention_smooth`, the
+``*_workspace_bytes`` queries and :func:`mlg_status_string`. :class:`Csr`
+bundles the caller-owned CSR buffers. Descriptors (:func:`make_system`,
+``Csr.struct()``) hold raw device addresses: the tensors behind them must
+outlive every call that uses them.
 """
 from __future__ import annotations
 

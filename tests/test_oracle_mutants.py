@@ -24,7 +24,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 
 SWITCH = ["test_oracle_switch.py"]
-BUILD = ["test_oracle_build.py"]
+BUILD = ["test_oracle_build.py", "test_oracle_build_random.py"]
 ATTN = ["test_oracle_attention.py"]
 SMOOTH = ["test_oracle_smooth.py"]
 LOCAL = ["test_oracle_local.py"]

@@ -25,9 +25,9 @@ ROOT = os.path.dirname(HERE)
 
 SWITCH = ["test_oracle_switch.py"]
 BUILD = ["test_oracle_build.py", "test_oracle_build_random.py"]
-ATTN = ["test_oracle_attention.py"]
-SMOOTH = ["test_oracle_smooth.py"]
-LOCAL = ["test_oracle_local.py"]
+ATTN = ["test_oracle_attention.py", "test_oracle_attention_random.py"]
+SMOOTH = ["test_oracle_smooth.py", "test_oracle_attention_random.py"]
+LOCAL = ["test_oracle_local.py", "test_oracle_attention_random.py"]
 VERLET = ["test_oracle_verlet.py"]
 
 # (name, pin files, text of the definition, the planted mistake)

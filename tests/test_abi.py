@@ -276,3 +276,28 @@ def test_binding_signatures_match_header(mlg):
         assert got == want, (name, got, want)
         want_ret = "ptr" if "*" in ret else _c_kind(ret)
         assert _ct_kind(fn.restype) == want_ret, (name, fn.restype, ret)
+
+
+def test_forward_launch_counts(mlg):
+    """The kernel launches of one mlg_forward, as the benchmark counts them
+    (a host-side plan, no GPU):
+      diamond-64:    one-launch build + c = 128 head-group attention (1 layer)    = 2
+      diamond-512:   one-launch build + one fused launch for all 6 layers        = 2
+      Fe BCC 65,536: init, bin, cell scan, scatter, count, row scan (3), fill,
+                     + fused tile and the generic kernel for rows over 128       = 11
+      protein 5,964: init, bounding box, bin, cell scan (3), scatter, count,
+                     row scan, fill, + head-group kernel per layer (2)           = 12
+      Fe BCC 524,288: init, bin, cell scan (3), scatter, count, row scan (3),
+                     fill, + one fused tile launch                               = 12"""
+    from neighbour_graph_attention_b200 import configs as C
+
+    want = {1: 2, 2: 2, 3: 11, 4: 12, 5: 12}
+    for key, n in want.items():
+        w = C.workload(key)
+        L = w.a * w.cells if w.periodic else 0.0
+        box = np.diag([L] * 3) if w.periodic else np.zeros((3, 3))
+        pbc = [1, 1, 1] if w.periodic else [0, 0, 0]
+        dt = mlg.MLG_F64 if w.dtype == "f64" else mlg.MLG_F32
+        got = mlg.mlg_forward_launch_count(w.n_atoms, w.rcut, box, pbc, w.nnei_max, w.channels,
+                                           w.heads, w.n_layers, dt)
+        assert got == n, (w.name, got, n)

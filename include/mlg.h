@@ -82,8 +82,11 @@ typedef enum {
                                         broken exactly by (source, shift)) */
     MLG_STATUS_INTERNAL = 32u,       /* the count and fill passes disagreed on a row (never
                                         expected); that row is incomplete */
-    MLG_STATUS_TIMEOUT = 64u         /* a bounded wait for an on-chip copy ran out (never
-                                        expected); the attention output is incomplete */
+    MLG_STATUS_TIMEOUT = 64u,        /* a bounded wait ran out (never expected in normal
+                                        use); the output of that call is incomplete */
+    MLG_STATUS_ROW_TOO_LONG = 128u   /* an attention call met a destination with more edges
+                                        than the nnei_max it was given; that destination's
+                                        output rows were not written */
 } mlg_status_bits;
 
 /* Arithmetic type of attention features and weights. */
@@ -181,8 +184,9 @@ size_t mlg_attention_workspace_bytes(int64_t n_centres, int32_t nnei_max, int32_
  *   G_out[a, h d + t] = sum_b P_ab v_b[t].
  * Slots beyond a destination's n edges do not exist (masked).  Reads E from csr->row_ptr
  * on the device; if *csr->status has MLG_STATUS_CAPACITY set, nothing is written.
- * nnei_max must be at least the longest row (the cap the CSR was built with): the rows
- * of a destination with more edges are not guaranteed to be written. */
+ * nnei_max is normally the cap the CSR was built with.  A destination with more than
+ * nnei_max edges is skipped on every kernel path: its output rows are left as they were
+ * and MLG_STATUS_ROW_TOO_LONG is OR-ed into *csr->status. */
 int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                         int32_t channels, int32_t heads, mlg_dtype dtype, const void* G_in,
                         void* G_out, const void* Wq, const void* Wk, const void* Wv, void* ws,
@@ -196,7 +200,8 @@ int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
  * exactly 0 and whose value is 0:
  *   m_a = max(max_b l_ab, 0 if phi > 0),  D~ = sum_b exp(l_ab - m_a) + phi exp(-m_a),
  *   G_out[a, h d + t] = sum_b exp(l_ab - m_a) v_b[t] / D~.
- * Destinations with more than nnei_max edges are left untouched.  Runs on
+ * Destinations with more than nnei_max edges are left untouched and flagged with
+ * MLG_STATUS_ROW_TOO_LONG.  Runs on
  * the generic kernel (no fused tiles yet); no workspace. */
 int mlg_block_attention_smooth(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                                int32_t channels, int32_t heads, mlg_dtype dtype,
@@ -257,8 +262,10 @@ int mlg_forward(const mlg_system* sys, double rcut, double r_on, int32_t nnei_ma
  *     scratch than the array holds (mlg_build_csr_workspace_bytes() >
  *     MLG_NOALLOC_SCRATCH_BYTES; about 150,000 atoms for a periodic box).
  *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture begins.
+ *     that device current) and caches it with the current context; make that
+ *     first call before any stream capture begins.  A later call under a new
+ *     context of that device (after cudaDeviceReset, for instance) looks the
+ *     address up again.
  *   - Every call shares the one array, and the array keeps the contents of
  *     the previous call; the build clears everything that must start at zero
  *     itself.  Two calls whose work overlaps on the GPU (different streams
@@ -268,7 +275,11 @@ int mlg_build_csr_noalloc(const mlg_system* sys, double rcut, double r_on, int32
 
 /* Number of kernel launches that one mlg_forward call with these arguments
  * issues on its stream (for accounting in benchmarks); 0 for invalid
- * arguments. */
+ * arguments.  Systems small enough for the one-launch build count it as one
+ * kernel; its 8-byte flag reset (a cudaMemsetAsync, not a kernel of this
+ * library) is not counted, and the count assumes the driver accepts that
+ * cooperative launch (if it refuses, the kernel chain of larger systems runs
+ * instead). */
 int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
                              const uint8_t pbc[3], int32_t nnei_max, int32_t channels,
                              int32_t heads, int32_t n_layers, mlg_dtype dtype);
@@ -283,8 +294,8 @@ int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
  * distance of its own).
  *   csr      CSR from mlg_build_csr (row_ptr, sw, capacity, status used);
  *            rows must hold at most nnei_max edges (true for a CSR built
- *            with the same nnei_max); longer rows give a zero row and set
- *            MLG_STATUS_INTERNAL.
+ *            with the same nnei_max); a longer row gives a zero output row and
+ *            sets MLG_STATUS_ROW_TOO_LONG.
  *   H_in     device [n_centres][channels] centre features, dtype.
  *   G_in     device [E][channels] edge features in CSR order, dtype.
  *   out      device [n_centres][channels], dtype; must not alias H_in or G_in.
@@ -306,6 +317,21 @@ int mlg_local_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
  * Returns MLG_ERR_INVALID_ARG for null pointers with n > 0 or n < 0,
  * MLG_ERR_CUDA if the launch fails. */
 int mlg_exp2_neg(const double* y, double* out, int64_t n, mlg_stream_t stream);
+
+/* Diagnostics: the one-launch build of a small system (mlg_build_csr's
+ * arguments) with its bounded waits shortened to `polls` polls each (about
+ * 0.3 us apart) and CTA 0 withholding the flag that releases the other CTAs
+ * after binning.  The other CTAs' waits therefore run out: they OR
+ * MLG_STATUS_TIMEOUT into *csr->status and leave; CTA 0 then gives up at the
+ * grid barrier the same way.  No copy is in flight at either wait, so the
+ * launch ends cleanly and the context stays usable; the CSR outputs are
+ * incomplete.  For tests of the timeout path of those waits.  Returns
+ * MLG_ERR_UNSUPPORTED when the system does not take the one-launch build (or
+ * the driver refuses the cooperative launch), MLG_ERR_INVALID_ARG for
+ * polls < 1, otherwise as mlg_build_csr. */
+int mlg_build_csr_wait_test(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+                            const mlg_csr* csr, void* ws, size_t ws_bytes, int32_t polls,
+                            mlg_stream_t stream);
 
 /* A static string naming a host status code. */
 const char* mlg_status_string(int status);

@@ -397,8 +397,15 @@ int launch_fused_build(const BuildArgs& a, const BuildPlan& plan, int nsplit, Fu
   return MLG_ERR_UNSUPPORTED;
 }
 
+// Test knobs of the one-launch build's bounded waits (nullptr: normal build).
+struct FusedWaitTest {
+  long long polls;   // polls of each wait before it gives up
+  int hold_release;  // CTA 0 never releases the binned atoms
+};
+
 int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
-               const mlg_csr* csr, void* ws, size_t ws_bytes, cudaStream_t stream) {
+               const mlg_csr* csr, void* ws, size_t ws_bytes, cudaStream_t stream,
+               const FusedWaitTest* wait_test = nullptr) {
   if (sys == nullptr || sys->coords == nullptr) return MLG_ERR_INVALID_ARG;
   if (sys->types != nullptr && sys->n_types < 1) return MLG_ERR_INVALID_ARG;
   int rc = check_build_args(rcut, r_on, nnei_max, csr);
@@ -411,8 +418,13 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   if (ws == nullptr || ws_bytes < L.total || ((uintptr_t)ws % kAlign) != 0)
     return MLG_ERR_WORKSPACE;
   char* w = static_cast<char*>(ws);
-  const BuildArgs a = make_build_args(sys, rcut, r_on, nnei_max, csr, w, L);
+  BuildArgs a = make_build_args(sys, rcut, r_on, nnei_max, csr, w, L);
   const int nsplit = build_nsplit(plan);
+  if (wait_test != nullptr) {
+    if (!use_fused_build(plan, n)) return MLG_ERR_UNSUPPORTED;
+    a.spin_polls = wait_test->polls;
+    a.hold_release = wait_test->hold_release;
+  }
   if (use_fused_build(plan, n)) {
     // the whole build in one cooperative launch (small systems); systems of
     // at most 75 atoms take the larger stage, which holds any 27-cell stencil
@@ -421,7 +433,8 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
     const int rc2 = 27 * n <= kCellCandSmall
                         ? launch_fused_build<kCellCandSmall>(a, plan, nsplit, sync, stream)
                         : launch_fused_build<kCellCand>(a, plan, nsplit, sync, stream);
-    if (rc2 != MLG_ERR_UNSUPPORTED) return rc2;  // refused (not co-resident): the chain below
+    if (rc2 != MLG_ERR_UNSUPPORTED || wait_test != nullptr) return rc2;
+    // refused (not co-resident): the kernel chain below
   }
   launch_count_phase(a, plan, nsplit, stream);
   launch_scan<long long>(a.kept, n, reinterpret_cast<long long*>(a.row_ptr), a.partial,
@@ -728,6 +741,7 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
     ta.n_centres = n_centres;
     ta.capacity = csr->capacity;
     ta.n_layers = n_layers;
+    ta.nnei_max = nnei_max;
     ta.G = G_in;
     ta.out = G_out;
     for (int k = 0; k < 3 * n_layers; ++k) ta.W[k] = W[k];
@@ -752,6 +766,7 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
       ha.sw = csr->sw;
       ha.n_centres = n_centres;
       ha.capacity = csr->capacity;
+      ha.nnei_max = nnei_max;
       ha.G = in;
       ha.out = dst;
       ha.Wq = W[3 * l];
@@ -976,6 +991,14 @@ int mlg_exp2_neg(const double* y, double* out, int64_t n, mlg_stream_t stream) {
   return launch_status();
 }
 
+int mlg_build_csr_wait_test(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
+                             const mlg_csr* csr, void* ws, size_t ws_bytes, int32_t polls,
+                             mlg_stream_t stream) {
+  if (polls < 1) return MLG_ERR_INVALID_ARG;
+  const FusedWaitTest t{(long long)polls, 1};
+  return build_impl(sys, rcut, r_on, nnei_max, csr, ws, ws_bytes, (cudaStream_t)stream, &t);
+}
+
 int mlg_version(void) { return 100; }
 
 }  // extern "C"
@@ -1002,10 +1025,30 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kNoAllocMaxDevices];  // device address of the array, per device
+CUcontext g_noalloc_ctx[kNoAllocMaxDevices];  // the context that address belongs to
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The calling thread's current context (nullptr if it cannot be read).
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr)
+      return nullptr;
+    fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  CUcontext ctx = nullptr;
+  return fn(&ctx) == CUDA_SUCCESS ? ctx : nullptr;
+}
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// with that device current and cached together with the context it belongs
+// to; a new context of the device (after a device reset the module is loaded
+// again, at a possibly different address) triggers a fresh lookup.
 int noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -1014,7 +1057,8 @@ int noalloc_scratch(void** out) {
   }
   if (dev < 0 || dev >= kNoAllocMaxDevices) return MLG_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  CUcontext ctx = current_context();
+  if (g_noalloc_ptr[dev] == nullptr || ctx == nullptr || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr) {
@@ -1022,6 +1066,7 @@ int noalloc_scratch(void** out) {
       return MLG_ERR_CUDA;
     }
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = current_context();  // made current by the lookup if it was not yet
   }
   *out = g_noalloc_ptr[dev];
   return MLG_OK;

@@ -73,7 +73,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn_generic(AttnArgs a) {
   for (int64_t i = blockIdx.x; i < a.n_centres; i += gridDim.x) {
     const int64_t base = a.row_ptr[i];
     const int n = (int)(a.row_ptr[i + 1] - base);
-    if (n <= a.min_n || n > NM || base + n > a.capacity) continue;
+    if (n > NM) {  // longer than the caller's nnei_max: not written, flagged
+      if (threadIdx.x == 0) atomicOr(a.status, (uint32_t)MLG_STATUS_ROW_TOO_LONG);
+      continue;
+    }
+    if (n <= a.min_n || base + n > a.capacity) continue;
     for (int t = threadIdx.x; t < n; t += blockDim.x) sS[t] = (T)a.sw[base + t];
     __syncthreads();
     for (int h = 0; h < a.H; ++h) {

@@ -425,14 +425,15 @@ __global__ void __launch_bounds__(NT, 1) k_attn_dmma(TileArgs a) {
       const int c_end = meta.c_end;
       while (c < c_end) {
         const int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
-        if (n > 0 && n <= NBC * 8) break;
+        if (n > 0 && n <= NBC * 8 && n <= a.nnei_max) break;
+        if (n > a.nnei_max) atomicOr(a.status, (uint32_t)MLG_STATUS_ROW_TOO_LONG);
         ++c;
       }
       meta.c0[0] = c;
       while (c < c_end && k < 64) {
         const int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
         const int n8 = (n + 7) & ~7;
-        if (n > NBC * 8 || rows + n8 > R) break;
+        if (n > NBC * 8 || n > a.nnei_max || rows + n8 > R) break;
         meta.off[0][k] = rows;
         meta.task0[0][k] = tasks;
         tasks += H * full_qblocks(n) + (H / 2) * half_qblocks(n);

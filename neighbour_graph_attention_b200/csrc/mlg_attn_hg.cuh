@@ -28,6 +28,7 @@ struct HgArgs {
   const double* sw;
   int64_t n_centres;
   int64_t capacity;
+  int nnei_max;  // centres with more edges are skipped and flagged
   const void* G;
   void* out;
   const void* Wq;
@@ -120,13 +121,14 @@ __global__ void __launch_bounds__(NT) k_attn_hg(HgArgs a) {
       const int c_end = meta.c_end;
       while (c < c_end) {
         int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
-        if (n > 0 && n <= R) break;
+        if (n > 0 && n <= R && n <= a.nnei_max) break;
+        if (n > a.nnei_max && g == 0) atomicOr(a.status, (uint32_t)MLG_STATUS_ROW_TOO_LONG);
         ++c;
       }
       meta.row0[0] = c < c_end ? a.row_ptr[c] : 0;
       while (c < c_end && k < Cfg::MAXC) {
         int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
-        if (n > R || rows + n > R) break;
+        if (n > R || n > a.nnei_max || rows + n > R) break;
         meta.off[0][k] = rows;
         meta.task0[0][k] = tasks;
         tasks += (n * HG + 31) / 32;

@@ -32,6 +32,7 @@ struct TileArgs {
   int64_t n_centres;
   int64_t capacity;
   int n_layers;  // 1 .. kMaxFusedLayers
+  int nnei_max;  // centres with more edges are skipped and flagged (MLG_STATUS_ROW_TOO_LONG)
   const void* G;
   void* out;
   const void* W[3 * kMaxFusedLayers];  // q, k, v of each layer: device [C][C]

@@ -97,6 +97,9 @@ struct BuildArgs {
   uint32_t* status;
   int32_t src_offset;        // added to written source indices (systems of a batch)
   int zero_globals;          // k_init clears n_truncated and status (not in a batch)
+  long long spin_polls;      // one-launch build: polls of each bounded wait (0: the default)
+  int hold_release;          // one-launch build: CTA 0 never releases the binned atoms, so
+                             // the other CTAs' waits run out (tests of the timeout path)
   // workspace
   CellGrid* grid;
   unsigned long long* bbox;  // [6] ordered bits: min x, y, z, max x, y, z
@@ -1372,9 +1375,10 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-// polls until *p >= want; false if the limit ran out first
-__device__ __forceinline__ bool wait_at_least(const unsigned* p, unsigned want) {
-  for (long long it = 0; it < kFusedSpinLimit; ++it) {
+// polls until *p >= want; false if `polls` polls (0: kFusedSpinLimit) ran out first
+__device__ __forceinline__ bool wait_at_least(const unsigned* p, unsigned want, long long polls) {
+  const long long limit = polls > 0 ? polls : kFusedSpinLimit;
+  for (long long it = 0; it < limit; ++it) {
     if (ld_acquire_gpu(p) >= want) return true;
     __nanosleep(256);
   }
@@ -1458,13 +1462,13 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2)
       if (cell >= 0) scatter_atom_at(a, sg, i, s_hist[cell] + s_rank[i], s_w[i]);
     }
     __syncthreads();
-    if (tid == 0) {
+    if (tid == 0 && !a.hold_release) {
       __threadfence();
       st_release_gpu(&sync->ready, 1u);
     }
   }
   if (tid == 0) {
-    s_ok = blockIdx.x == 0 ? 1 : (wait_at_least(&sync->ready, 1u) ? 1 : 0);
+    s_ok = blockIdx.x == 0 ? 1 : (wait_at_least(&sync->ready, 1u, a.spin_polls) ? 1 : 0);
     if (s_ok && blockIdx.x != 0) sg = *a.grid;
     reinterpret_cast<CellStageT<CAP>*>(s_dyn)->staged_cell = -1;
   }
@@ -1485,7 +1489,7 @@ __global__ void __launch_bounds__(kCellWarps * 32, 2)
   if (tid == 0) {
     __threadfence();
     atomicAdd(&sync->arrived, 1u);
-    s_ok = wait_at_least(&sync->arrived, gridDim.x) ? 1 : 0;
+    s_ok = wait_at_least(&sync->arrived, gridDim.x, a.spin_polls) ? 1 : 0;
   }
   __syncthreads();
   if (!s_ok) {

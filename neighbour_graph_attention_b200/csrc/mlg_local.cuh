@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kLocalThreads) k_local_attn(LocalArgs a) {
     T* orow = out + i * c;
     if (n <= 0 || n > NM) {  // no edges: a zero row; longer than nnei_max: flagged
       for (int m = tid; m < c; m += blockDim.x) orow[m] = T(0);
-      if (n > NM && tid == 0) atomicOr(a.status, (uint32_t)MLG_STATUS_INTERNAL);
+      if (n > NM && tid == 0) atomicOr(a.status, (uint32_t)MLG_STATUS_ROW_TOO_LONG);
       continue;
     }
     for (int m = tid; m < c; m += blockDim.x) sx[m] = Hn[i * c + m];

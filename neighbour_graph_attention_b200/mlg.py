@@ -46,6 +46,7 @@ MLG_STATUS_IMAGE_RANGE = 8
 MLG_STATUS_TIES = 16
 MLG_STATUS_INTERNAL = 32
 MLG_STATUS_TIMEOUT = 64
+MLG_STATUS_ROW_TOO_LONG = 128
 
 MLG_F32 = 0
 MLG_F64 = 1
@@ -106,6 +107,9 @@ _lib.mlg_local_attention.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c
                                      ctypes.c_int, _p, _p, _p, _p, _p, _p, _p]
 _lib.mlg_exp2_neg.restype = ctypes.c_int
 _lib.mlg_exp2_neg.argtypes = [_p, _p, _c_i64, _p]
+_lib.mlg_build_csr_wait_test.restype = ctypes.c_int
+_lib.mlg_build_csr_wait_test.argtypes = [ctypes.POINTER(mlg_system), _c_dbl, _c_dbl, _c_i32,
+                                         ctypes.POINTER(mlg_csr), _p, _c_sz, _c_i32, _p]
 _lib.mlg_status_string.restype = ctypes.c_char_p
 _lib.mlg_status_string.argtypes = [ctypes.c_int]
 _lib.mlg_version.restype = ctypes.c_int
@@ -274,6 +278,18 @@ def mlg_build_csr(system: mlg_system, rcut: float, r_on: float, nnei_max: int, c
     code = _lib.mlg_build_csr(ctypes.byref(system), float(rcut), float(r_on), int(nnei_max),
                               ctypes.byref(c), _ptr(ws), nbytes, _stream_handle(stream))
     return _check(code, "mlg_build_csr", check)
+
+
+def mlg_build_csr_wait_test(system: mlg_system, rcut: float, r_on: float, nnei_max: int,
+                            csr: Csr, ws, polls: int, stream=None, check: bool = True) -> int:
+    """Diagnostics: the one-launch build with its bounded waits made to run
+    out after ``polls`` polls (the device status then has MLG_STATUS_TIMEOUT)."""
+    c = csr.struct()
+    nbytes = int(ws.numel() * ws.element_size())
+    code = _lib.mlg_build_csr_wait_test(ctypes.byref(system), float(rcut), float(r_on),
+                                        int(nnei_max), ctypes.byref(c), _ptr(ws), nbytes,
+                                        int(polls), _stream_handle(stream))
+    return _check(code, "mlg_build_csr_wait_test", check)
 
 
 MLG_NOALLOC_SCRATCH_BYTES = 8 << 20

@@ -84,9 +84,13 @@ typedef enum {
                                         expected); that row is incomplete */
     MLG_STATUS_TIMEOUT = 64u,        /* a bounded wait ran out (never expected in normal
                                         use); the output of that call is incomplete */
-    MLG_STATUS_ROW_TOO_LONG = 128u   /* an attention call met a destination with more edges
+    MLG_STATUS_ROW_TOO_LONG = 128u,  /* an attention call met a destination with more edges
                                         than the nnei_max it was given; that destination's
                                         output rows were not written */
+    MLG_STATUS_LIST_INCOMPLETE = 256u /* mlg_verlet_step: the candidate list misses pairs
+                                        (a destination had more than 256 candidates within
+                                        rcut + skin, or the list's capacity was too small);
+                                        the refined CSR may miss edges */
 } mlg_status_bits;
 
 /* Arithmetic type of attention features and weights. */
@@ -243,6 +247,57 @@ int mlg_forward(const mlg_system* sys, double rcut, double r_on, int32_t nnei_ma
                 int32_t channels, int32_t heads, int32_t n_layers, mlg_dtype dtype,
                 const void* const* W, const void* G0, void* G_out, const mlg_csr* csr,
                 void* ws, size_t ws_bytes, mlg_stream_t stream);
+
+/* Verlet-skin reuse of the neighbour search across MD steps (DPA4 LAMMPS
+ * issue, Proposed optimizations: keep the device tensors of the edge
+ * construction while the neighbour list is unchanged, rebuild when the MD
+ * engine's skin criterion asks for it).
+ *
+ * The list: every (source, shift) within rcut + skin of each destination at
+ * the coordinates it was built at, as a CSR in canonical order, with no cap
+ * other than 256 candidates per destination.  All members are caller-owned
+ * DEVICE memory. */
+typedef struct {
+    mlg_csr cand;          /* candidate CSR (row_ptr [N+1], src, shift; the vec, dist and sw
+                              arrays are written by its build too); capacity >= N * 256
+                              always suffices */
+    double* coords_ref;    /* [N][3]: the coordinates the candidates were found at */
+    uint32_t* state;       /* bit 0: the list is valid.  Zero it before the first call (and
+                              whenever the atoms are renumbered or the box changes) */
+    int64_t* n_builds;     /* counter of list builds (diagnostics; the library adds 1 per
+                              build) */
+} mlg_verlet_list;
+
+/* Bytes of device workspace that mlg_verlet_step needs; 0 for invalid arguments. */
+size_t mlg_verlet_workspace_bytes(int64_t n_atoms, double rcut, double skin, const double box[9],
+                                  const uint8_t pbc[3]);
+
+/* One MD step's destination CSR through the Verlet list, all on `stream`
+ * without a host synchronisation:
+ *   1. a device reduction finds the largest displacement of any atom since
+ *      the list was built (raw coordinates: an atom re-wrapped into the box
+ *      has moved by a box length); when 2 * that >= skin, a coordinate is not
+ *      finite, or bit 0 of *list->state is clear, a device word asks for a
+ *      rebuild;
+ *   2. the build kernels, gated on that word, rebuild the list (the regular
+ *      build at rcut + skin with cap 256; types are validated there) and store
+ *      the coordinates; when no rebuild is asked for they return at once;
+ *   3. the refine re-evaluates every candidate at the current coordinates
+ *      with the build's own operation order, keeps r < rcut, caps each
+ *      destination to the nnei_max nearest by (r^2, source, shift) and writes
+ *      `out` in canonical order.
+ * `out` is then bit for bit what mlg_build_csr(sys, rcut, r_on, nnei_max)
+ * gives at the current coordinates (pairs within rcut now were within
+ * rcut + skin at the list's coordinates while no atom has moved skin / 2).
+ * Resets *out->status and *out->n_truncated; the input bits of the list's
+ * last build (non-finite coordinate, type range, image range) are OR-ed into
+ * *out->status, and MLG_STATUS_LIST_INCOMPLETE when the list overflowed.
+ *   skin      >= 0 (0 rebuilds every step)
+ *   ws        >= mlg_verlet_workspace_bytes(), 256-byte aligned
+ * The box and pbc must stay those the list was built with. */
+int mlg_verlet_step(const mlg_system* sys, double rcut, double r_on, double skin,
+                    int32_t nnei_max, const mlg_verlet_list* list, const mlg_csr* out, void* ws,
+                    size_t ws_bytes, mlg_stream_t stream);
 
 /* Size of the library's built-in scratch array for mlg_build_csr_noalloc. */
 #define MLG_NOALLOC_SCRATCH_BYTES (8u << 20)

@@ -17,6 +17,7 @@
 #include "mlg_attn_dmma.cuh"
 #include "mlg_attn_tc.cuh"
 #include "mlg_local.cuh"
+#include "mlg_verlet.cuh"
 
 using namespace mlg;
 
@@ -244,8 +245,8 @@ void launch_scan(const int* in, int64_t n, TOut* out, long long* partial, ScanTa
     return;
   }
   int tiles = (int)scan_tiles(n);
-  k_scan_reduce<<<tiles, kScanThreads, 0, s>>>(in, n, partial);
-  k_scan_top<<<1, 1024, 0, s>>>(partial, tiles);
+  k_scan_reduce<<<tiles, kScanThreads, 0, s>>>(in, n, partial, tail.gate);
+  k_scan_top<<<1, 1024, 0, s>>>(partial, tiles, tail.gate);
   k_scan_down<TOut><<<tiles, kScanThreads, 0, s>>>(in, n, partial, tiles, out, tail);
 }
 
@@ -341,7 +342,7 @@ void launch_count_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
   }
   k_bin<<<atom_blocks, tb, 0, stream>>>(a, plan);
   launch_scan<int>(a.cell_count, plan.ncell_cap, a.cell_start, a.partial,
-                   ScanTail{nullptr, nullptr, 0}, stream);
+                   ScanTail{nullptr, nullptr, 0, a.gate}, stream);
   k_scatter<<<atom_blocks, tb, 0, stream>>>(a);
   if (plan.max_reach <= 1) {
     const size_t sm_count_ = cellscan_smem(false);
@@ -397,15 +398,17 @@ int launch_fused_build(const BuildArgs& a, const BuildPlan& plan, int nsplit, Fu
   return MLG_ERR_UNSUPPORTED;
 }
 
-// Test knobs of the one-launch build's bounded waits (nullptr: normal build).
-struct FusedWaitTest {
-  long long polls;   // polls of each wait before it gives up
-  int hold_release;  // CTA 0 never releases the binned atoms
+// Options of a build beyond mlg_build_csr's arguments.
+struct BuildOptions {
+  const uint32_t* gate = nullptr;  // device word: 0 = every kernel returns at once
+  bool wait_test = false;          // one-launch build only, with the two knobs below
+  long long polls = 0;             // polls of each bounded wait before it gives up
+  int hold_release = 0;            // CTA 0 never releases the binned atoms
 };
 
 int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
                const mlg_csr* csr, void* ws, size_t ws_bytes, cudaStream_t stream,
-               const FusedWaitTest* wait_test = nullptr) {
+               const BuildOptions& opt = BuildOptions()) {
   if (sys == nullptr || sys->coords == nullptr) return MLG_ERR_INVALID_ARG;
   if (sys->types != nullptr && sys->n_types < 1) return MLG_ERR_INVALID_ARG;
   int rc = check_build_args(rcut, r_on, nnei_max, csr);
@@ -420,10 +423,11 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   char* w = static_cast<char*>(ws);
   BuildArgs a = make_build_args(sys, rcut, r_on, nnei_max, csr, w, L);
   const int nsplit = build_nsplit(plan);
-  if (wait_test != nullptr) {
+  a.gate = opt.gate;
+  if (opt.wait_test) {
     if (!use_fused_build(plan, n)) return MLG_ERR_UNSUPPORTED;
-    a.spin_polls = wait_test->polls;
-    a.hold_release = wait_test->hold_release;
+    a.spin_polls = opt.polls;
+    a.hold_release = opt.hold_release;
   }
   if (use_fused_build(plan, n)) {
     // the whole build in one cooperative launch (small systems); systems of
@@ -433,12 +437,12 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
     const int rc2 = 27 * n <= kCellCandSmall
                         ? launch_fused_build<kCellCandSmall>(a, plan, nsplit, sync, stream)
                         : launch_fused_build<kCellCand>(a, plan, nsplit, sync, stream);
-    if (rc2 != MLG_ERR_UNSUPPORTED || wait_test != nullptr) return rc2;
+    if (rc2 != MLG_ERR_UNSUPPORTED || opt.wait_test) return rc2;
     // refused (not co-resident): the kernel chain below
   }
   launch_count_phase(a, plan, nsplit, stream);
   launch_scan<long long>(a.kept, n, reinterpret_cast<long long*>(a.row_ptr), a.partial,
-                         ScanTail{a.n_edges, a.status, a.capacity}, stream);
+                         ScanTail{a.n_edges, a.status, a.capacity, a.gate}, stream);
   launch_fill_phase(a, plan, nsplit, stream);
   return launch_status();
 }
@@ -786,6 +790,113 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
   return MLG_OK;
 }
 
+// Workspace of mlg_verlet_step: the list build's workspace (at rcut + skin),
+// the check's scratch words, the refine's per-destination counts and scan
+// partials.
+struct VerletLayout {
+  size_t build_bytes, scratch, kept, raw, partial, total;
+};
+
+int verlet_layout(int64_t n, double rcut, double skin, const double* box, const uint8_t* pbc,
+                  VerletLayout* V) {
+  if (!(skin >= 0.0) || !std::isfinite(skin)) return MLG_ERR_INVALID_ARG;
+  BuildPlan plan;
+  int rc = make_plan(n, rcut + skin, box, pbc, &plan);
+  if (rc != MLG_OK) return rc;
+  size_t off = align_up(build_layout(n, plan.ncell_cap).total);
+  V->build_bytes = off;
+  V->scratch = off;
+  off = align_up(off + 16);
+  V->kept = off;
+  off = align_up(off + (size_t)n * sizeof(int));
+  V->raw = off;
+  off = align_up(off + (size_t)n * sizeof(int));
+  V->partial = off;
+  off = align_up(off + (size_t)(scan_tiles(n) + 2) * sizeof(long long));
+  V->total = off;
+  return MLG_OK;
+}
+
+int verlet_step_impl(const mlg_system* sys, double rcut, double r_on, double skin,
+                     int32_t nnei_max, const mlg_verlet_list* list, const mlg_csr* out, void* ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+  if (sys == nullptr || sys->coords == nullptr || list == nullptr) return MLG_ERR_INVALID_ARG;
+  if (list->coords_ref == nullptr || list->state == nullptr || list->n_builds == nullptr)
+    return MLG_ERR_INVALID_ARG;
+  if (sys->types != nullptr && sys->n_types < 1) return MLG_ERR_INVALID_ARG;
+  int rc = check_build_args(rcut, r_on, nnei_max, out);
+  if (rc != MLG_OK) return rc;
+  rc = check_csr(&list->cand);
+  if (rc != MLG_OK) return rc;
+  const int64_t n = sys->n_atoms;
+  VerletLayout V;
+  rc = verlet_layout(n, rcut, skin, sys->box, sys->pbc, &V);
+  if (rc != MLG_OK) return rc;
+  if (ws == nullptr || ws_bytes < V.total || ((uintptr_t)ws % kAlign) != 0)
+    return MLG_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  uint32_t* gate = reinterpret_cast<uint32_t*>(w + V.scratch);
+  if (cudaMemsetAsync(gate, 0, 16, stream) != cudaSuccess) return MLG_ERR_CUDA;
+  // 1. the displacement check decides on the device whether the list is rebuilt
+  VerletCheckArgs ca;
+  ca.n = n;
+  ca.coords = sys->coords;
+  ca.coords_ref = list->coords_ref;
+  ca.state = list->state;
+  ca.skin = skin;
+  ca.gate = gate;
+  ca.done = reinterpret_cast<unsigned int*>(gate + 1);
+  ca.dmax = reinterpret_cast<unsigned long long*>(w + V.scratch + 8);
+  ca.out_status = out->status;
+  ca.out_trunc = out->n_truncated;
+  const int64_t cblocks = (n + 255) / 256;
+  const int64_t cmax = (int64_t)sm_count() * 4;
+  k_verlet_check<<<(unsigned)(cblocks < cmax ? cblocks : cmax), 256, 0, stream>>>(ca);
+  // 2. the list's build, gated on that decision, and its coordinates
+  BuildOptions opt;
+  opt.gate = gate;
+  rc = build_impl(sys, rcut + skin, r_on, kVerletListCap, &list->cand, w, V.build_bytes, stream,
+                  opt);
+  if (rc != MLG_OK) return rc;
+  const int64_t t3 = (3 * n + 255) / 256;
+  k_verlet_commit<<<(unsigned)(t3 < cmax ? t3 : cmax), 256, 0, stream>>>(
+      gate, n, sys->coords, list->coords_ref, list->state, list->n_builds);
+  // 3. the refine: count, scan, fill
+  RefineArgs ra;
+  std::memset(&ra, 0, sizeof(ra));
+  ra.n = n;
+  ra.coords = sys->coords;
+  std::memcpy(ra.box, sys->box, sizeof(ra.box));
+  ra.rcut = rcut;
+  ra.r_on = r_on;
+  ra.rc2 = rcut * rcut;
+  ra.nnei_max = nnei_max;
+  taylor_coeffs(ra.taylor);
+  ra.cp = list->cand.row_ptr;
+  ra.cs = list->cand.src;
+  ra.ch = list->cand.shift;
+  ra.cand_status = list->cand.status;
+  ra.cand_trunc = list->cand.n_truncated;
+  ra.kept = reinterpret_cast<int*>(w + V.kept);
+  ra.raw = reinterpret_cast<int*>(w + V.raw);
+  ra.capacity = out->capacity;
+  ra.row_ptr = out->row_ptr;
+  ra.src = out->src;
+  ra.shift = out->shift;
+  ra.vec = out->vec;
+  ra.dist = out->dist;
+  ra.sw = out->sw;
+  ra.n_truncated = out->n_truncated;
+  ra.status = out->status;
+  const unsigned rblocks = (unsigned)((n + kRefineWarps - 1) / kRefineWarps);
+  k_refine_count<<<rblocks, kRefineWarps * 32, 0, stream>>>(ra);
+  launch_scan<long long>(ra.kept, n, reinterpret_cast<long long*>(out->row_ptr),
+                         reinterpret_cast<long long*>(w + V.partial),
+                         ScanTail{out->n_edges, out->status, out->capacity, nullptr}, stream);
+  k_refine_fill<<<rblocks, kRefineWarps * 32, 0, stream>>>(ra);
+  return launch_status();
+}
+
 int forward_launches(int64_t n_atoms, int32_t nnei_max, int32_t channels, int32_t heads,
                      int32_t n_layers, mlg_dtype dtype) {
   const int D = heads > 0 ? channels / heads : 0;
@@ -991,12 +1102,29 @@ int mlg_exp2_neg(const double* y, double* out, int64_t n, mlg_stream_t stream) {
   return launch_status();
 }
 
+size_t mlg_verlet_workspace_bytes(int64_t n_atoms, double rcut, double skin, const double box[9],
+                                  const uint8_t pbc[3]) {
+  VerletLayout V;
+  if (verlet_layout(n_atoms, rcut, skin, box, pbc, &V) != MLG_OK) return 0;
+  return V.total;
+}
+
+int mlg_verlet_step(const mlg_system* sys, double rcut, double r_on, double skin,
+                    int32_t nnei_max, const mlg_verlet_list* list, const mlg_csr* out, void* ws,
+                    size_t ws_bytes, mlg_stream_t stream) {
+  return verlet_step_impl(sys, rcut, r_on, skin, nnei_max, list, out, ws, ws_bytes,
+                          (cudaStream_t)stream);
+}
+
 int mlg_build_csr_wait_test(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
                              const mlg_csr* csr, void* ws, size_t ws_bytes, int32_t polls,
                              mlg_stream_t stream) {
   if (polls < 1) return MLG_ERR_INVALID_ARG;
-  const FusedWaitTest t{(long long)polls, 1};
-  return build_impl(sys, rcut, r_on, nnei_max, csr, ws, ws_bytes, (cudaStream_t)stream, &t);
+  BuildOptions opt;
+  opt.wait_test = true;
+  opt.polls = polls;
+  opt.hold_release = 1;
+  return build_impl(sys, rcut, r_on, nnei_max, csr, ws, ws_bytes, (cudaStream_t)stream, opt);
 }
 
 int mlg_version(void) { return 100; }

@@ -100,6 +100,8 @@ struct BuildArgs {
   long long spin_polls;      // one-launch build: polls of each bounded wait (0: the default)
   int hold_release;          // one-launch build: CTA 0 never releases the binned atoms, so
                              // the other CTAs' waits run out (tests of the timeout path)
+  const uint32_t* gate;      // device word or nullptr: when it is 0 every kernel of the
+                             // build returns at once (a rebuild decided on the device)
   // workspace
   CellGrid* grid;
   unsigned long long* bbox;  // [6] ordered bits: min x, y, z, max x, y, z
@@ -114,6 +116,12 @@ struct BuildArgs {
   int* raw;                  // [n]
   long long* partial;        // scan partials
 };
+
+// False when the build is gated off by a device word (uniform for a launch:
+// the word is written by an earlier kernel on the same stream).
+__device__ __forceinline__ bool gated_off(const uint32_t* gate) {
+  return gate != nullptr && *gate == 0u;
+}
 
 constexpr int kFillMaxCand = 256;  // shared-memory candidates per destination
 constexpr int kCountWarps = 8;
@@ -231,6 +239,7 @@ __device__ __forceinline__ CellGrid derive_grid(const BuildPlan& p,
 // ----------------------------------------------------------------- kernels
 
 __global__ void k_init(BuildArgs a, int ncell_cap) {
+  if (gated_off(a.gate)) return;
   int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t m = t; m <= ncell_cap; m += stride) a.cell_count[m] = 0;
@@ -275,6 +284,7 @@ __device__ void bbox_accumulate(const BuildArgs& a, const BuildPlan& p, int64_t 
 }
 
 __global__ void k_bbox(BuildArgs a, BuildPlan p) {
+  if (gated_off(a.gate)) return;
   bbox_accumulate(a, p, (int64_t)blockIdx.x * blockDim.x + threadIdx.x,
                   (int64_t)gridDim.x * blockDim.x);
 }
@@ -352,6 +362,7 @@ __device__ __forceinline__ void bin_atom(const BuildArgs& a, const CellGrid& g, 
 }
 
 __global__ void k_bin(BuildArgs a, BuildPlan p) {
+  if (gated_off(a.gate)) return;
   CellGrid g = derive_grid(p, a.bbox);
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.grid = g;
   bin_atom(a, g, (int64_t)blockIdx.x * blockDim.x + threadIdx.x, a.cell_count, a.atom_rank);
@@ -376,6 +387,7 @@ __device__ __forceinline__ void scatter_atom_at(const BuildArgs& a, const CellGr
 }
 
 __global__ void k_scatter(BuildArgs a) {
+  if (gated_off(a.gate)) return;
   __shared__ CellGrid sg;
   if (threadIdx.x == 0) sg = *a.grid;
   __syncthreads();
@@ -495,6 +507,7 @@ __device__ __forceinline__ bool test_candidate(const CellGrid& g, const Centre& 
 }
 
 __global__ void __launch_bounds__(kCountWarps * 32) k_count(BuildArgs a) {
+  if (gated_off(a.gate)) return;
   __shared__ CellGrid sg;
   __shared__ WarpScratch sw[kCountWarps];
   __shared__ int s_trunc;
@@ -861,6 +874,7 @@ __device__ uint32_t fill_row_global(const BuildArgs& a, const CellGrid& g, const
 }
 
 __global__ void __launch_bounds__(kFillWarps * 32) k_fill(BuildArgs a) {
+  if (gated_off(a.gate)) return;
   __shared__ CellGrid sg;
   __shared__ WarpScratch sws[kFillWarps];
   extern __shared__ unsigned long long s_fill[];  // [warps][2][kFillMaxCand]
@@ -1186,6 +1200,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
 
 template <bool FILL>
 __global__ void __launch_bounds__(kCellWarps * 32, FILL ? 3 : 4) k_cellscan(BuildArgs a) {
+  if (gated_off(a.gate)) return;
   __shared__ CellGrid sg;
   __shared__ WarpScratch sws[kCellWarps];
   extern __shared__ __align__(16) unsigned char s_dyn[];
@@ -1244,6 +1259,7 @@ struct ScanTail {
   int64_t* n_edges;
   uint32_t* status;
   int64_t capacity;
+  const uint32_t* gate;  // as BuildArgs::gate (nullptr: always run)
 };
 
 // One block: tiles of blockDim.x x 4 items, each thread 4 contiguous items,
@@ -1278,11 +1294,14 @@ __device__ void scan_block(const int* in, int64_t n, TOut* out, ScanTail tail) {
 template <typename TOut>
 __global__ void __launch_bounds__(1024) k_scan_single(const int* in, int64_t n, TOut* out,
                                                       ScanTail tail) {
+  if (gated_off(tail.gate)) return;
   scan_block<TOut>(in, n, out, tail);
 }
 
 __global__ void __launch_bounds__(kScanThreads) k_scan_reduce(const int* in, int64_t n,
-                                                              long long* partial) {
+                                                              long long* partial,
+                                                              const uint32_t* gate) {
+  if (gated_off(gate)) return;
   const int64_t base = (int64_t)blockIdx.x * kScanTile;
   long long s = 0;
 #pragma unroll
@@ -1302,7 +1321,9 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_reduce(const int* in, int
 }
 
 // one block: exclusive scan of the tile sums in place; partial[ntiles] = total
-__global__ void __launch_bounds__(1024) k_scan_top(long long* partial, int ntiles) {
+__global__ void __launch_bounds__(1024) k_scan_top(long long* partial, int ntiles,
+                                                   const uint32_t* gate) {
+  if (gated_off(gate)) return;
   long long carry = 0;
   for (int base = 0; base < ntiles; base += blockDim.x) {
     int t = base + threadIdx.x;
@@ -1320,6 +1341,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_down(const int* in, int64
                                                             const long long* partial,
                                                             int ntiles, TOut* out,
                                                             ScanTail tail) {
+  if (gated_off(tail.gate)) return;
   const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * kScanItems;
   int v[kScanItems];
   long long s = 0;
@@ -1400,6 +1422,7 @@ __host__ __device__ constexpr bool fused_build_fits(int64_t n, int ncell_cap) {
 template <int CAP>
 __global__ void __launch_bounds__(kCellWarps * 32, 2)
     k_build_fused(BuildArgs a, BuildPlan p, int ncell_cap, int nsplit, FusedSync* sync) {
+  if (gated_off(a.gate)) return;  // before any wait: every CTA leaves alike
   __shared__ CellGrid sg;
   __shared__ WarpScratch sws[kCellWarps];
   __shared__ int s_ok;

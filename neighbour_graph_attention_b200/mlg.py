@@ -47,6 +47,7 @@ MLG_STATUS_TIES = 16
 MLG_STATUS_INTERNAL = 32
 MLG_STATUS_TIMEOUT = 64
 MLG_STATUS_ROW_TOO_LONG = 128
+MLG_STATUS_LIST_INCOMPLETE = 256
 
 MLG_F32 = 0
 MLG_F64 = 1
@@ -63,6 +64,10 @@ class mlg_system(ctypes.Structure):
 class mlg_csr(ctypes.Structure):
     _fields_ = [("capacity", _c_i64), ("row_ptr", _p), ("src", _p), ("shift", _p), ("vec", _p),
                 ("dist", _p), ("sw", _p), ("n_edges", _p), ("n_truncated", _p), ("status", _p)]
+
+
+class mlg_verlet_list(ctypes.Structure):
+    _fields_ = [("cand", mlg_csr), ("coords_ref", _p), ("state", _p), ("n_builds", _p)]
 
 
 _lib.mlg_build_csr_workspace_bytes.restype = _c_sz
@@ -107,6 +112,12 @@ _lib.mlg_local_attention.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c
                                      ctypes.c_int, _p, _p, _p, _p, _p, _p, _p]
 _lib.mlg_exp2_neg.restype = ctypes.c_int
 _lib.mlg_exp2_neg.argtypes = [_p, _p, _c_i64, _p]
+_lib.mlg_verlet_workspace_bytes.restype = _c_sz
+_lib.mlg_verlet_workspace_bytes.argtypes = [_c_i64, _c_dbl, _c_dbl, _p, _p]
+_lib.mlg_verlet_step.restype = ctypes.c_int
+_lib.mlg_verlet_step.argtypes = [ctypes.POINTER(mlg_system), _c_dbl, _c_dbl, _c_dbl, _c_i32,
+                                 ctypes.POINTER(mlg_verlet_list), ctypes.POINTER(mlg_csr), _p,
+                                 _c_sz, _p]
 _lib.mlg_build_csr_wait_test.restype = ctypes.c_int
 _lib.mlg_build_csr_wait_test.argtypes = [ctypes.POINTER(mlg_system), _c_dbl, _c_dbl, _c_i32,
                                          ctypes.POINTER(mlg_csr), _p, _c_sz, _c_i32, _p]
@@ -278,6 +289,54 @@ def mlg_build_csr(system: mlg_system, rcut: float, r_on: float, nnei_max: int, c
     code = _lib.mlg_build_csr(ctypes.byref(system), float(rcut), float(r_on), int(nnei_max),
                               ctypes.byref(c), _ptr(ws), nbytes, _stream_handle(stream))
     return _check(code, "mlg_build_csr", check)
+
+
+@dataclass
+class VerletList:
+    """Caller-owned device buffers of a Verlet candidate list (torch tensors):
+    the candidate CSR at rcut + skin, the coordinates it was built at, its
+    state word (zero: no valid list yet) and a counter of its builds."""
+
+    cand: Csr
+    coords_ref: object
+    state: object
+    n_builds: object
+
+    @classmethod
+    def empty(cls, n_atoms: int, capacity: int, device="cuda"):
+        import torch
+        return cls(Csr.empty(n_atoms, capacity, device=device),
+                   torch.zeros((max(n_atoms, 1), 3), dtype=torch.float64, device=device),
+                   torch.zeros(1, dtype=torch.int32, device=device),
+                   torch.zeros(1, dtype=torch.int64, device=device))
+
+    def struct(self) -> mlg_verlet_list:
+        v = mlg_verlet_list()
+        v.cand = self.cand.struct()
+        v.coords_ref = _ptr(self.coords_ref)
+        v.state = _ptr(self.state)
+        v.n_builds = _ptr(self.n_builds)
+        return v
+
+
+def mlg_verlet_workspace_bytes(n_atoms: int, rcut: float, skin: float, box, pbc) -> int:
+    b, q = _box_pbc(box, pbc)
+    return int(_lib.mlg_verlet_workspace_bytes(int(n_atoms), float(rcut), float(skin),
+                                               b.ctypes.data, q.ctypes.data))
+
+
+def mlg_verlet_step(system: mlg_system, rcut: float, r_on: float, skin: float, nnei_max: int,
+                    vlist: VerletList, out: Csr, ws, ws_bytes: int | None = None, stream=None,
+                    check: bool = True) -> int:
+    """One step's CSR through the Verlet list (rebuilt on the device when some
+    atom has moved skin / 2 or more), written to ``out``."""
+    v = vlist.struct()
+    c = out.struct()
+    nbytes = int(ws.numel() * ws.element_size()) if ws_bytes is None else int(ws_bytes)
+    code = _lib.mlg_verlet_step(ctypes.byref(system), float(rcut), float(r_on), float(skin),
+                                int(nnei_max), ctypes.byref(v), ctypes.byref(c), _ptr(ws),
+                                nbytes, _stream_handle(stream))
+    return _check(code, "mlg_verlet_step", check)
 
 
 def mlg_build_csr_wait_test(system: mlg_system, rcut: float, r_on: float, nnei_max: int,

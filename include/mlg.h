@@ -205,8 +205,10 @@ int mlg_block_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
  *   m_a = max(max_b l_ab, 0 if phi > 0),  D~ = sum_b exp(l_ab - m_a) + phi exp(-m_a),
  *   G_out[a, h d + t] = sum_b exp(l_ab - m_a) v_b[t] / D~.
  * Destinations with more than nnei_max edges are left untouched and flagged with
- * MLG_STATUS_ROW_TOO_LONG.  Runs on
- * the generic kernel (no fused tiles yet); no workspace. */
+ * MLG_STATUS_ROW_TOO_LONG.  Runs on the fused kernels of mlg_block_attention
+ * (the phantoms only start each row's running softmax at maximum 0 with sum
+ * phi), except fp64 with 32 channels, which takes the generic kernel; no
+ * workspace. */
 int mlg_block_attention_smooth(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                                int32_t channels, int32_t heads, mlg_dtype dtype,
                                const void* G_in, void* G_out, const void* Wq, const void* Wk,
@@ -229,6 +231,15 @@ int mlg_attention_stack(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                         int32_t channels, int32_t heads, int32_t n_layers, mlg_dtype dtype,
                         const void* const* W, const void* G_in, void* G_out, void* ws,
                         size_t ws_bytes, mlg_stream_t stream);
+
+/* mlg_attention_stack with the slot-occupancy softmax of
+ * mlg_block_attention_smooth in every layer (the phantom count nnei_max - n of a
+ * destination depends on the geometry only, so it is the same in every layer).
+ * Same arguments, workspace and outputs as mlg_attention_stack. */
+int mlg_attention_stack_smooth(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                               int32_t channels, int32_t heads, int32_t n_layers,
+                               mlg_dtype dtype, const void* const* W, const void* G_in,
+                               void* G_out, void* ws, size_t ws_bytes, mlg_stream_t stream);
 
 /* Bytes of device workspace for mlg_forward: the build's workspace plus, for
  * n_layers >= 2, one [capacity][channels] buffer for the layer ping-pong. */

@@ -16,6 +16,7 @@
 #include "mlg_attn_hg.cuh"
 #include "mlg_attn_dmma.cuh"
 #include "mlg_attn_tc.cuh"
+#include "mlg_attn_tc2.cuh"
 #include "mlg_local.cuh"
 #include "mlg_verlet.cuh"
 
@@ -608,7 +609,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-bool encode_slab_map(CUtensorMap* map, const void* G, int64_t rows, int C) {
+bool encode_slab_map(CUtensorMap* map, const void* G, int64_t rows, int C, int box_rows = 128) {
   static EncodeTiledFn fn = nullptr;
   if (fn == nullptr) {
     void* p = nullptr;
@@ -621,7 +622,7 @@ bool encode_slab_map(CUtensorMap* map, const void* G, int64_t rows, int C) {
   }
   const cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)(rows > 0 ? rows : 1)};
   const cuuint64_t strides[1] = {(cuuint64_t)C * 4};
-  const cuuint32_t box[2] = {4, 128};
+  const cuuint32_t box[2] = {4, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(G), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -646,6 +647,21 @@ int launch_tc(TileArgs& ta, cudaStream_t stream) {
   int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
   if (grid < 1) grid = 1;
   kern<<<grid, NT, Cfg::SMEM, stream>>>(ta, map);
+  return launch_status();
+}
+
+// fp32, 32 channels, 4 heads, one layer: every product on tcgen05 (centres of
+// up to 64 edges); one CTA of 320 threads per SM holding all of its TMEM.
+int launch_tc2(TileArgs& ta, cudaStream_t stream) {
+  auto kern = k_attn_tc2;
+  prefer_shared(kern, tc2::SMEM);
+  if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
+  CUtensorMap map;
+  if (!encode_slab_map(&map, ta.G, ta.capacity, tc2::C, 32)) return MLG_ERR_CUDA;
+  const int64_t want = sm_count();
+  int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
+  if (grid < 1) grid = 1;
+  kern<<<grid, tc2::NT, tc2::SMEM, stream>>>(ta, map);
   return launch_status();
 }
 
@@ -720,11 +736,13 @@ int check_attention_args(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
 
 // n_layers attention layers G^{l+1} = attention(G^l), G^0 = G_in, result in
 // G_out.  `pong` is a [capacity][channels] buffer, needed only for
-// n_layers >= 2 on the generic path.
+// n_layers >= 2 on the generic path.  With `smooth`, every layer uses the
+// slot-occupancy softmax (phantom slots up to nnei_max); the FP64 tensor-core
+// kernel has no such variant, so that shape runs on the generic kernel.
 int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
                          int32_t channels, int32_t heads, mlg_dtype dtype, int32_t n_layers,
                          const void* const* W, const void* G_in, void* G_out, void* pong,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, int smooth = 0) {
   int rc = check_attention_args(csr, n_centres, nnei_max, channels, heads, dtype, G_in, G_out);
   if (rc != MLG_OK) return rc;
   if (n_layers < 1 || W == nullptr) return MLG_ERR_INVALID_ARG;
@@ -734,6 +752,7 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
   if (n_centres == 0) return MLG_OK;
   const int D = channels / heads;
   int R = tile_rows(dtype, channels, D, nnei_max);
+  if (smooth && dtype == MLG_F64) R = 0;  // no slot-occupancy FP64 tensor-core kernel
   bool tile_ok = R > 0 && n_layers <= kMaxFusedLayers && aligned16(G_in) && aligned16(G_out);
   for (int k = 0; tile_ok && k < 3 * n_layers; ++k) tile_ok = aligned16(W[k]);
   int min_n = 0;  // generic path: centres with more than min_n edges
@@ -746,12 +765,25 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
     ta.capacity = csr->capacity;
     ta.n_layers = n_layers;
     ta.nnei_max = nnei_max;
+    ta.smooth = smooth;
     ta.G = G_in;
     ta.out = G_out;
     for (int k = 0; k < 3 * n_layers; ++k) ta.W[k] = W[k];
     ta.status = csr->status;
-    rc = launch_tile_shape(dtype, channels, D, nnei_max, ta, stream);
-    if (rc != MLG_OK) return rc;
+    if (dtype == MLG_F32 && channels == 32 && D == 8 && n_layers == 1) {
+      // centres of up to 64 edges with every product on tcgen05; longer ones
+      // (up to the tile) on the kernel whose logits and P V run on the FP32 pipe
+      rc = launch_tc2(ta, stream);
+      if (rc != MLG_OK) return rc;
+      if (nnei_max > tc2::MAXN) {
+        ta.min_n = tc2::MAXN;
+        rc = launch_tile_shape(dtype, channels, D, nnei_max, ta, stream);
+        if (rc != MLG_OK) return rc;
+      }
+    } else {
+      rc = launch_tile_shape(dtype, channels, D, nnei_max, ta, stream);
+      if (rc != MLG_OK) return rc;
+    }
     if (nnei_max <= R) return MLG_OK;  // no centre can exceed the tile
     min_n = R;
   }
@@ -771,6 +803,7 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
       ha.n_centres = n_centres;
       ha.capacity = csr->capacity;
       ha.nnei_max = nnei_max;
+      ha.smooth = smooth;
       ha.G = in;
       ha.out = dst;
       ha.Wq = W[3 * l];
@@ -782,7 +815,7 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
     }
     if (min_n >= 0) {
       rc = launch_generic(csr, n_centres, nnei_max, channels, heads, dtype, in, dst, W[3 * l],
-                          W[3 * l + 1], W[3 * l + 2], min_n, stream);
+                          W[3 * l + 1], W[3 * l + 2], min_n, stream, smooth);
       if (rc != MLG_OK) return rc;
     }
     in = dst;
@@ -901,7 +934,10 @@ int forward_launches(int64_t n_atoms, int32_t nnei_max, int32_t channels, int32_
                      int32_t n_layers, mlg_dtype dtype) {
   const int D = heads > 0 ? channels / heads : 0;
   int R = tile_rows(dtype, channels, D, nnei_max);
-  if (R > 0 && n_layers <= kMaxFusedLayers) return 1 + (nnei_max > R ? n_layers : 0);
+  if (R > 0 && n_layers <= kMaxFusedLayers) {
+    const bool tc2_path = dtype == MLG_F32 && channels == 32 && D == 8 && n_layers == 1;
+    return 1 + (tc2_path && nnei_max > tc2::MAXN ? 1 : 0) + (nnei_max > R ? n_layers : 0);
+  }
   int Rg = hg_rows(dtype, channels, D);
   if (Rg > 0) return n_layers * (1 + (nnei_max > Rg ? 1 : 0));
   (void)n_atoms;
@@ -1007,9 +1043,9 @@ int mlg_block_attention_smooth(const mlg_csr* csr, int64_t n_centres, int32_t nn
   int rc = check_attention_args(csr, n_centres, nnei_max, channels, heads, dtype, G_in, G_out);
   if (rc != MLG_OK) return rc;
   if (!Wq || !Wk || !Wv) return MLG_ERR_INVALID_ARG;
-  if (n_centres == 0) return MLG_OK;
-  return launch_generic(csr, n_centres, nnei_max, channels, heads, dtype, G_in, G_out, Wq, Wk, Wv,
-                        0, (cudaStream_t)stream, 1);
+  const void* W[3] = {Wq, Wk, Wv};
+  return attention_stack_impl(csr, n_centres, nnei_max, channels, heads, dtype, 1, W, G_in, G_out,
+                              nullptr, (cudaStream_t)stream, 1);
 }
 
 size_t mlg_attention_stack_workspace_bytes(int64_t capacity, int32_t channels, int32_t n_layers,
@@ -1017,6 +1053,17 @@ size_t mlg_attention_stack_workspace_bytes(int64_t capacity, int32_t channels, i
   if (capacity < 0 || channels < 1 || n_layers < 1) return 0;
   size_t el = dtype == MLG_F64 ? 8 : 4;
   return n_layers >= 2 ? align_up((size_t)(capacity > 0 ? capacity : 1) * channels * el) : 0;
+}
+
+int mlg_attention_stack_smooth(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
+                               int32_t channels, int32_t heads, int32_t n_layers,
+                               mlg_dtype dtype, const void* const* W, const void* G_in,
+                               void* G_out, void* ws, size_t ws_bytes, mlg_stream_t stream) {
+  if (csr == nullptr) return MLG_ERR_INVALID_ARG;
+  size_t need = mlg_attention_stack_workspace_bytes(csr->capacity, channels, n_layers, dtype);
+  if (need > 0 && (ws == nullptr || ws_bytes < need)) return MLG_ERR_WORKSPACE;
+  return attention_stack_impl(csr, n_centres, nnei_max, channels, heads, dtype, n_layers, W, G_in,
+                              G_out, need > 0 ? ws : nullptr, (cudaStream_t)stream, 1);
 }
 
 int mlg_attention_stack(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,

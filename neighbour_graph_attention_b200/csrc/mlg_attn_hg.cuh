@@ -29,6 +29,7 @@ struct HgArgs {
   int64_t n_centres;
   int64_t capacity;
   int nnei_max;  // centres with more edges are skipped and flagged
+  int smooth;    // slot-occupancy softmax (phantom slots up to nnei_max)
   const void* G;
   void* out;
   const void* Wq;
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(NT) k_attn_hg(HgArgs a) {
     __syncthreads();
 
     // ---- 2. attention of the group's heads (outputs into the q slots)
-    tile_attention<T, HG, D, GW, NT, QS>(sQ, meta, 0, warp, lane);
+    tile_attention<T, HG, D, GW, NT, QS>(sQ, meta, 0, warp, lane, a.smooth ? a.nnei_max : 0);
     __syncthreads();
     // ---- 3. the group's output columns, row by row (coalesced segments)
     constexpr int OV = GW * (int)sizeof(T) / 16;

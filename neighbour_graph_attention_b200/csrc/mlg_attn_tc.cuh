@@ -191,14 +191,14 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
       const int c_end = meta.c_end;
       while (c < c_end) {
         const int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
-        if (n > 0 && n <= R && n <= a.nnei_max) break;
+        if (n > a.min_n && n <= R && n <= a.nnei_max) break;
         if (n > a.nnei_max) atomicOr(a.status, (uint32_t)MLG_STATUS_ROW_TOO_LONG);
         ++c;
       }
       meta.row0[b] = c < c_end ? a.row_ptr[c] : 0;
       while (c < c_end && k < 64) {
         const int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
-        if (n > R || n > a.nnei_max || rows + n > R) break;
+        if (n <= a.min_n || n > R || n > a.nnei_max || rows + n > R) break;
         meta.off[b][k] = rows;
         meta.task0[b][k] = tasks;
         tasks += (n * H + 31) / 32;
@@ -327,7 +327,8 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
       tc_fence_before();
       __syncthreads();
       // ---- 2. attention (SIMT), output into the q slots
-      tile_attention<float, H, D, C, NT, QS>(sQ, meta, cur, warp, lane);
+      tile_attention<float, H, D, C, NT, QS>(sQ, meta, cur, warp, lane,
+                                             a.smooth ? a.nnei_max : 0);
       __syncthreads();
     }
     if (meta.fail) break;

@@ -1,0 +1,613 @@
+// mlg_attn_tc2.cuh -- fp32 block-dense attention with every product on the
+// 5th-generation tensor cores: the projection, the logits S = Q K^T and the
+// weighted sum P V (tcgen05.mma kind::tf32, 3xTF32 splits, accumulators in
+// TMEM).  Shape: 32 channels, 4 heads of 8, one layer, centres of 1..64
+// edges (the Fe BCC systems have 64); other centres are left to the kernels
+// that handle them in the same call.
+//
+// Per centre i with n edges (NeighborGraph issue, Proposed fix: each
+// centre's edges are one small dense block, attended to with dense
+// products, unequal lengths masked per row, outputs returned to the edges):
+//   q_a = s_a G_a Wq log2(e)/sqrt(d),  k_b = s_b G_b Wk,  v_b = G_b Wv
+//   S_ab = q_a . k_b (per head),  P_ab = 2^(S_ab - max_b S_ab),
+//   O_a = sum_b P_ab v_b / sum_b P_ab.
+//
+// Tiles of 128 rows hold up to two centres, each starting at a multiple of
+// 32 rows, so that every warp's TMEM lane quadrant belongs to one centre.
+//   projection  D[128 x 96] = X[128 x 32] . [Wq|Wk|Wv], 3xTF32 (12 MMAs)
+//   Q           read back, scaled, split into TF32 hi/lo and stored back
+//               into TMEM: the A operand of the logits (A from TMEM)
+//   K, V^T      read back, split, stored as shared-memory B operands
+//   logits      per (head, centre): S = Q_h . K_h^T over the centre's keys,
+//               M = 128 (only the centre's rows are used), N = ceil16(n), 3 MMAs
+//   softmax     one thread per row: its S row from TMEM, max, 2^(S - max),
+//               sum; P split into hi (top 11 bits) and lo (the rest, exact)
+//               and written back to TMEM over S
+//   P V         per (head, centre): O += [P_hi | P_lo] . [V_hi^T ; V_lo^T]
+//               (N = 16: columns 0-7 collect .V_hi, 8-15 .V_lo; all four
+//               products of the two splits), A from TMEM
+//   epilogue    O = (cols 0-7 + cols 8-15) / sum, staged in shared memory,
+//               one bulk copy per centre
+// The rounding of a split product is that of an fp32 product: each operand
+// x = hi + lo with |lo| <= 2^-11 |x| (rounded hi) or 2^-10 |x| (truncated
+// hi) and lo exact, so the dropped lo.lo term and the TF32 reading of lo are
+// below 2^-20 of the product.
+//
+// Warp roles (320 threads, one CTA per SM):
+//   warp 0     issues every MMA (one elected thread) and commits them to
+//              mbarriers
+//   warp 1     plans tiles and loads each slab with 2-D TMA boxes of
+//              {4 channels x 32 rows} straight into the K-major operand
+//              layout; the next slab lands while the current tile computes
+//   warps 2-5  group 0: split, Q and K, softmax of heads 0 and 2, epilogue
+//   warps 6-9  group 1: split, V, softmax of heads 1 and 3, epilogue
+// A warp w reads TMEM lanes 32 (w % 4) .. +31, i.e. tile rows of one
+// quadrant.  Every wait is bounded; on expiry the kernel records
+// MLG_STATUS_TIMEOUT, every role leaves its loop, and the CTA lets its
+// last slab copy land before it frees TMEM and exits.
+#pragma once
+
+#include <cuda.h>
+
+#include "mlg_common.cuh"
+#include "mlg_attn_tile.cuh"
+#include "mlg_attn_tc.cuh"
+
+namespace mlg {
+
+namespace tc2 {
+
+constexpr int C = 32, D = 8, H = 4, N3 = 96, R = 128;
+constexpr int MAXN = 64;        // most edges of a centre handled here
+constexpr int NT = 320;         // threads
+constexpr int GT = 128;         // threads per compute group
+constexpr int VLBO = 144;       // V^T operand: bytes between 4-key chunks (bank spread)
+
+// TMEM columns (512 allocated)
+constexpr uint32_t T_PROJ = 0;    // projection D: q 0-31, k 32-63, v 64-95; Q lo at 96-127
+constexpr uint32_t T_QLO = 96;
+constexpr uint32_t T_O = 128;     // O of (head h, centre c): T_O + (2 h + c) * 16
+constexpr uint32_t T_SP = 256;    // S / P buffer b: T_SP + 128 b (S of centre c at +64 c;
+                                  // P hi at +0, P lo at +64)
+
+// shared memory layout (bytes)
+constexpr size_t W_BYTES = (size_t)N3 * C * 4;          // one of W hi / lo (B operand)
+constexpr size_t A_BYTES = (size_t)R * C * 4;           // one of X hi / lo, the raw slab
+constexpr size_t K_BYTES = (size_t)R * D * 4;           // one head of K hi or lo
+constexpr size_t V_BYTES = (size_t)(R / 4) * VLBO;      // one head of V^T hi or lo
+constexpr size_t OFF_WHI = 0;
+constexpr size_t OFF_WLO = OFF_WHI + W_BYTES;
+constexpr size_t OFF_X = OFF_WLO + W_BYTES;             // raw slab (TMA target)
+constexpr size_t OFF_AHI = OFF_X + A_BYTES;
+constexpr size_t OFF_ALO = OFF_AHI + A_BYTES;
+constexpr size_t OFF_K = OFF_ALO + A_BYTES;             // [head][hi, lo]
+constexpr size_t OFF_V = OFF_K + 2 * H * K_BYTES;       // [head][hi, lo]
+constexpr size_t OFF_OUT = OFF_V + 2 * H * V_BYTES;     // [128][32] row-major staging
+constexpr size_t OFF_META = OFF_OUT + A_BYTES;
+
+struct Plan {
+  int ncent;        // 0: no work left
+  int grp[2];       // first 32-row group of each centre
+  int n[2];         // edges of each centre
+  long long row0[2];
+};
+
+struct Meta {
+  Plan plan[2];             // ring of two: the tile being computed and the next
+  int fail;
+  uint32_t tmem;
+  int last_slot;            // ring slot of the last slab copy issued (-1: none)
+  uint32_t last_par;        // and the parity of the phase it completes
+  uint64_t bar_xfull[2];    // slab and plan of ring slot landed (TMA tx)
+  uint64_t bar_xfree;       // the groups have split the slab (count 2 * GT)
+  uint64_t bar_w;           // weights split (count 2 * GT)
+  uint64_t bar_a;           // A operands split (count 2 * GT)
+  uint64_t bar_proj;        // projection done (commit)
+  uint64_t bar_qk;          // Q in TMEM, K in shared memory (count GT)
+  uint64_t bar_v;           // V^T in shared memory (count GT)
+  uint64_t bar_s[2];        // logits of buffer b done (commit)
+  uint64_t bar_p[2];        // P of buffer b written (count GT)
+  uint64_t bar_pv[2];       // P V of buffer b's head done (commit)
+  uint64_t bar_epi;         // both groups staged their outputs (count 2 * GT)
+  uint64_t bar_fin;         // every MMA of the CTA done (commit, at exit)
+};
+constexpr size_t SMEM = OFF_META + sizeof(Meta);
+static_assert(SMEM <= 227 * 1024, "shared memory");
+static_assert(SMEM > 116 * 1024, "one CTA per SM (the kernel holds all 512 TMEM columns)");
+
+// A waiter's view of an mbarrier: the parity of the phase it waits for next.
+struct Waiter {
+  uint32_t par = 0;
+  __device__ __forceinline__ bool wait(uint64_t* bar) {
+    const bool ok = mbar_wait(bar, par);
+    par ^= 1u;
+    return ok;
+  }
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void umma_tf32_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(addr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__host__ __device__ constexpr uint32_t idesc_tf32(int m, int n) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(m >> 4) << 24);
+}
+
+// The centre (0, 1) whose 32-row groups include group g, or -1.
+__device__ __forceinline__ int centre_of_group(const Plan& p, int g) {
+  for (int c = 0; c < p.ncent; ++c)
+    if (g >= p.grp[c] && g < p.grp[c] + (p.n[c] + 31) / 32) return c;
+  return -1;
+}
+
+}  // namespace tc2
+
+__global__ void __launch_bounds__(tc2::NT, 1)
+    k_attn_tc2(TileArgs a, const __grid_constant__ CUtensorMap gmap) {
+  using namespace tc2;
+  extern __shared__ __align__(1024) unsigned char smem_t2[];
+  unsigned char* sm = smem_t2;
+  Meta& mt = *reinterpret_cast<Meta*>(sm + OFF_META);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t E = a.row_ptr[a.n_centres];
+  if (E > a.capacity || (*a.status & MLG_STATUS_CAPACITY)) return;
+
+  if (tid == 0) {
+    mt.fail = 0;
+    mt.last_slot = -1;
+    mt.last_par = 0;
+    mbar_init(&mt.bar_xfull[0], 1);
+    mbar_init(&mt.bar_xfull[1], 1);
+    mbar_init(&mt.bar_xfree, 2 * GT);
+    mbar_init(&mt.bar_w, 2 * GT);
+    mbar_init(&mt.bar_a, 2 * GT);
+    mbar_init(&mt.bar_proj, 1);
+    mbar_init(&mt.bar_qk, GT);
+    mbar_init(&mt.bar_v, GT);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&mt.bar_s[b], 1);
+      mbar_init(&mt.bar_p[b], GT);
+      mbar_init(&mt.bar_pv[b], 1);
+    }
+    mbar_init(&mt.bar_epi, 2 * GT);
+    mbar_init(&mt.bar_fin, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&mt.tmem)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = mt.tmem;
+
+  if (warp == 1) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const int64_t r0 = E * blockIdx.x / gridDim.x, r1 = E * (blockIdx.x + 1) / gridDim.x;
+      auto lb = [&](int64_t r) {
+        int64_t lo = 0, hi = a.n_centres;
+        while (lo < hi) {
+          const int64_t mid = (lo + hi) >> 1;
+          if (a.row_ptr[mid] < r) lo = mid + 1; else hi = mid;
+        }
+        return lo;
+      };
+      int64_t c = lb(r0);
+      const int64_t c_end = blockIdx.x + 1 == gridDim.x ? a.n_centres : lb(r1);
+      const int nlim = a.nnei_max < MAXN ? a.nnei_max : MAXN;
+      Waiter wfree;
+      for (int t = 0;; ++t) {
+        const int s = t & 1;
+        if (t > 0 && !wfree.wait(&mt.bar_xfree)) {  // the previous slab was split
+          mt.fail = 1;
+          break;
+        }
+        Plan p;
+        p.ncent = 0;
+        int groups = 0;
+        while (c < c_end && p.ncent < 2) {
+          const int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
+          if (n > a.nnei_max) atomicOr(a.status, (uint32_t)MLG_STATUS_ROW_TOO_LONG);
+          if (n < 1 || n > nlim) {  // empty, too long, or left to another kernel
+            ++c;
+            continue;
+          }
+          const int g = (n + 31) / 32;
+          if (groups + g > R / 32) break;
+          p.grp[p.ncent] = groups;
+          p.n[p.ncent] = n;
+          p.row0[p.ncent] = a.row_ptr[c];
+          ++p.ncent;
+          groups += g;
+          ++c;
+        }
+        mt.plan[s] = p;
+        if (p.ncent == 0) {
+          mbar_arrive(&mt.bar_xfull[s]);  // no copy: the phase completes at once
+          break;
+        }
+        fence_proxy_async();
+        uint32_t bytes = 0;
+        for (int k = 0; k < p.ncent; ++k) bytes += (uint32_t)((p.n[k] + 31) / 32) * 32 * C * 4;
+        mbar_expect_tx(&mt.bar_xfull[s], bytes);
+        for (int k = 0; k < p.ncent; ++k)
+          for (int g = 0; g < (p.n[k] + 31) / 32; ++g)
+            for (int cc = 0; cc < C / 4; ++cc)
+              tma_load_2d(sm + OFF_X + (size_t)cc * (R * 16) + (size_t)(p.grp[k] + g) * 512,
+                          &gmap, 4 * cc, (int)(p.row0[k] + 32 * g), &mt.bar_xfull[s]);
+        mt.last_slot = s;
+        mt.last_par = (uint32_t)((t >> 1) & 1);  // the phase of slot s this copy completes
+      }
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      Waiter wa, wqk, wv, wp[2], wpv[2], ww;
+      bool ok = ww.wait(&mt.bar_w);
+      for (int t = 0; ok; ++t) {
+        if (!wa.wait(&mt.bar_a)) { ok = false; break; }
+        const Plan p = mt.plan[t & 1];
+        if (p.ncent == 0) break;
+        if (t > 0) {
+          // the last two P V of the previous tile (heads 2 and 3) have read
+          // their P and Q before the projection rewrites that TMEM
+          if (!wpv[0].wait(&mt.bar_pv[0]) || !wpv[1].wait(&mt.bar_pv[1])) { ok = false; break; }
+        }
+        tc_fence_after();
+        // projection: D[128 x 96] = X . W, 3xTF32, small terms first
+        {
+          const uint32_t ahi = smem_u32(sm + OFF_AHI), alo = smem_u32(sm + OFF_ALO);
+          const uint32_t bhi = smem_u32(sm + OFF_WHI), blo = smem_u32(sm + OFF_WLO);
+          const uint32_t id = idesc_tf32(R, N3);
+#pragma unroll
+          for (int s = 0; s < C / 8; ++s) {
+            const uint32_t aoff = (uint32_t)(s * R * 32), boff = (uint32_t)(s * N3 * 32);
+            const uint64_t dah = umma_sdesc(ahi + aoff, R * 16, 128);
+            const uint64_t dal = umma_sdesc(alo + aoff, R * 16, 128);
+            const uint64_t dbh = umma_sdesc(bhi + boff, N3 * 16, 128);
+            const uint64_t dbl = umma_sdesc(blo + boff, N3 * 16, 128);
+            umma_tf32(tmem + T_PROJ, dal, dbh, id, s > 0 ? 1u : 0u);
+            umma_tf32(tmem + T_PROJ, dah, dbl, id, 1u);
+            umma_tf32(tmem + T_PROJ, dah, dbh, id, 1u);
+          }
+          umma_commit(&mt.bar_proj);
+        }
+        // logits of head h into buffer b: per centre, 3 MMAs (A = Q from TMEM)
+        auto issue_s = [&](int h, int b) {
+          for (int c = 0; c < p.ncent; ++c) {
+            const int nn = (p.n[c] + 15) & ~15;
+            const uint32_t id = idesc_tf32(R, nn);
+            const uint32_t khi = smem_u32(sm + OFF_K + (size_t)(2 * h) * K_BYTES) + 512u * p.grp[c];
+            const uint32_t klo = khi + (uint32_t)K_BYTES;
+            const uint64_t dkh = umma_sdesc(khi, R * 16, 128);
+            const uint64_t dkl = umma_sdesc(klo, R * 16, 128);
+            const uint32_t d = tmem + T_SP + 128u * b + 64u * c;
+            umma_tf32_ts(d, tmem + T_QLO + 8u * h, dkh, id, 0u);
+            umma_tf32_ts(d, tmem + T_PROJ + 8u * h, dkl, id, 1u);
+            umma_tf32_ts(d, tmem + T_PROJ + 8u * h, dkh, id, 1u);
+          }
+          umma_commit(&mt.bar_s[b]);
+        };
+        if (!wqk.wait(&mt.bar_qk)) { ok = false; break; }
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 1);
+        if (!wv.wait(&mt.bar_v)) { ok = false; break; }
+        for (int h = 0; h < H && ok; ++h) {
+          const int b = h & 1;
+          if (!wp[b].wait(&mt.bar_p[b])) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t id = idesc_tf32(R, 16);
+          for (int c = 0; c < p.ncent; ++c) {
+            const int ks = ((p.n[c] + 15) & ~15) / 8;
+            const uint32_t vhi = smem_u32(sm + OFF_V + (size_t)(2 * h) * V_BYTES);
+            const uint32_t sbo = (uint32_t)V_BYTES;  // hi rows (t) -> lo rows (t)
+            const uint32_t d = tmem + T_O + 16u * (2 * h + c);
+            const uint32_t pb = tmem + T_SP + 128u * b;
+            for (int k = 0; k < ks; ++k) {
+              const uint32_t kc = (uint32_t)(p.grp[c] * 8 + 2 * k);  // 4-key chunk
+              const uint64_t dv = umma_sdesc(vhi + kc * VLBO, VLBO, sbo);
+              umma_tf32_ts(d, pb + 8u * k, dv, id, k > 0 ? 1u : 0u);
+            }
+            for (int k = 0; k < ks; ++k) {
+              const uint32_t kc = (uint32_t)(p.grp[c] * 8 + 2 * k);
+              const uint64_t dv = umma_sdesc(vhi + kc * VLBO, VLBO, sbo);
+              umma_tf32_ts(d, pb + 64u + 8u * k, dv, id, 1u);
+            }
+          }
+          umma_commit(&mt.bar_pv[b]);
+          if (h + 2 < H) {
+            // the buffer is free once this P V has read it
+            if (!wpv[b].wait(&mt.bar_pv[b])) { ok = false; break; }
+            issue_s(h + 2, b);
+          }
+        }
+      }
+      if (!ok) mt.fail = 1;
+      // every MMA issued here is complete before TMEM is freed
+      umma_commit(&mt.bar_fin);
+      if (!mbar_wait(&mt.bar_fin, 0u)) mt.fail = 1;
+    }
+  } else {
+    // ------------------------------------------------------------ compute groups
+    const int grp = (warp - 2) >> 2;           // 0 or 1
+    const int gt = tid - 64 - grp * GT;        // 0..127 within the group
+    const int quad = warp & 3;                 // TMEM lane quadrant
+    const int row = quad * 32 + lane;          // tile row of this thread
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const float qscale = (float)(1.4426950408889634 / 2.8284271247461903);  // log2(e)/sqrt(8)
+    Waiter wx[2], wproj, ws[2], wpv[2], wepi;
+    bool ok = true;
+    // weights of the layer, split into TF32 hi / lo, K-major [96 x 32]
+    for (int e = tid - 64; e < C * N3; e += 2 * GT) {
+      const int k = e / N3, nn = e - k * N3;
+      const int m = nn / C, cc = nn - m * C;
+      const float w = static_cast<const float*>(a.W[m])[k * C + cc];
+      const float hi = tf32_rna(w);
+      const uint32_t off = kmajor_offset(nn, k, N3);
+      *reinterpret_cast<float*>(sm + OFF_WHI + off) = hi;
+      *reinterpret_cast<float*>(sm + OFF_WLO + off) = tf32_rna(w - hi);
+    }
+    fence_proxy_async();
+    mbar_arrive(&mt.bar_w);
+    float rinv[2] = {0.f, 0.f};
+    for (int t = 0; ok; ++t) {
+      const int s = t & 1;
+      if (!wx[s].wait(&mt.bar_xfull[s])) { ok = false; break; }
+      const Plan p = mt.plan[s];
+      if (p.ncent == 0) {
+        mbar_arrive(&mt.bar_a);  // lets the MMA thread see the end
+        break;
+      }
+      // ---- split the slab into the A operands; rows outside the centres are 0
+      {
+        const float* sX = reinterpret_cast<const float*>(sm + OFF_X);
+        float* sAh = reinterpret_cast<float*>(sm + OFF_AHI);
+        float* sAl = reinterpret_cast<float*>(sm + OFF_ALO);
+        for (int e = tid - 64; e < R * C; e += 2 * GT) {
+          const int core = e >> 5, w = e & 31;
+          const int r = (core % (R / 8)) * 8 + (w >> 2);
+          const int cg = centre_of_group(p, r >> 5);
+          const bool valid = cg >= 0 && r - 32 * p.grp[cg] < p.n[cg];
+          const float x = valid ? sX[e] : 0.f;
+          const float hi = tf32_rna(x);
+          sAh[e] = hi;
+          sAl[e] = tf32_rna(x - hi);
+        }
+      }
+      fence_proxy_async();
+      mbar_arrive(&mt.bar_xfree);
+      mbar_arrive(&mt.bar_a);
+      const int cw = centre_of_group(p, quad);   // this warp's centre (-1: none)
+      const int nrow = cw >= 0 ? p.n[cw] : 0;
+      const bool vrow = cw >= 0 && row - 32 * p.grp[cw] < nrow;
+      if (!wproj.wait(&mt.bar_proj)) { ok = false; break; }
+      tc_fence_after();
+      if (grp == 0) {
+        // ---- Q: scaled by s_a log2(e)/sqrt(d), split, back into TMEM (hi over
+        // the raw q columns, lo at T_QLO); K: scaled by s_b, split, K-major B operand
+        const float sw = vrow ? (float)a.sw[p.row0[cw] + (row - 32 * p.grp[cw])] : 0.f;
+        uint32_t v[16], hv[16], lv[16];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          tmem_ld16(tmem + lane_addr + T_PROJ + 16u * part, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float x = __uint_as_float(v[j]) * (sw * qscale);
+            const float hi = tf32_rna(x);
+            hv[j] = __float_as_uint(hi);
+            lv[j] = __float_as_uint(tf32_rna(x - hi));
+          }
+          tmem_st16(tmem + lane_addr + T_PROJ + 16u * part, hv);
+          tmem_st16(tmem + lane_addr + T_QLO + 16u * part, lv);
+        }
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          tmem_ld16(tmem + lane_addr + T_PROJ + 32u + 16u * part, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int h = 2 * part + hh;
+            float4 kh[2], kl[2];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float x = __uint_as_float(v[8 * hh + j]) * sw;
+              const float hi = tf32_rna(x);
+              reinterpret_cast<float*>(kh)[j] = hi;
+              reinterpret_cast<float*>(kl)[j] = tf32_rna(x - hi);
+            }
+            unsigned char* kb = sm + OFF_K + (size_t)(2 * h) * K_BYTES;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              const uint32_t off = kmajor_offset(row, 4 * ch, R);
+              *reinterpret_cast<float4*>(kb + off) = kh[ch];
+              *reinterpret_cast<float4*>(kb + K_BYTES + off) = kl[ch];
+            }
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(&mt.bar_qk);
+      } else {
+        // ---- V^T: split, B operand [16 x keys] (rows 0-7 hi, 8-15 lo)
+        uint32_t v[16];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          tmem_ld16(tmem + lane_addr + T_PROJ + 64u + 16u * part, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int h = 2 * part + hh;
+            unsigned char* vb = sm + OFF_V + (size_t)(2 * h) * V_BYTES;
+            const uint32_t base = (uint32_t)(row >> 2) * VLBO + (uint32_t)(row & 3) * 4;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float x = __uint_as_float(v[8 * hh + j]);
+              const float hi = tf32_rna(x);
+              *reinterpret_cast<float*>(vb + base + 16u * j) = hi;
+              *reinterpret_cast<float*>(vb + V_BYTES + base + 16u * j) = tf32_rna(x - hi);
+            }
+          }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(&mt.bar_v);
+      }
+      // ---- softmax of this group's heads (buffer b = grp)
+      const int b = grp;
+      for (int hi2 = 0; hi2 < 2 && ok; ++hi2) {
+        if (!ws[b].wait(&mt.bar_s[b])) { ok = false; break; }
+        if (hi2 == 1 && !wpv[b].wait(&mt.bar_pv[b])) { ok = false; break; }  // in step
+        tc_fence_after();
+        float sv[MAXN];
+        const int nn = (nrow + 15) & ~15;
+        if (cw >= 0) {
+          uint32_t v[16];
+#pragma unroll
+          for (int q = 0; q < MAXN / 16; ++q) {
+            if (16 * q < nn) {
+              tmem_ld16(tmem + lane_addr + T_SP + 128u * b + 64u * cw + 16u * q, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) sv[16 * q + j] = __uint_as_float(v[j]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) sv[16 * q + j] = -INFINITY;
+            }
+          }
+          float mx = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < MAXN; ++j) {
+            if (j >= nrow) sv[j] = -INFINITY;
+            mx = fmaxf(mx, sv[j]);
+          }
+          // slot-occupancy softmax: phi phantom slots of logit 0 and value 0
+          const int phi = a.smooth ? a.nnei_max - nrow : 0;
+          if (phi > 0) mx = fmaxf(mx, 0.f);
+          if (!vrow) mx = 0.f;
+          float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+          for (int j = 0; j < MAXN; j += 4) {
+            sv[j] = ex2(sv[j] - mx);
+            sv[j + 1] = ex2(sv[j + 1] - mx);
+            sv[j + 2] = ex2(sv[j + 2] - mx);
+            sv[j + 3] = ex2(sv[j + 3] - mx);
+            l0 += sv[j];
+            l1 += sv[j + 1];
+            l2 += sv[j + 2];
+            l3 += sv[j + 3];
+          }
+          const float l = (l0 + l1) + (l2 + l3) + (phi > 0 ? (float)phi * ex2(-mx) : 0.f);
+          rinv[hi2] = vrow ? 1.f / l : 0.f;
+#pragma unroll
+          for (int q = 0; q < MAXN / 16; ++q) {
+            if (16 * q < nn) {
+              uint32_t ph[16], pl[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float pj = vrow ? sv[16 * q + j] : 0.f;
+                const uint32_t hb = __float_as_uint(pj) & 0xFFFFE000u;
+                ph[j] = hb;
+                pl[j] = __float_as_uint(pj - __uint_as_float(hb));
+              }
+              tmem_st16(tmem + lane_addr + T_SP + 128u * b + 16u * q, ph);
+              tmem_st16(tmem + lane_addr + T_SP + 128u * b + 64u + 16u * q, pl);
+            }
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(&mt.bar_p[b]);
+      }
+      if (!ok) break;
+      // ---- epilogue: wait for the P V of this group's second head
+      if (!wpv[b].wait(&mt.bar_pv[b])) { ok = false; break; }
+      tc_fence_after();
+      if (grp == 0 && gt == 0) bulk_wait_read_all();  // the staging buffer is free
+      // both groups must have seen the staging free: group 0 thread 0 waits first
+      // (its bulk copies are the only readers), then every thread of both groups
+      // arrives, and the writes follow the barrier
+      mbar_arrive(&mt.bar_epi);
+      if (!wepi.wait(&mt.bar_epi)) { ok = false; break; }
+      if (cw >= 0) {
+        float* so = reinterpret_cast<float*>(sm + OFF_OUT);
+        uint32_t v[16];
+#pragma unroll
+        for (int hi2 = 0; hi2 < 2; ++hi2) {
+          const int h = grp + 2 * hi2;
+          tmem_ld16(tmem + lane_addr + T_O + 16u * (2 * h + cw), v);
+          tmem_wait_ld();
+          float4 o[2];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            reinterpret_cast<float*>(o)[j] =
+                (__uint_as_float(v[j]) + __uint_as_float(v[8 + j])) * rinv[hi2];
+          if (vrow) {
+            *reinterpret_cast<float4*>(so + row * C + h * D) = o[0];
+            *reinterpret_cast<float4*>(so + row * C + h * D + 4) = o[1];
+          }
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(&mt.bar_epi);
+      if (!wepi.wait(&mt.bar_epi)) { ok = false; break; }
+      if (grp == 0 && gt == 0) {
+        float* out = static_cast<float*>(a.out);
+        const float* so = reinterpret_cast<const float*>(sm + OFF_OUT);
+        for (int c = 0; c < p.ncent; ++c)
+          bulk_s2g(out + p.row0[c] * C, so + 32 * p.grp[c] * C, (uint32_t)(p.n[c] * C * 4));
+        bulk_commit();
+      }
+    }
+    if (grp == 0 && gt == 0) bulk_wait_all();
+    if (!ok) mt.fail = 1;
+  }
+  // ---- teardown: report, let a slab copy in flight land, free TMEM
+  __syncthreads();
+  if (tid == 0 && mt.fail) atomicOr(a.status, kStatusTimeout);
+  if (warp == 1 && lane == 0 && mt.fail && mt.last_slot >= 0)
+    mbar_wait(&mt.bar_xfull[mt.last_slot], mt.last_par);  // a slab copy may still land
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+}  // namespace mlg

@@ -33,6 +33,8 @@ struct TileArgs {
   int64_t capacity;
   int n_layers;  // 1 .. kMaxFusedLayers
   int nnei_max;  // centres with more edges are skipped and flagged (MLG_STATUS_ROW_TOO_LONG)
+  int min_n;     // centres with at most min_n edges are left to another kernel (0: none)
+  int smooth;    // slot-occupancy softmax: nnei_max - n phantom slots of logit 0, value 0
   const void* G;
   void* out;
   const void* W[3 * kMaxFusedLayers];  // q, k, v of each layer: device [C][C]
@@ -201,9 +203,13 @@ __device__ __forceinline__ void softmax_block(const T* q, T* o, T& mx, T& l, con
 // Warp tasks: 32 consecutive (head, row) pairs of one centre; lanes of a warp
 // walk the keys in lock-step, so k_b and v_b are broadcast reads.  The output
 // of (row, h) overwrites the q slot that only its own lane read.
+// With smooth_nnei > 0 (the slot-occupancy softmax, NeighborGraph issue,
+// Numerics note) a centre of n edges also has phi = smooth_nnei - n phantom
+// slots of logit 0 and value 0; they enter the running softmax as a first
+// block: maximum 0, sum phi, output 0.
 template <typename T, int HEADS, int D, int KOFF, int NT, int QS>
 __device__ __forceinline__ void tile_attention(T* sQ, const TileMeta& meta, int buf, int warp,
-                                               int lane) {
+                                               int lane, int smooth_nnei = 0) {
   const int ncent = meta.ncent[buf];
   const int ntask = meta.task0[buf][ncent];
   for (int task = warp; task < ntask; task += NT / 32) {
@@ -223,6 +229,10 @@ __device__ __forceinline__ void tile_attention(T* sQ, const TileMeta& meta, int 
       o[t] = T(0);
     }
     T mx = T(-INFINITY), l = T(0);
+    if (smooth_nnei > n) {
+      mx = T(0);
+      l = T(smooth_nnei - n);
+    }
     const T* kb = sQ + base * QS + KOFF + h * D;
     const T* vb = sQ + base * QS + 2 * KOFF + h * D;
     const int nfull = n & ~7;

@@ -99,6 +99,10 @@ _lib.mlg_attention_stack.restype = ctypes.c_int
 _lib.mlg_attention_stack.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32, _c_i32,
                                      _c_i32, ctypes.c_int, ctypes.POINTER(_p), _p, _p, _p, _c_sz,
                                      _p]
+_lib.mlg_attention_stack_smooth.restype = ctypes.c_int
+_lib.mlg_attention_stack_smooth.argtypes = [ctypes.POINTER(mlg_csr), _c_i64, _c_i32, _c_i32,
+                                            _c_i32, _c_i32, ctypes.c_int, ctypes.POINTER(_p), _p,
+                                            _p, _p, _c_sz, _p]
 _lib.mlg_build_csr_batch_workspace_bytes.restype = _c_sz
 _lib.mlg_build_csr_batch_workspace_bytes.argtypes = [ctypes.POINTER(mlg_system), _c_i32, _c_dbl]
 _lib.mlg_build_csr_batch.restype = ctypes.c_int
@@ -273,6 +277,22 @@ def mlg_attention_stack(csr: Csr, n_centres: int, nnei_max: int, channels: int, 
                                     _ptr(G_in), _ptr(G_out), _ptr(ws), nbytes,
                                     _stream_handle(stream))
     return _check(code, "mlg_attention_stack", check)
+
+
+def mlg_attention_stack_smooth(csr: Csr, n_centres: int, nnei_max: int, channels: int,
+                               heads: int, n_layers: int, dtype: int, W, G_in, G_out, ws=None,
+                               ws_bytes: int | None = None, stream=None,
+                               check: bool = True) -> int:
+    """``mlg_attention_stack`` with the slot-occupancy softmax in every layer."""
+    ptrs = (_p * len(W))(*[_ptr(w) for w in W])
+    c = csr.struct()
+    nbytes = 0 if ws is None else (int(ws.numel() * ws.element_size()) if ws_bytes is None
+                                   else int(ws_bytes))
+    code = _lib.mlg_attention_stack_smooth(ctypes.byref(c), int(n_centres), int(nnei_max),
+                                           int(channels), int(heads), int(n_layers),
+                                           int(dtype), ptrs, _ptr(G_in), _ptr(G_out), _ptr(ws),
+                                           nbytes, _stream_handle(stream))
+    return _check(code, "mlg_attention_stack_smooth", check)
 
 
 def _check(code: int, where: str, check: bool):

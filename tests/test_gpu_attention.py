@@ -166,6 +166,10 @@ def _random_graph(n_atoms, density, rcut, nnei_max, seed):
     ("f64", 32, 4, 2, 0.2, 96),    # ~62 edges: fused tile (<= 64) + generic for larger rows
     ("f32", 64, 4, 1, 0.41, 181),  # ~128 edges: fused tile (<= 128) + generic for larger
     ("f32", 32, 4, 2, 0.004, 128), # dilute: many centres without edges between full ones
+    ("f32", 32, 4, 1, 0.13, 64),   # one layer, ragged rows <= 64: every product on tcgen05
+    ("f32", 32, 4, 1, 0.2, 128),   # ~62 edges: tcgen05 tiles (<= 64) + FP32-pipe tile (<= 128)
+    ("f32", 32, 4, 1, 0.41, 181),  # ~128 edges: both tile kernels + generic for larger rows
+    ("f32", 32, 4, 1, 0.004, 64),  # dilute, one layer: centres without edges between
     ("f64", 128, 4, 2, 0.3, 96),   # head-group kernel, two layers (ping-pong)
     ("f32", 128, 8, 2, 0.31, 181), # head-group kernel (<= 96 edges) + generic for larger
 ])
@@ -196,13 +200,62 @@ def test_stack_mixed_row_sizes(dtype, channels, heads, n_layers, density, nnei):
     outs = oracle.forward(gpu["row_ptr"], gpu["sw"], G, W, heads, dtype)
     ok, err = U.attn_tolerance_ok(w, gout[:e].cpu().numpy(), outs[-1])
     assert ok, (err, counts.min(), counts.max())
-    if (density, nnei) in ((0.2, 96), (0.41, 181), (0.31, 181)):  # both sides of the tile limit
-        limit = {0.2: 64, 0.41: 128, 0.31: 96}[density]
+    if (density, nnei) in ((0.2, 96), (0.41, 181), (0.31, 181), (0.2, 128)):
+        # both sides of a tile limit
+        limit = {(0.2, 96): 64, (0.41, 181): 128, (0.31, 181): 96, (0.2, 128): 64}[
+            (density, nnei)]
         assert counts.min() <= limit < counts.max()
     if (density, nnei) == (0.13, 40):    # query blocks end in every position of a 16-row block
         assert set(range(16)) <= set(int(c) % 16 for c in counts if c > 0)
     # rows past E are never written
     assert bool((gout[e:] == 0).all())
+
+
+@pytest.mark.parametrize("dtype,channels,heads,n_layers,density,nnei", [
+    ("f32", 32, 4, 1, 0.13, 64),   # every product on tcgen05
+    ("f32", 32, 4, 1, 0.2, 128),   # tcgen05 tiles (<= 64) + FP32-pipe tile (<= 128)
+    ("f32", 32, 4, 2, 0.2, 96),    # two fused layers on the FP32-pipe tile
+    ("f32", 64, 4, 1, 0.41, 181),  # fused tile (<= 128) + generic for larger rows
+    ("f32", 128, 8, 2, 0.31, 181), # head-group kernel (<= 96) + generic, two layers
+    ("f64", 128, 4, 2, 0.3, 96),   # head-group kernel, fp64, two layers
+    ("f64", 32, 4, 2, 0.13, 64),   # fp64, 32 channels: the generic kernel
+])
+def test_smooth_stack_matches_oracle(dtype, channels, heads, n_layers, density, nnei):
+    """The slot-occupancy softmax in the fused kernels and through the layer
+    stack (mlg_attention_stack_smooth) against the oracle's smooth attention
+    chained layer by layer (fp32 layers rounded to fp32 between layers, as the
+    fp32 path stores them)."""
+    import oracle
+    from neighbour_graph_attention_b200.configs import Workload
+
+    m = U.mlg()
+    gpu, csr_t = _random_graph(3000, density, 4.2, nnei, 19)
+    e = gpu["n_edges"]
+    rp = gpu["row_ptr"]
+    w = Workload(0, "random", "random", 0, 0, 0, 3000, 4.2, 3.7, nnei, channels, heads, n_layers,
+                 dtype)
+    rng = np.random.default_rng(8)
+    W = rng.normal(0, 1 / np.sqrt(channels), (n_layers, 3, channels, channels)).astype(w.np_dtype)
+    G = rng.normal(0, 1, (e, channels)).astype(w.np_dtype)
+    dt = U.torch_dtype(w)
+    g0 = torch.as_tensor(G, device="cuda")
+    gout = torch.zeros_like(g0)
+    Wt = [torch.as_tensor(W[l][k], device="cuda") for l in range(n_layers) for k in range(3)]
+    ws = m.workspace(m.mlg_attention_stack_workspace_bytes(csr_t.capacity, channels, n_layers,
+                                                           U.mlg_dtype(w)))
+    m.mlg_attention_stack_smooth(csr_t, 3000, nnei, channels, heads, n_layers, U.mlg_dtype(w),
+                                 Wt, g0, gout, ws)
+    torch.cuda.synchronize()
+    assert int(csr_t.status.item()) == 0
+    sw = gpu["sw"] if dtype == "f64" else gpu["sw"].astype(np.float32).astype(np.float64)
+    ref = G.astype(np.float64)
+    for l in range(n_layers):
+        ref = oracle.attention_smooth(rp, sw, ref, W[l][0], W[l][1], W[l][2], heads, nnei)
+        if dtype == "f32":
+            ref = ref.astype(np.float32).astype(np.float64)
+    ok, err = U.attn_tolerance_ok(w, gout.cpu().numpy(), ref)
+    assert ok, err
+    assert (np.diff(rp) < nnei).any()  # phantoms take part
 
 
 def test_peaked_softmax_f64():
@@ -300,6 +353,34 @@ def test_nan_feature_confined_to_its_centre():
     o6 = gout[:e].cpu().numpy()
     assert np.isnan(o6[bad]).all() and np.isfinite(o6[~bad]).all()
     ok, err = U.attn_tolerance_ok(w, o6[~bad], outs[-1][~bad])
+    assert ok, err
+
+
+def test_nan_feature_confined_to_its_centre_f32_tensor_core_tiles():
+    """fp32, 32 channels, one layer (every product on tcgen05, two centres per
+    tile): a NaN in one edge feature reaches every row of its centre and no
+    row of any other centre, including the other centre of its tile."""
+    import oracle
+    from neighbour_graph_attention_b200.configs import Workload
+
+    gpu, csr_t = _random_graph(3000, 0.13, 4.2, 64, 17)
+    rp = gpu["row_ptr"]
+    e = gpu["n_edges"]
+    w = Workload(0, "random", "random", 0, 0, 0, 3000, 4.2, 3.7, 64, 32, 4, 1, "f32")
+    rng = np.random.default_rng(31)
+    W = [rng.normal(0, 1 / np.sqrt(32), (32, 32)).astype(np.float32) for _ in range(3)]
+    G = rng.normal(size=(e, 32)).astype(np.float32)
+    for i in (5, 6, 1200):   # neighbours in one tile, and a centre elsewhere
+        if rp[i + 1] > rp[i]:
+            G[int(rp[i]), 3] = np.nan
+    bad = np.zeros(e, dtype=bool)
+    for i in (5, 6, 1200):
+        bad[int(rp[i]):int(rp[i + 1])] = rp[i + 1] > rp[i]
+    out = U.gpu_attention(csr_t, 3000, w, G, *W)
+    sw = gpu["sw"].astype(np.float32).astype(np.float64)
+    ref = oracle.attention(rp, sw, G, *W, 4)
+    assert np.isnan(out[bad]).all() and np.isfinite(out[~bad]).all()
+    ok, err = U.attn_tolerance_ok(w, out[~bad], ref[~bad])
     assert ok, err
 
 

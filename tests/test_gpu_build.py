@@ -42,6 +42,38 @@ def test_csr_bit_exact(key, seed):
     U.assert_csr_equal(gpu, ref)
 
 
+def _digests():
+    import json
+    import os
+
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "csr_digests.json")
+    with open(path) as f:
+        return json.load(f)["graphs"]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("key", [3, 5])
+def test_csr_full_size_digests(key, seed):
+    """Every array of the full-size Fe BCC graphs (65,536 and 524,288 atoms),
+    edge for edge: SHA-256 of the device CSR against digests of the oracle's
+    brute-force CSR, written by tests/golden/make_csr_digests.py (which calls
+    only the oracle)."""
+    import hashlib
+
+    rec = _digests()[f"{key}:{seed}"]
+    w = C.workload(key)
+    s = C.system(key, seed)
+    assert (rec["n_atoms"], rec["rcut"], rec["nnei_max"]) == (w.n_atoms, w.rcut, w.nnei_max)
+    gpu, _ = U.gpu_build(s["coords"], s["box"], s["pbc"], w.rcut, w.r_on, w.nnei_max,
+                         s["types"], s["n_types"])
+    assert gpu["status"] == 0
+    assert gpu["n_edges"] == rec["n_edges"] and gpu["n_truncated"] == rec["n_truncated"]
+    for k, dt in (("row_ptr", np.int64), ("src", np.int32), ("shift", np.int32),
+                  ("vec", np.float64), ("dist", np.float64), ("sw", np.float64)):
+        a = np.ascontiguousarray(gpu[k], dtype=dt)
+        assert hashlib.sha256(a.tobytes()).hexdigest() == rec["sha256"][k], k
+
+
 def test_largest_system_sampled_and_properties():
     import oracle
 

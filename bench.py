@@ -42,6 +42,8 @@ FALLBACK_HBM_GBS = 6650.0
 SM_COUNT, SM_MAX_GHZ = 148, 1.965
 FP64_PEAK_TFLOPS = SM_COUNT * 64 * 2 * SM_MAX_GHZ / 1e3
 FP32_PEAK_TFLOPS = SM_COUNT * 128 * 2 * SM_MAX_GHZ / 1e3
+# Special-function unit (ex2): 16 per SM per clock.
+SFU_PEAK_TEXP = SM_COUNT * 16 * SM_MAX_GHZ / 1e3
 
 # Attention kernel of each workload and its DRAM traffic per launch
 # (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture of that
@@ -52,8 +54,20 @@ ATTN_KERNEL = {
     2: ("k_attn_dmma<160,5,640>", 5.622e6),   # profiles/k_attn_dmma_f64_diamond512.md
     3: ("k_attn_tc<64,16,512>", None),
     4: ("k_attn_hg<float,128,16,...>", None),
-    5: ("k_attn_tc<32,8,512>", None),
+    5: ("k_attn_tc2 (logits and P.V on tcgen05; k_attn_tc<32,8,512> for rows over 64)", None),
 }
+
+
+def tensor_core_path(w) -> bool:
+    """fp32, 32 channels, 4 heads, one layer: every product on tcgen05, so the
+    softmax's exponentials (special-function unit) bound the kernel, not FMAs."""
+    return w.dtype == "f32" and w.channels == 32 and w.heads == 4 and w.n_layers == 1
+
+
+def attention_exps(row_ptr, heads):
+    """Per layer: one exponential per logit, sum_i n_i^2 * heads."""
+    n = np.diff(np.asarray(row_ptr)).astype(np.float64)
+    return float(np.sum(n * n)) * heads
 
 
 def parse_args(argv=None):
@@ -456,13 +470,27 @@ def main(argv=None):
     kname, traffic = ATTN_KERNEL.get(w.key, ("attention stack", None))
     if args.cells is not None:   # a resized system: the stored capture does not apply
         traffic = None
-    roofline = {"bound": "alu", "achieved": achieved_tf, "peak": peak_fp, "unit": "TFLOP/s",
-                "frac": achieved_tf / peak_fp, "traffic": traffic,
-                "kernel": "%s (all %d layer(s) in one launch)" % (kname, w.n_layers),
-                "algorithmic_flops_per_launch": flops,
-                "peak_basis": ("derived: 148 SMs x %d %s FMA/clk x 2 x 1.965 GHz" %
-                               (64 if w.dtype == "f64" else 128, w.dtype.upper())),
-                "hbm_frac_of_" + hbm_src: abytes / (attn_avg * 1e-3) / 1e9 / hbm_peak}
+    if tensor_core_path(w):
+        # products on the tensor cores: the exponentials bound the kernel
+        # (special-function unit), ahead of HBM and of the tensor pipe
+        exps = attention_exps(row_ptr, w.heads) * w.n_layers
+        achieved_ex = exps / (attn_avg * 1e-3) / 1e12
+        roofline = {"bound": "alu", "achieved": achieved_ex, "peak": SFU_PEAK_TEXP,
+                    "unit": "Texp/s", "frac": achieved_ex / SFU_PEAK_TEXP, "traffic": traffic,
+                    "kernel": kname, "algorithmic_exps_per_launch": exps,
+                    "algorithmic_flops_per_launch": flops, "achieved_tflops": achieved_tf,
+                    "peak_basis": "derived: 148 SMs x 16 ex2/clk x 1.965 GHz (special-function "
+                                  "unit; the exponentials' floor exceeds the HBM and "
+                                  "tensor-pipe floors)",
+                    "hbm_frac_of_" + hbm_src: abytes / (attn_avg * 1e-3) / 1e9 / hbm_peak}
+    else:
+        roofline = {"bound": "alu", "achieved": achieved_tf, "peak": peak_fp,
+                    "unit": "TFLOP/s", "frac": achieved_tf / peak_fp, "traffic": traffic,
+                    "kernel": "%s (all %d layer(s) in one launch)" % (kname, w.n_layers),
+                    "algorithmic_flops_per_launch": flops,
+                    "peak_basis": ("derived: 148 SMs x %d %s FMA/clk x 2 x 1.965 GHz" %
+                                   (64 if w.dtype == "f64" else 128, w.dtype.upper())),
+                    "hbm_frac_of_" + hbm_src: abytes / (attn_avg * 1e-3) / 1e9 / hbm_peak}
     build_gbs = bbytes / (build_avg * 1e-3) / 1e9
     roofline_build = {"bound": "hbm", "achieved": build_gbs, "peak": hbm_peak, "unit": "GB/s",
                       "frac": build_gbs / hbm_peak, "peak_source": hbm_src,

@@ -17,6 +17,7 @@
 #include "mlg_attn_dmma.cuh"
 #include "mlg_attn_tc.cuh"
 #include "mlg_attn_tc2.cuh"
+#include "mlg_attn_hgtc.cuh"
 #include "mlg_local.cuh"
 #include "mlg_verlet.cuh"
 
@@ -705,15 +706,41 @@ int launch_hg(HgArgs& ha, cudaStream_t stream) {
 
 int hg_rows(mlg_dtype dtype, int C, int D) {
   if (dtype == MLG_F64 && C == 128 && D == 32) return 128;
-  if (dtype == MLG_F32 && C == 128 && D == 16) return 96;
+  if (dtype == MLG_F32 && C == 128 && D == 16) return hgtc::R;
   return 0;
+}
+
+// fp32, 128 channels, heads of 16: the projection on tcgen05, grid (centre
+// ranges x 4 head groups), one CTA per SM.
+int launch_hgtc(const HgArgs& ha, cudaStream_t stream) {
+  auto kern = k_attn_hgtc;
+  prefer_shared(kern, hgtc::SMEM);
+  if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
+  CUtensorMap map;
+  if (!encode_slab_map(&map, ha.G, ha.capacity, hgtc::C, 128)) return MLG_ERR_CUDA;
+  HgtcArgs a;
+  a.row_ptr = ha.row_ptr;
+  a.sw = ha.sw;
+  a.n_centres = ha.n_centres;
+  a.capacity = ha.capacity;
+  a.nnei_max = ha.nnei_max;
+  a.smooth = ha.smooth;
+  a.out = ha.out;
+  a.Wq = ha.Wq;
+  a.Wk = ha.Wk;
+  a.Wv = ha.Wv;
+  a.status = ha.status;
+  int64_t gx = ((int64_t)sm_count() + hgtc::NG - 1) / hgtc::NG;
+  if (gx > ha.n_centres) gx = ha.n_centres;
+  if (gx < 1) gx = 1;
+  kern<<<dim3((unsigned)gx, hgtc::NG), hgtc::NT, hgtc::SMEM, stream>>>(a, map);
+  return launch_status();
 }
 
 int launch_hg_shape(mlg_dtype dtype, int C, int D, HgArgs& ha, cudaStream_t s) {
   if (dtype == MLG_F64 && C == 128 && D == 32)
     return launch_hg<double, 128, 32, 1, 128, 256, 8, 6, 16>(ha, s);
-  if (dtype == MLG_F32 && C == 128 && D == 16)
-    return launch_hg<float, 128, 16, 2, 96, 256, 6, 6, 16>(ha, s);
+  if (dtype == MLG_F32 && C == 128 && D == 16) return launch_hgtc(ha, s);
   return MLG_ERR_UNSUPPORTED;
 }
 

@@ -26,7 +26,8 @@ def graph(key, seed):
     return gpu, csr_t
 
 
-@pytest.mark.parametrize("key,seed", [(1, 0), (1, 1), (2, 0), (2, 2), (3, 0), (4, 0), (4, 1)])
+@pytest.mark.parametrize("key,seed", [(1, 0), (1, 1), (2, 0), (2, 2), (3, 0), (3, 1), (3, 2),
+                                      (4, 0), (4, 1), (5, 1), (5, 2)])
 def test_one_layer_matches_oracle(key, seed):
     import oracle
 
@@ -80,7 +81,7 @@ def test_sum_to_one_through_gpu(key):
     assert np.max(np.abs(out.astype(np.float64) - 1.0)) <= tol
 
 
-@pytest.mark.parametrize("key", [2, 4])
+@pytest.mark.parametrize("key", [2, 3, 4, 5])
 def test_forward_matches_oracle(key):
     import oracle
 

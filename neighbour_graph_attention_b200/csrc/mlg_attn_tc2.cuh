@@ -15,9 +15,10 @@
 // Tiles of 128 rows hold up to two centres, each starting at a multiple of
 // 32 rows, so that every warp's TMEM lane quadrant belongs to one centre.
 //   projection  D[128 x 96] = X[128 x 32] . [Wq|Wk|Wv], 3xTF32 (12 MMAs)
-//   Q           read back, scaled, split into TF32 hi/lo and stored back
-//               into TMEM: the A operand of the logits (A from TMEM)
-//   K, V^T      read back, split, stored as shared-memory B operands
+//   Q, K, V^T   read back, scaled, split into TF32 hi/lo and stored as
+//               shared-memory operands; the projection's TMEM is then free,
+//               and the next tile's projection runs during this tile's
+//               softmax (its slab is split right after this read-back)
 //   logits      per (head, centre): S = Q_h . K_h^T over the centre's keys,
 //               M = 128 (only the centre's rows are used), N = ceil16(n), 3 MMAs
 //   softmax     one thread per row: its S row from TMEM, max, 2^(S - max),
@@ -41,6 +42,8 @@
 //              layout; the next slab lands while the current tile computes
 //   warps 2-5  group 0: split, Q and K, softmax of heads 0 and 2, epilogue
 //   warps 6-9  group 1: split, V, softmax of heads 1 and 3, epilogue
+// Per tile: read-back of the projection, split of the next slab (whose
+// projection the MMA thread then issues), softmax, epilogue.
 // A warp w reads TMEM lanes 32 (w % 4) .. +31, i.e. tile rows of one
 // quadrant.  Every wait is bounded; on expiry the kernel records
 // MLG_STATUS_TIMEOUT, every role leaves its loop, and the CTA lets its
@@ -64,8 +67,7 @@ constexpr int GT = 128;         // threads per compute group
 constexpr int VLBO = 144;       // V^T operand: bytes between 4-key chunks (bank spread)
 
 // TMEM columns (512 allocated)
-constexpr uint32_t T_PROJ = 0;    // projection D: q 0-31, k 32-63, v 64-95; Q lo at 96-127
-constexpr uint32_t T_QLO = 96;
+constexpr uint32_t T_PROJ = 0;    // projection D: q 0-31, k 32-63, v 64-95 (128 allocated)
 constexpr uint32_t T_O = 128;     // O of (head h, centre c): T_O + (2 h + c) * 16
 constexpr uint32_t T_SP = 256;    // S / P buffer b: T_SP + 128 b (S of centre c at +64 c;
                                   // P hi at +0, P lo at +64)
@@ -80,7 +82,8 @@ constexpr size_t OFF_WLO = OFF_WHI + W_BYTES;
 constexpr size_t OFF_X = OFF_WLO + W_BYTES;             // raw slab (TMA target)
 constexpr size_t OFF_AHI = OFF_X + A_BYTES;
 constexpr size_t OFF_ALO = OFF_AHI + A_BYTES;
-constexpr size_t OFF_K = OFF_ALO + A_BYTES;             // [head][hi, lo]
+constexpr size_t OFF_Q = OFF_ALO + A_BYTES;             // [head][hi, lo], as K
+constexpr size_t OFF_K = OFF_Q + 2 * H * K_BYTES;       // [head][hi, lo]
 constexpr size_t OFF_V = OFF_K + 2 * H * K_BYTES;       // [head][hi, lo]
 constexpr size_t OFF_OUT = OFF_V + 2 * H * V_BYTES;     // [128][32] row-major staging
 constexpr size_t OFF_META = OFF_OUT + A_BYTES;
@@ -101,9 +104,9 @@ struct Meta {
   uint64_t bar_xfull[2];    // slab and plan of ring slot landed (TMA tx)
   uint64_t bar_xfree;       // the groups have split the slab (count 2 * GT)
   uint64_t bar_w;           // weights split (count 2 * GT)
-  uint64_t bar_a;           // A operands split (count 2 * GT)
+  uint64_t bar_a;           // A operands of a tile split, or no tile left (count 2 * GT)
   uint64_t bar_proj;        // projection done (commit)
-  uint64_t bar_qk;          // Q in TMEM, K in shared memory (count GT)
+  uint64_t bar_qk;          // Q and K in shared memory (count GT)
   uint64_t bar_v;           // V^T in shared memory (count GT)
   uint64_t bar_s[2];        // logits of buffer b done (commit)
   uint64_t bar_p[2];        // P of buffer b written (count GT)
@@ -275,56 +278,69 @@ __global__ void __launch_bounds__(tc2::NT, 1)
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       Waiter wa, wqk, wv, wp[2], wpv[2], ww;
-      bool ok = ww.wait(&mt.bar_w);
-      for (int t = 0; ok; ++t) {
-        if (!wa.wait(&mt.bar_a)) { ok = false; break; }
-        const Plan p = mt.plan[t & 1];
-        if (p.ncent == 0) break;
-        if (t > 0) {
-          // the last two P V of the previous tile (heads 2 and 3) have read
-          // their P and Q before the projection rewrites that TMEM
-          if (!wpv[0].wait(&mt.bar_pv[0]) || !wpv[1].wait(&mt.bar_pv[1])) { ok = false; break; }
-        }
-        tc_fence_after();
-        // projection: D[128 x 96] = X . W, 3xTF32, small terms first
-        {
-          const uint32_t ahi = smem_u32(sm + OFF_AHI), alo = smem_u32(sm + OFF_ALO);
-          const uint32_t bhi = smem_u32(sm + OFF_WHI), blo = smem_u32(sm + OFF_WLO);
-          const uint32_t id = idesc_tf32(R, N3);
+      const uint32_t qhi0 = smem_u32(sm + OFF_Q);
+      // projection of the tile whose A operands are split: D[128 x 96] = X . W,
+      // 3xTF32, small terms first
+      auto issue_proj = [&]() {
+        const uint32_t ahi = smem_u32(sm + OFF_AHI), alo = smem_u32(sm + OFF_ALO);
+        const uint32_t bhi = smem_u32(sm + OFF_WHI), blo = smem_u32(sm + OFF_WLO);
+        const uint32_t id = idesc_tf32(R, N3);
 #pragma unroll
-          for (int s = 0; s < C / 8; ++s) {
-            const uint32_t aoff = (uint32_t)(s * R * 32), boff = (uint32_t)(s * N3 * 32);
-            const uint64_t dah = umma_sdesc(ahi + aoff, R * 16, 128);
-            const uint64_t dal = umma_sdesc(alo + aoff, R * 16, 128);
-            const uint64_t dbh = umma_sdesc(bhi + boff, N3 * 16, 128);
-            const uint64_t dbl = umma_sdesc(blo + boff, N3 * 16, 128);
-            umma_tf32(tmem + T_PROJ, dal, dbh, id, s > 0 ? 1u : 0u);
-            umma_tf32(tmem + T_PROJ, dah, dbl, id, 1u);
-            umma_tf32(tmem + T_PROJ, dah, dbh, id, 1u);
-          }
-          umma_commit(&mt.bar_proj);
+        for (int s = 0; s < C / 8; ++s) {
+          const uint32_t aoff = (uint32_t)(s * R * 32), boff = (uint32_t)(s * N3 * 32);
+          const uint64_t dah = umma_sdesc(ahi + aoff, R * 16, 128);
+          const uint64_t dal = umma_sdesc(alo + aoff, R * 16, 128);
+          const uint64_t dbh = umma_sdesc(bhi + boff, N3 * 16, 128);
+          const uint64_t dbl = umma_sdesc(blo + boff, N3 * 16, 128);
+          umma_tf32(tmem + T_PROJ, dal, dbh, id, s > 0 ? 1u : 0u);
+          umma_tf32(tmem + T_PROJ, dah, dbl, id, 1u);
+          umma_tf32(tmem + T_PROJ, dah, dbh, id, 1u);
         }
-        // logits of head h into buffer b: per centre, 3 MMAs (A = Q from TMEM)
+        umma_commit(&mt.bar_proj);
+      };
+      bool ok = ww.wait(&mt.bar_w) && wa.wait(&mt.bar_a);
+      Plan p = mt.plan[0];
+      if (ok && p.ncent > 0) {
+        tc_fence_after();
+        issue_proj();
+      }
+      for (int t = 0; ok && p.ncent > 0; ++t) {
+        // logits of head h into buffer b: per centre, 3 MMAs (Q and K from shared memory)
         auto issue_s = [&](int h, int b) {
+          const uint32_t qhi = qhi0 + (uint32_t)(2 * h) * (uint32_t)K_BYTES;
+          const uint32_t qlo = qhi + (uint32_t)K_BYTES;
+          const uint64_t dqh = umma_sdesc(qhi, R * 16, 128);
+          const uint64_t dql = umma_sdesc(qlo, R * 16, 128);
           for (int c = 0; c < p.ncent; ++c) {
             const int nn = (p.n[c] + 15) & ~15;
             const uint32_t id = idesc_tf32(R, nn);
-            const uint32_t khi = smem_u32(sm + OFF_K + (size_t)(2 * h) * K_BYTES) + 512u * p.grp[c];
+            const uint32_t khi =
+                smem_u32(sm + OFF_K + (size_t)(2 * h) * K_BYTES) + 512u * p.grp[c];
             const uint32_t klo = khi + (uint32_t)K_BYTES;
             const uint64_t dkh = umma_sdesc(khi, R * 16, 128);
             const uint64_t dkl = umma_sdesc(klo, R * 16, 128);
             const uint32_t d = tmem + T_SP + 128u * b + 64u * c;
-            umma_tf32_ts(d, tmem + T_QLO + 8u * h, dkh, id, 0u);
-            umma_tf32_ts(d, tmem + T_PROJ + 8u * h, dkl, id, 1u);
-            umma_tf32_ts(d, tmem + T_PROJ + 8u * h, dkh, id, 1u);
+            umma_tf32(d, dql, dkh, id, 0u);
+            umma_tf32(d, dqh, dkl, id, 1u);
+            umma_tf32(d, dqh, dkh, id, 1u);
           }
           umma_commit(&mt.bar_s[b]);
         };
         if (!wqk.wait(&mt.bar_qk)) { ok = false; break; }
+        if (t > 0) {
+          // the last two P V of the previous tile have read their P buffers
+          if (!wpv[0].wait(&mt.bar_pv[0]) || !wpv[1].wait(&mt.bar_pv[1])) { ok = false; break; }
+        }
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 1);
         if (!wv.wait(&mt.bar_v)) { ok = false; break; }
+        // the groups have read the projection out of TMEM: the next tile's
+        // projection runs on the tensor cores during this tile's softmax
+        if (!wa.wait(&mt.bar_a)) { ok = false; break; }
+        const Plan pn = mt.plan[(t + 1) & 1];
+        tc_fence_after();
+        if (pn.ncent > 0) issue_proj();
         for (int h = 0; h < H && ok; ++h) {
           const int b = h & 1;
           if (!wp[b].wait(&mt.bar_p[b])) { ok = false; break; }
@@ -354,6 +370,7 @@ __global__ void __launch_bounds__(tc2::NT, 1)
             issue_s(h + 2, b);
           }
         }
+        p = pn;
       }
       if (!ok) mt.fail = 1;
       // every MMA issued here is complete before TMEM is freed
@@ -382,17 +399,12 @@ __global__ void __launch_bounds__(tc2::NT, 1)
     }
     fence_proxy_async();
     mbar_arrive(&mt.bar_w);
-    float rinv[2] = {0.f, 0.f};
-    for (int t = 0; ok; ++t) {
-      const int s = t & 1;
-      if (!wx[s].wait(&mt.bar_xfull[s])) { ok = false; break; }
-      const Plan p = mt.plan[s];
-      if (p.ncent == 0) {
-        mbar_arrive(&mt.bar_a);  // lets the MMA thread see the end
-        break;
-      }
-      // ---- split the slab into the A operands; rows outside the centres are 0
-      {
+    // the slab of ring slot s split into the A operands (rows outside the
+    // centres are 0); returns the slot's plan (ncent 0: no work left)
+    auto split = [&](int s, Plan& p) -> bool {
+      if (!wx[s].wait(&mt.bar_xfull[s])) return false;
+      p = mt.plan[s];
+      if (p.ncent > 0) {
         const float* sX = reinterpret_cast<const float*>(sm + OFF_X);
         float* sAh = reinterpret_cast<float*>(sm + OFF_AHI);
         float* sAl = reinterpret_cast<float*>(sm + OFF_ALO);
@@ -406,59 +418,52 @@ __global__ void __launch_bounds__(tc2::NT, 1)
           sAh[e] = hi;
           sAl[e] = tf32_rna(x - hi);
         }
+        fence_proxy_async();
+        mbar_arrive(&mt.bar_xfree);
       }
-      fence_proxy_async();
-      mbar_arrive(&mt.bar_xfree);
-      mbar_arrive(&mt.bar_a);
+      mbar_arrive(&mt.bar_a);  // also tells the MMA thread when no work is left
+      return true;
+    };
+    float rinv[2] = {0.f, 0.f};
+    Plan p;
+    ok = split(0, p);
+    for (int t = 0; ok && p.ncent > 0; ++t) {
       const int cw = centre_of_group(p, quad);   // this warp's centre (-1: none)
       const int nrow = cw >= 0 ? p.n[cw] : 0;
       const bool vrow = cw >= 0 && row - 32 * p.grp[cw] < nrow;
       if (!wproj.wait(&mt.bar_proj)) { ok = false; break; }
       tc_fence_after();
       if (grp == 0) {
-        // ---- Q: scaled by s_a log2(e)/sqrt(d), split, back into TMEM (hi over
-        // the raw q columns, lo at T_QLO); K: scaled by s_b, split, K-major B operand
+        // ---- Q (scaled by s_a log2(e)/sqrt(d)) and K (scaled by s_b), split,
+        // K-major shared-memory operands of the logits
         const float sw = vrow ? (float)a.sw[p.row0[cw] + (row - 32 * p.grp[cw])] : 0.f;
-        uint32_t v[16], hv[16], lv[16];
+        uint32_t v[16];
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+        for (int part = 0; part < 4; ++part) {
           tmem_ld16(tmem + lane_addr + T_PROJ + 16u * part, v);
           tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float x = __uint_as_float(v[j]) * (sw * qscale);
-            const float hi = tf32_rna(x);
-            hv[j] = __float_as_uint(hi);
-            lv[j] = __float_as_uint(tf32_rna(x - hi));
-          }
-          tmem_st16(tmem + lane_addr + T_PROJ + 16u * part, hv);
-          tmem_st16(tmem + lane_addr + T_QLO + 16u * part, lv);
-        }
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          tmem_ld16(tmem + lane_addr + T_PROJ + 32u + 16u * part, v);
-          tmem_wait_ld();
+          const float f = part < 2 ? sw * qscale : sw;
+          unsigned char* base = sm + (part < 2 ? OFF_Q : OFF_K);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            const int h = 2 * part + hh;
-            float4 kh[2], kl[2];
+            const int h = 2 * (part & 1) + hh;
+            float4 xh[2], xl[2];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float x = __uint_as_float(v[8 * hh + j]) * sw;
+              const float x = __uint_as_float(v[8 * hh + j]) * f;
               const float hi = tf32_rna(x);
-              reinterpret_cast<float*>(kh)[j] = hi;
-              reinterpret_cast<float*>(kl)[j] = tf32_rna(x - hi);
+              reinterpret_cast<float*>(xh)[j] = hi;
+              reinterpret_cast<float*>(xl)[j] = tf32_rna(x - hi);
             }
-            unsigned char* kb = sm + OFF_K + (size_t)(2 * h) * K_BYTES;
+            unsigned char* hb = base + (size_t)(2 * h) * K_BYTES;
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
               const uint32_t off = kmajor_offset(row, 4 * ch, R);
-              *reinterpret_cast<float4*>(kb + off) = kh[ch];
-              *reinterpret_cast<float4*>(kb + K_BYTES + off) = kl[ch];
+              *reinterpret_cast<float4*>(hb + off) = xh[ch];
+              *reinterpret_cast<float4*>(hb + K_BYTES + off) = xl[ch];
             }
           }
         }
-        tmem_wait_st();
         fence_proxy_async();
         tc_fence_before();
         mbar_arrive(&mt.bar_qk);
@@ -487,6 +492,10 @@ __global__ void __launch_bounds__(tc2::NT, 1)
         tc_fence_before();
         mbar_arrive(&mt.bar_v);
       }
+      // ---- the next tile's slab into the A operands (its projection then
+      // overlaps this tile's softmax)
+      Plan pn;
+      if (!split((t + 1) & 1, pn)) { ok = false; break; }
       // ---- softmax of this group's heads (buffer b = grp)
       const int b = grp;
       for (int hi2 = 0; hi2 < 2 && ok; ++hi2) {
@@ -558,9 +567,9 @@ __global__ void __launch_bounds__(tc2::NT, 1)
       if (!wpv[b].wait(&mt.bar_pv[b])) { ok = false; break; }
       tc_fence_after();
       if (grp == 0 && gt == 0) bulk_wait_read_all();  // the staging buffer is free
-      // both groups must have seen the staging free: group 0 thread 0 waits first
-      // (its bulk copies are the only readers), then every thread of both groups
-      // arrives, and the writes follow the barrier
+      // group 0 thread 0 (whose bulk copies are the only readers of the
+      // staging buffer) waits first; every thread of both groups then arrives,
+      // and the writes follow the barrier
       mbar_arrive(&mt.bar_epi);
       if (!wepi.wait(&mt.bar_epi)) { ok = false; break; }
       if (cw >= 0) {
@@ -593,6 +602,7 @@ __global__ void __launch_bounds__(tc2::NT, 1)
           bulk_s2g(out + p.row0[c] * C, so + 32 * p.grp[c] * C, (uint32_t)(p.n[c] * C * 4));
         bulk_commit();
       }
+      p = pn;
     }
     if (grp == 0 && gt == 0) bulk_wait_all();
     if (!ok) mt.fail = 1;

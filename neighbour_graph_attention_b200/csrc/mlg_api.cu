@@ -349,7 +349,7 @@ void launch_count_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
   if (plan.max_reach <= 1) {
     const size_t sm_count_ = cellscan_smem(false);
     prefer_shared(k_cellscan<false>, sm_count_);
-    k_cellscan<false><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kCellWarps * 32,
+    k_cellscan<false><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kScanWarps * 32,
                         sm_count_, stream>>>(a);
   } else {
     k_count<<<(int)((a.n + kCountWarps - 1) / kCountWarps), kCountWarps * 32, 0, stream>>>(a);
@@ -362,7 +362,7 @@ void launch_fill_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
   if (plan.max_reach <= 1) {
     const size_t sm_fill = cellscan_smem(true);
     prefer_shared(k_cellscan<true>, sm_fill);
-    k_cellscan<true><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kCellWarps * 32,
+    k_cellscan<true><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kScanWarps * 32,
                        sm_fill, stream>>>(a);
   } else {
     const size_t fill_smem = (size_t)kFillWarps * 2 * kFillMaxCand * sizeof(unsigned long long);

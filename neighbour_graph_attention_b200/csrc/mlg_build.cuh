@@ -906,7 +906,19 @@ __global__ void __launch_bounds__(kFillWarps * 32) k_fill(BuildArgs a) {
 // to the per-centre traversal of global memory.
 constexpr int kCellCand = 768;       // stage capacity of the kernel chain
 constexpr int kCellCandSmall = 2048; // one-launch build of systems of at most 75 atoms
-constexpr int kCellWarps = 8;
+constexpr int kCellWarps = 8;   // warps of the one-launch build's CTAs
+// warps of the per-cell count and fill CTAs of the kernel chain, and their
+// minimum resident CTAs per SM (launch bounds)
+#ifndef MLG_SCAN_WARPS
+#define MLG_SCAN_WARPS 8
+#endif
+#ifndef MLG_COUNT_MINB
+#define MLG_COUNT_MINB 4
+#endif
+#ifndef MLG_FILL_MINB
+#define MLG_FILL_MINB 3
+#endif
+constexpr int kScanWarps = MLG_SCAN_WARPS;
 static_assert(kCellCandSmall <= (1 << kSlotBits), "staged_key slot bits");
 
 template <int CAP>
@@ -928,19 +940,19 @@ struct CellStageT {
 };
 using CellStage = CellStageT<kCellCand>;
 
-// Dynamic shared memory of the per-cell scans: the stage, the fill's key
-// buffers, and (REC) the candidates' exact records.
-constexpr size_t kCellKeysBytes = (size_t)kCellWarps * 2 * kFillMaxCand * sizeof(unsigned long long);
-template <int CAP>
+// Dynamic shared memory of the per-cell scans (NW warps): the stage, the
+// fill's key buffers, and (REC) the candidates' exact records.
+template <int CAP, int NW = kCellWarps>
 struct CellSmem {
+  static constexpr size_t keys_bytes = (size_t)NW * 2 * kFillMaxCand * sizeof(unsigned long long);
   static constexpr size_t keys_off = ((sizeof(CellStageT<CAP>) + 15) / 16) * 16;
-  static constexpr size_t rec_off = keys_off + kCellKeysBytes;
+  static constexpr size_t rec_off = keys_off + keys_bytes;
   static constexpr size_t bytes(bool fill, bool rec) {
-    return rec ? rec_off + (size_t)CAP * sizeof(Rec) : keys_off + (fill ? kCellKeysBytes : 0);
+    return rec ? rec_off + (size_t)CAP * sizeof(Rec) : keys_off + (fill ? keys_bytes : 0);
   }
 };
 __host__ __device__ constexpr size_t cellscan_smem(bool fill, bool rec = false) {
-  return CellSmem<kCellCand>::bytes(fill, rec);
+  return CellSmem<kCellCand, kScanWarps>::bytes(fill, rec);
 }
 
 // Count (FILL = false: raw, kept, truncations) or fill (FILL: the CSR rows)
@@ -951,20 +963,20 @@ __host__ __device__ constexpr size_t cellscan_smem(bool fill, bool rec = false) 
 // the same cell from an earlier call are reused.  With STASH (and REC) the
 // count keeps each warp's accepted keys and distances in its key buffer, and
 // a fill of the same centre by the same warp starts from them.
-template <bool FILL, bool REC, bool STASH = false, int CAP = kCellCand>
+template <bool FILL, bool REC, bool STASH = false, int CAP = kCellCand, int NW = kCellWarps>
 __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratch* sws,
                               unsigned char* s_dyn, int cell, int ys, int nsplit,
                               const int* row_off) {
   CellStageT<CAP>& cs = *reinterpret_cast<CellStageT<CAP>*>(s_dyn);
   unsigned long long* s_keys =
-      reinterpret_cast<unsigned long long*>(s_dyn + CellSmem<CAP>::keys_off);
-  Rec* s_rec = reinterpret_cast<Rec*>(s_dyn + CellSmem<CAP>::rec_off);  // REC only
+      reinterpret_cast<unsigned long long*>(s_dyn + CellSmem<CAP, NW>::keys_off);
+  Rec* s_rec = reinterpret_cast<Rec*>(s_dyn + CellSmem<CAP, NW>::rec_off);  // REC only
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (cell >= sg.ncell) return;
   const bool reuse = cs.staged_cell == cell;
   const int c_lo = reuse ? cs.c_lo : a.cell_start[cell];
   const int c_hi = reuse ? cs.c_hi : a.cell_start[cell + 1];
-  if (c_lo + ys * kCellWarps >= c_hi) return;
+  if (c_lo + ys * NW >= c_hi) return;
   const int cz = cell % sg.n[2], cy = (cell / sg.n[2]) % sg.n[1], cx = cell / (sg.n[2] * sg.n[1]);
   if (!reuse) {
     __syncthreads();  // earlier readers of the staging arrays are done
@@ -1015,13 +1027,13 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
         cs.c_hi = c_hi;
       }
     }
-    if (STASH && tid < kCellWarps) cs.stash_ci[tid] = -1;  // stashed slots refer to the old staging
+    if (STASH && tid < NW) cs.stash_ci[tid] = -1;  // stashed slots refer to the old staging
     __syncthreads();
     if (!cs.fallback) {
       // stage the candidates: slot t of stencil cell s (pre[s] <= t <
       // pre[s + 1]); two slots per thread and round, loads first
       const int K = cs.ncand;
-      constexpr int NT = kCellWarps * 32;
+      constexpr int NT = NW * 32;
       for (int t0 = tid; t0 < K; t0 += 2 * NT) {
         int q[2], tp[2];
         float4 pv[2];
@@ -1066,7 +1078,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
   const int self_tp = (64 << 14) | (64 << 7) | 64;
   unsigned long long* keys = s_keys + (size_t)warp * 2 * kFillMaxCand;
   uint32_t st = 0;
-  for (int ci = c_lo + ys * kCellWarps + warp; ci < c_hi; ci += nsplit * kCellWarps) {
+  for (int ci = c_lo + ys * NW + warp; ci < c_hi; ci += nsplit * NW) {
     // the centre's own record: staged (self stencil cell) or global
     const int self_slot = cs.self_pre + (ci - c_lo);
     const bool staged_self = REC && !cs.fallback;
@@ -1199,10 +1211,11 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
 }
 
 template <bool FILL>
-__global__ void __launch_bounds__(kCellWarps * 32, FILL ? 3 : 4) k_cellscan(BuildArgs a) {
+__global__ void __launch_bounds__(kScanWarps * 32, FILL ? MLG_FILL_MINB : MLG_COUNT_MINB)
+    k_cellscan(BuildArgs a) {
   if (gated_off(a.gate)) return;
   __shared__ CellGrid sg;
-  __shared__ WarpScratch sws[kCellWarps];
+  __shared__ WarpScratch sws[kScanWarps];
   extern __shared__ __align__(16) unsigned char s_dyn[];
   if (threadIdx.x == 0) {
     sg = *a.grid;
@@ -1210,7 +1223,8 @@ __global__ void __launch_bounds__(kCellWarps * 32, FILL ? 3 : 4) k_cellscan(Buil
   }
   __syncthreads();
   // blockIdx.y splits a cell's centres over several CTAs (small grids)
-  cellscan_item<FILL, false>(a, sg, sws, s_dyn, blockIdx.x, blockIdx.y, gridDim.y, nullptr);
+  cellscan_item<FILL, false, false, kCellCand, kScanWarps>(a, sg, sws, s_dyn, blockIdx.x,
+                                                           blockIdx.y, gridDim.y, nullptr);
 }
 
 // ------------------------------------------------------------------ scans

@@ -17,6 +17,7 @@
 #include "mlg_attn_dmma.cuh"
 #include "mlg_attn_tc.cuh"
 #include "mlg_attn_tc2.cuh"
+#include "mlg_attn_tc3.cuh"
 #include "mlg_attn_hgtc.cuh"
 #include "mlg_local.cuh"
 #include "mlg_verlet.cuh"
@@ -653,16 +654,25 @@ int launch_tc(TileArgs& ta, cudaStream_t stream) {
 
 // fp32, 32 channels, 4 heads, one layer: every product on tcgen05 (centres of
 // up to 64 edges); one CTA of 320 threads per SM holding all of its TMEM.
+#ifndef MLG_TC_ATTN
+#define MLG_TC_ATTN 3
+#endif
 int launch_tc2(TileArgs& ta, cudaStream_t stream) {
+#if MLG_TC_ATTN == 3
+  auto kern = k_attn_tc3;
+  const size_t smem = tc3::SMEM;
+#else
   auto kern = k_attn_tc2;
-  prefer_shared(kern, tc2::SMEM);
+  const size_t smem = tc2::SMEM;
+#endif
+  prefer_shared(kern, smem);
   if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
   CUtensorMap map;
   if (!encode_slab_map(&map, ta.G, ta.capacity, tc2::C, 32)) return MLG_ERR_CUDA;
   const int64_t want = sm_count();
   int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
   if (grid < 1) grid = 1;
-  kern<<<grid, tc2::NT, tc2::SMEM, stream>>>(ta, map);
+  kern<<<grid, tc2::NT, smem, stream>>>(ta, map);
   return launch_status();
 }
 

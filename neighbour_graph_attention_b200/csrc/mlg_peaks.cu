@@ -165,7 +165,7 @@ __global__ void k_bf16_16816(float* out, int iters) {
 // kind::tf32 of M = 128, N, K = 8 into one TMEM accumulator (A from shared
 // memory, or with TS from TMEM), then commits and waits (bounded).  The
 // operands are small constant tiles; only the issue rate matters.
-template <int N, bool TS>
+template <int N, bool TS, int NCHAIN = 1>
 __global__ void __launch_bounds__(128) k_umma_tf32(float* out, int iters) {
   using namespace mlg;
   __shared__ __align__(1024) float sA[128 * 8];
@@ -198,13 +198,15 @@ __global__ void __launch_bounds__(128) k_umma_tf32(float* out, int iters) {
     for (int it = 0; it < iters; ++it) {
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
+        // NCHAIN independent accumulators, used round-robin
+        const uint32_t d = tmem + (uint32_t)((u % NCHAIN) * N);
         if (TS)
           asm volatile(
               "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
               "r"(tmem + 256u), "l"(db), "r"(id), "r"(1u));
         else
-          umma_tf32(tmem, da, db, id, 1u);
+          umma_tf32(d, da, db, id, 1u);
       }
     }
     umma_commit(&bar);
@@ -278,15 +280,25 @@ int main() {
   const double u96 = umma(k_umma_tf32<96, false>, 96);
   const double u64ts = umma(k_umma_tf32<64, true>, 64);
   const double u16ts = umma(k_umma_tf32<16, true>, 16);
+  // independent accumulator chains (does a short MMA pipeline across them?)
+  const double u16ts4 = umma(k_umma_tf32<16, true, 4>, 16);
+  const double u16ts8 = umma(k_umma_tf32<16, true, 8>, 16);
+  const double u64ts4 = umma(k_umma_tf32<64, true, 4>, 64);
+  const double u16ss8 = umma(k_umma_tf32<16, false, 8>, 16);
+  const double u128ss2 = umma(k_umma_tf32<128, false, 2>, 128);
   cudaError_t e = cudaGetLastError();
   printf("{\"sm_count\": %d, \"clock_khz_attr\": %d, \"fp64_fma_tflops\": %.3f, "
          "\"fp32_fma_tflops\": %.3f, \"ex2_tops\": %.4f, \"dmma_m8n8k4_tflops\": %.3f, "
          "\"dmma_m16n8k16_tflops\": %.3f, \"mma_sync_tf32_m16n8k8_tflops\": %.3f, "
          "\"mma_sync_bf16_m16n8k16_tflops\": %.3f, \"tcgen05_tf32_m128n256_tflops\": %.2f, "
          "\"tcgen05_tf32_m128n96_tflops\": %.2f, \"tcgen05_tf32_ts_m128n64_tflops\": %.2f, "
-         "\"tcgen05_tf32_ts_m128n16_tflops\": %.2f, \"cuda\": \"%s\"}\n",
+         "\"tcgen05_tf32_ts_m128n16_tflops\": %.2f, \"tcgen05_tf32_ts_m128n16_4chains_tflops\": "
+         "%.2f, \"tcgen05_tf32_ts_m128n16_8chains_tflops\": %.2f, "
+         "\"tcgen05_tf32_ts_m128n64_4chains_tflops\": %.2f, "
+         "\"tcgen05_tf32_ss_m128n16_8chains_tflops\": %.2f, "
+         "\"tcgen05_tf32_ss_m128n128_2chains_tflops\": %.2f, \"cuda\": \"%s\"}\n",
          sms, clk, dfma, ffma, ex2, dmma884, dmma16816, tf32, bf16, u256, u96, u64ts, u16ts,
-         cudaGetErrorString(e));
+         u16ts4, u16ts8, u64ts4, u16ss8, u128ss2, cudaGetErrorString(e));
   cudaFree(dbuf);
   cudaFree(fbuf);
   return e == cudaSuccess ? 0 : 1;

@@ -30,7 +30,8 @@
 //               on the special-function unit, sum
 //   P V         o = sum_b p_b v_b with broadcast reads of the centre's v_b
 //               rows, packed fp32x2 FMAs
-//   epilogue    o / sum staged in shared memory, one bulk copy per centre
+//   output      o / sum straight to global memory: each thread's 8 values of
+//               a head are one whole 32-byte sector of its output row
 // The projection's TMEM is free once Q, K and V are read back, so the next
 // slab is split at once and its projection runs during this tile's softmax.
 //
@@ -38,8 +39,8 @@
 //   warp 0     issues every MMA (one elected thread)
 //   warp 1     plans tiles and loads each slab with 2-D TMA boxes of
 //              {4 channels x 32 rows} straight into the K-major operand layout
-//   warps 2-5  group 0: split, Q and K, heads 0 and 2, epilogue
-//   warps 6-9  group 1: split, V, heads 1 and 3, epilogue
+//   warps 2-5  group 0: split, Q and K, heads 0 and 2
+//   warps 6-9  group 1: split, V, heads 1 and 3
 // Every wait is bounded; on expiry the kernel records MLG_STATUS_TIMEOUT,
 // every role leaves its loop, the MMA thread waits for its own MMAs and the
 // producer for its last copy before TMEM is freed.
@@ -85,8 +86,7 @@ constexpr size_t OFF_ALO = OFF_AHI + A_BYTES;
 constexpr size_t OFF_Q = OFF_ALO + A_BYTES;             // [head][hi, lo]
 constexpr size_t OFF_K = OFF_Q + 2 * H * K_BYTES;       // [head][hi, lo]
 constexpr size_t OFF_V = OFF_K + 2 * H * K_BYTES;       // [128][VS] fp32
-constexpr size_t OFF_OUT = OFF_V + (size_t)R * VS * 4;  // [128][32] row-major staging
-constexpr size_t OFF_META = OFF_OUT + A_BYTES;
+constexpr size_t OFF_META = OFF_V + (size_t)R * VS * 4;
 
 struct Meta {
   Plan plan[2];             // ring of two: the tile being computed and the next
@@ -103,7 +103,7 @@ struct Meta {
   uint64_t bar_v;           // V rows in shared memory (count GT)
   uint64_t bar_s[2];        // logits of buffer b done (commit)
   uint64_t bar_sfree[2];    // logits of buffer b read into registers (count GT)
-  uint64_t bar_epi;         // both groups staged their outputs (count 2 * GT)
+  uint64_t bar_vfree;       // both groups are done with the V rows of a tile (count 2 * GT)
   uint64_t bar_fin;         // every MMA of the CTA done (commit, at exit)
 };
 constexpr size_t SMEM = OFF_META + sizeof(Meta);
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(tc3::NT, 1)
       mbar_init(&mt.bar_s[b], 1);
       mbar_init(&mt.bar_sfree[b], GT);
     }
-    mbar_init(&mt.bar_epi, 2 * GT);
+    mbar_init(&mt.bar_vfree, 2 * GT);
     mbar_init(&mt.bar_fin, 1);
     fence_mbar_init();
   }
@@ -293,12 +293,11 @@ __global__ void __launch_bounds__(tc3::NT, 1)
   } else {
     // ------------------------------------------------------------ compute groups
     const int grp = (warp - 2) >> 2;           // 0 or 1
-    const int gt = tid - 64 - grp * GT;        // 0..127 within the group
     const int quad = warp & 3;                 // TMEM lane quadrant
     const int row = quad * 32 + lane;          // tile row of this thread
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const float qscale = (float)(1.4426950408889634 / 2.8284271247461903);  // log2(e)/sqrt(8)
-    Waiter wx[2], wproj, ws[2], wv, wepi;
+    Waiter wx[2], wproj, ws[2], wv, wvf;
     bool ok = true;
     // weights of the layer, split into TF32 hi / lo, K-major [96 x 32]
     for (int e = tid - 64; e < C * N3; e += 2 * GT) {
@@ -338,7 +337,7 @@ __global__ void __launch_bounds__(tc3::NT, 1)
       return true;
     };
     const float* sV = reinterpret_cast<const float*>(sm + OFF_V);
-    float* so = reinterpret_cast<float*>(sm + OFF_OUT);
+    float* out = static_cast<float*>(a.out);
     Plan p;
     ok = split(0, p);
     for (int t = 0; ok && p.ncent > 0; ++t) {
@@ -383,7 +382,9 @@ __global__ void __launch_bounds__(tc3::NT, 1)
         tc_fence_before();
         mbar_arrive(&mt.bar_qk);
       } else {
-        // ---- V rows, fp32 (padded stride: conflict-free 16-byte stores)
+        // ---- V rows, fp32 (padded stride: conflict-free 16-byte stores), once
+        // group 0 is done with the previous tile's rows
+        if (t > 0 && !wvf.wait(&mt.bar_vfree)) { ok = false; break; }
         uint32_t v[16];
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -405,12 +406,6 @@ __global__ void __launch_bounds__(tc3::NT, 1)
       if (!split((t + 1) & 1, pn)) { ok = false; break; }
       // ---- V rows of this tile must be in place (group 1 wrote them)
       if (!wv.wait(&mt.bar_v)) { ok = false; break; }
-      // ---- the staging buffer must be free (the previous bulk copies have
-      // read it): group 0 thread 0 waits, then every thread of both groups
-      // arrives; the writes below follow the barrier
-      if (grp == 0 && gt == 0) bulk_wait_read_all();
-      mbar_arrive(&mt.bar_epi);
-      if (!wepi.wait(&mt.bar_epi)) { ok = false; break; }
       // ---- heads grp and grp + 2: softmax and P V from registers
       const int b = grp;
       for (int hi2 = 0; hi2 < 2 && ok; ++hi2) {
@@ -478,28 +473,21 @@ __global__ void __launch_bounds__(tc3::NT, 1)
             }
           }
           if (vrow) {
+            // one whole 32-byte sector of the output row
             const float rl = 1.f / l;
-            *reinterpret_cast<float4*>(so + row * C + h * D) =
+            float* dst = out + (p.row0[cw] + (row - key0)) * C + h * D;
+            *reinterpret_cast<float4*>(dst) =
                 make_float4(o[0].x * rl, o[0].y * rl, o[1].x * rl, o[1].y * rl);
-            *reinterpret_cast<float4*>(so + row * C + h * D + 4) =
+            *reinterpret_cast<float4*>(dst + 4) =
                 make_float4(o[2].x * rl, o[2].y * rl, o[3].x * rl, o[3].y * rl);
           }
         }
       }
       if (!ok) break;
-      // ---- epilogue: both groups' heads staged, one bulk copy per centre
-      fence_proxy_async();
-      mbar_arrive(&mt.bar_epi);
-      if (!wepi.wait(&mt.bar_epi)) { ok = false; break; }
-      if (grp == 0 && gt == 0) {
-        float* out = static_cast<float*>(a.out);
-        for (int c = 0; c < p.ncent; ++c)
-          bulk_s2g(out + p.row0[c] * C, so + 32 * p.grp[c] * C, (uint32_t)(p.n[c] * C * 4));
-        bulk_commit();
-      }
+      // this group is done with the tile's V rows
+      mbar_arrive(&mt.bar_vfree);
       p = pn;
     }
-    if (grp == 0 && gt == 0) bulk_wait_all();
     if (!ok) mt.fail = 1;
   }
   // ---- teardown: report, let a slab copy in flight land, free TMEM

@@ -913,10 +913,10 @@ constexpr int kCellWarps = 8;   // warps of the one-launch build's CTAs
 #define MLG_SCAN_WARPS 8
 #endif
 #ifndef MLG_COUNT_MINB
-#define MLG_COUNT_MINB 4
+#define MLG_COUNT_MINB 5
 #endif
 #ifndef MLG_FILL_MINB
-#define MLG_FILL_MINB 3
+#define MLG_FILL_MINB 4
 #endif
 constexpr int kScanWarps = MLG_SCAN_WARPS;
 static_assert(kCellCandSmall <= (1 << kSlotBits), "staged_key slot bits");

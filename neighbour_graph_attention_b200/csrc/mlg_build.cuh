@@ -913,7 +913,7 @@ constexpr int kCellWarps = 8;   // warps of the one-launch build's CTAs
 #define MLG_SCAN_WARPS 8
 #endif
 #ifndef MLG_COUNT_MINB
-#define MLG_COUNT_MINB 5
+#define MLG_COUNT_MINB 4
 #endif
 #ifndef MLG_FILL_MINB
 #define MLG_FILL_MINB 4
@@ -934,7 +934,8 @@ struct CellStageT {
   int c_lo, c_hi;           // the staged cell's centres (cell-order range)
   int stash_ci[kCellWarps];   // STASH: centre whose accepted keys a warp still holds (-1: none)
   int stash_cnt[kCellWarps];  // and how many
-  float4 cand[CAP];   // position + image offset, atom index in .w
+  float4 cand[CAP + 64];  // position + image offset, atom index in .w; padded with
+                          // far-away sentinels to a multiple of 64 slots
   int cq[CAP];        // cell-order index (record of the exact data)
   int ct[CAP];        // packed image of the stencil cell
 };
@@ -1068,6 +1069,10 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
           if (REC) s_rec[t] = rv[u];
         }
       }
+      // sentinels up to a multiple of 64 slots: far away, so never accepted
+      // and never near the cutoff (their squared distance overflows to +inf)
+      for (int t = K + tid; t < ((K + 63) & ~63); t += NT)
+        cs.cand[t] = make_float4(1e30f, 1e30f, 1e30f, __int_as_float(-1));
     }
     __syncthreads();
   } else if (!FILL && threadIdx.x == 0) {
@@ -1075,7 +1080,6 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
   }
   if (!FILL) __syncthreads();
   const int K = cs.ncand;
-  const int self_tp = (64 << 14) | (64 << 7) | 64;
   unsigned long long* keys = s_keys + (size_t)warp * 2 * kFillMaxCand;
   uint32_t st = 0;
   for (int ci = c_lo + ys * NW + warp; ci < c_hi; ci += nsplit * NW) {
@@ -1134,38 +1138,50 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
     const bool need_d2 = FILL && a.raw[i] > n;
     constexpr bool kCollect = FILL || STASH;
     int cnt = 0;
-    for (int base = 0; base < K; base += 32) {
-      const int t = base + lane;
-      bool acc = false;
-      double r2 = 0.0;
-      int tp = 0, j = -1;
-      if (t < K) {
-        const float4 c4 = cs.cand[t];
-        const float dx = c4.x - pi.x, dy = c4.y - pi.y, dz = c4.z - pi.z;
-        const float r2f = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
-        tp = cs.ct[t];
-        j = __float_as_int(c4.w);
-        if (r2f < sg.r2lo) {
-          acc = !(j == i && tp == self_tp);
-        } else if (r2f <= sg.r2hi) {
-          acc = test_candidate(sg, cc, REC ? s_rec[t] : a.recs[cs.cq[t]], tp, a.rc2, &r2);
-        }
-      }
-      if (!kCollect) {
-        cnt += acc ? 1 : 0;
-      } else {
-        const unsigned m = __ballot_sync(kFull, acc);
-        if (acc) {
-          const int qd = cnt + __popc(m & lanemask_lt());
-          if (qd < kFillMaxCand) {
-            keys[qd] = REC ? staged_key(j, tp, t) : edge_key(j, tp);
-            if (!REC && need_d2) {
-              test_candidate(sg, cc, a.recs[cs.cq[t]], tp, a.rc2, &r2);
-              keys[kFillMaxCand + qd] = (unsigned long long)__double_as_longlong(r2);
-            }
+    // the candidates, two per lane per step (slots t0 and t0 + 32 of a block
+    // of 64); the fp32 prefilter decides all but the few within its margin of
+    // rcut^2, which take the exact test outside the common path.  The centre
+    // itself is the staged slot self_slot (its own cell, image 0).
+    auto collect = [&](bool acc, int t, const float4& c) {
+      const unsigned m = __ballot_sync(kFull, acc);
+      if (acc) {
+        const int qd = cnt + __popc(m & lanemask_lt());
+        if (qd < kFillMaxCand) {
+          const int j = __float_as_int(c.w), tp = cs.ct[t];
+          keys[qd] = REC ? staged_key(j, tp, t) : edge_key(j, tp);
+          if (!REC && need_d2) {
+            double r2;
+            test_candidate(sg, cc, a.recs[cs.cq[t]], tp, a.rc2, &r2);
+            keys[kFillMaxCand + qd] = (unsigned long long)__double_as_longlong(r2);
           }
         }
-        cnt += __popc(m);
+      }
+      cnt += __popc(m);
+    };
+    const int Kp = (K + 63) & ~63;
+    for (int base = 0; base < Kp; base += 64) {
+      const int t0 = base + lane, t1 = t0 + 32;
+      const float4 c0 = cs.cand[t0], c1 = cs.cand[t1];
+      const float dx0 = c0.x - pi.x, dy0 = c0.y - pi.y, dz0 = c0.z - pi.z;
+      const float dx1 = c1.x - pi.x, dy1 = c1.y - pi.y, dz1 = c1.z - pi.z;
+      const float r0 = fmaf(dz0, dz0, fmaf(dy0, dy0, dx0 * dx0));
+      const float r1 = fmaf(dz1, dz1, fmaf(dy1, dy1, dx1 * dx1));
+      bool a0 = r0 < sg.r2lo && t0 != self_slot;
+      bool a1 = r1 < sg.r2lo && t1 != self_slot;
+      const bool e0 = !(r0 < sg.r2lo) && r0 <= sg.r2hi;
+      const bool e1 = !(r1 < sg.r2lo) && r1 <= sg.r2hi;
+      if (__any_sync(kFull, e0 || e1)) {
+        double r2;
+        if (e0) a0 = test_candidate(sg, cc, REC ? s_rec[t0] : a.recs[cs.cq[t0]], cs.ct[t0],
+                                    a.rc2, &r2);
+        if (e1) a1 = test_candidate(sg, cc, REC ? s_rec[t1] : a.recs[cs.cq[t1]], cs.ct[t1],
+                                    a.rc2, &r2);
+      }
+      if (!kCollect) {
+        cnt += (a0 ? 1 : 0) + (a1 ? 1 : 0);
+      } else {
+        collect(a0, t0, c0);
+        collect(a1, t1, c1);
       }
     }
     if (REC && kCollect && (FILL ? need_d2 : cnt > a.nnei_max) && cnt <= kFillMaxCand) {

@@ -18,6 +18,7 @@
 #include "mlg_attn_tc.cuh"
 #include "mlg_attn_tc2.cuh"
 #include "mlg_attn_tc3.cuh"
+#include "mlg_attn_tc4.cuh"
 #include "mlg_attn_hgtc.cuh"
 #include "mlg_local.cuh"
 #include "mlg_verlet.cuh"
@@ -654,16 +655,27 @@ int launch_tc(TileArgs& ta, cudaStream_t stream) {
 
 // fp32, 32 channels, 4 heads, one layer: every product on tcgen05 (centres of
 // up to 64 edges); one CTA of 320 threads per SM holding all of its TMEM.
+// Which kernel takes fp32 rows of up to 64 edges at 32 channels, 4 heads,
+// one layer: 0 = the tile kernel of every fp32 row (logits and P V on the
+// FP32 pipe), 2 = every product on tcgen05, 3 = the logits on tcgen05 (two
+// groups of warps), 4 = the logits on tcgen05 (one group of warps per head).
 #ifndef MLG_TC_ATTN
-#define MLG_TC_ATTN 3
+#define MLG_TC_ATTN 0
 #endif
+constexpr bool kTcAttn = MLG_TC_ATTN != 0;
 int launch_tc2(TileArgs& ta, cudaStream_t stream) {
-#if MLG_TC_ATTN == 3
+#if MLG_TC_ATTN == 4
+  auto kern = k_attn_tc4;
+  const size_t smem = tc4::SMEM;
+  const int nt = tc4::NT;
+#elif MLG_TC_ATTN == 3
   auto kern = k_attn_tc3;
   const size_t smem = tc3::SMEM;
+  const int nt = tc3::NT;
 #else
   auto kern = k_attn_tc2;
   const size_t smem = tc2::SMEM;
+  const int nt = tc2::NT;
 #endif
   prefer_shared(kern, smem);
   if (cudaGetLastError() != cudaSuccess) return MLG_ERR_CUDA;
@@ -672,7 +684,7 @@ int launch_tc2(TileArgs& ta, cudaStream_t stream) {
   const int64_t want = sm_count();
   int grid = (int)(ta.n_centres < want ? ta.n_centres : want);
   if (grid < 1) grid = 1;
-  kern<<<grid, tc2::NT, smem, stream>>>(ta, map);
+  kern<<<grid, nt, smem, stream>>>(ta, map);
   return launch_status();
 }
 
@@ -807,7 +819,7 @@ int attention_stack_impl(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max
     ta.out = G_out;
     for (int k = 0; k < 3 * n_layers; ++k) ta.W[k] = W[k];
     ta.status = csr->status;
-    if (dtype == MLG_F32 && channels == 32 && D == 8 && n_layers == 1) {
+    if (kTcAttn && dtype == MLG_F32 && channels == 32 && D == 8 && n_layers == 1) {
       // centres of up to 64 edges with every product on tcgen05; longer ones
       // (up to the tile) on the kernel whose logits and P V run on the FP32 pipe
       rc = launch_tc2(ta, stream);
@@ -972,7 +984,8 @@ int forward_launches(int64_t n_atoms, int32_t nnei_max, int32_t channels, int32_
   const int D = heads > 0 ? channels / heads : 0;
   int R = tile_rows(dtype, channels, D, nnei_max);
   if (R > 0 && n_layers <= kMaxFusedLayers) {
-    const bool tc2_path = dtype == MLG_F32 && channels == 32 && D == 8 && n_layers == 1;
+    const bool tc2_path =
+        kTcAttn && dtype == MLG_F32 && channels == 32 && D == 8 && n_layers == 1;
     return 1 + (tc2_path && nnei_max > tc2::MAXN ? 1 : 0) + (nnei_max > R ? n_layers : 0);
   }
   int Rg = hg_rows(dtype, channels, D);

@@ -45,23 +45,20 @@ FP32_PEAK_TFLOPS = SM_COUNT * 128 * 2 * SM_MAX_GHZ / 1e3
 # Special-function unit (ex2): 16 per SM per clock.
 SFU_PEAK_TEXP = SM_COUNT * 16 * SM_MAX_GHZ / 1e3
 
-# Attention kernel of each workload and its DRAM traffic per launch
-# (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture of that
-# kernel, summarised under profiles/); None where no capture of the kernel as
-# it stands exists.  A change to a kernel resets its entry to None.
-ATTN_KERNEL = {
-    1: ("k_attn_hg<double,128,32,...>", None),
-    2: ("k_attn_dmma<160,5,640>", 5.622e6),   # profiles/k_attn_dmma_f64_diamond512.md
-    3: ("k_attn_tc<64,16,512>", None),
-    4: ("k_attn_hg<float,128,16,...>", None),
-    5: ("k_attn_tc2 (logits and P.V on tcgen05; k_attn_tc<32,8,512> for rows over 64)", None),
+# DRAM traffic per launch of a workload's attention (dram__bytes_read.sum +
+# dram__bytes_write.sum from one ncu capture, summarised under profiles/),
+# with the kernels it was taken on: used only while the library still
+# launches those kernels for the workload.  A change to a kernel removes its
+# entry.
+ATTN_TRAFFIC = {
+    2: ("k_attn_dmma", 5.622e6),   # profiles/k_attn_dmma_f64_diamond512.md
 }
 
 
-def tensor_core_path(w) -> bool:
-    """fp32, 32 channels, 4 heads, one layer: every product on tcgen05, so the
-    softmax's exponentials (special-function unit) bound the kernel, not FMAs."""
-    return w.dtype == "f32" and w.channels == 32 and w.heads == 4 and w.n_layers == 1
+def tensor_core_path(kernels: str) -> bool:
+    """The logits run on tcgen05 and P.V from registers: the softmax's
+    exponentials (special-function unit) are the roofline, not a pipe's FMAs."""
+    return "tcgen05 logits" in kernels
 
 
 def attention_exps(row_ptr, heads):
@@ -81,6 +78,10 @@ def parse_args(argv=None):
                    help="profiling only: conventional cells per axis of a lattice workload "
                         "(same shapes, fewer atoms)")
     p.add_argument("--impl", choices=["mlg", "reference"], default="mlg")
+    p.add_argument("--variant", choices=["block", "smooth", "local"], default="block",
+                   help="attention of the step: block-dense (default), block-dense with the "
+                        "slot-occupancy softmax in every layer, or local attention (one query "
+                        "per centre; the first layer's weights)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="CPU time budget of the oracle baseline sample")
@@ -96,6 +97,12 @@ def attention_flops(row_ptr, channels):
     """Per layer: sum_i (6 n_i c^2 + 4 n_i^2 c) (projections, QK^T, PV)."""
     n = np.diff(np.asarray(row_ptr)).astype(np.float64)
     return float(np.sum(6.0 * n * channels * channels + 4.0 * n * n * channels))
+
+
+def local_attention_flops(row_ptr, channels, heads):
+    """Local attention, reassociated: sum_i 2 (3 c^2 + 2 n_i c H)."""
+    n = np.diff(np.asarray(row_ptr)).astype(np.float64)
+    return float(np.sum(2.0 * (3.0 * channels * channels + 2.0 * n * channels * heads)))
 
 
 def attention_bytes(n_atoms, n_edges, channels, elem):
@@ -324,12 +331,16 @@ def select_workload(args):
 
 
 def workload_config(w, args, extra=None):
+    layers = 1 if getattr(args, "variant", "block") == "local" else w.n_layers
     cfg = {"workload": f"{w.name}: {w.n_atoms} atoms, {w.lattice}, rcut {w.rcut} A, "
                        f"nnei_max {w.nnei_max}, c={w.channels}, heads={w.heads}, "
-                       f"layers={w.n_layers}, {w.dtype}",
+                       f"layers={layers}, {w.dtype}",
            "workload_index": w.key, "seed": args.seed, "n_atoms": w.n_atoms,
            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU",
            "l2": "flushed between timed steps (256 MiB write)"}
+    if getattr(args, "variant", "block") != "block":
+        cfg["variant"] = {"smooth": "slot-occupancy softmax in every layer",
+                          "local": "local attention (one query per centre)"}[args.variant]
     if extra:
         cfg.update(extra)
     return cfg
@@ -385,7 +396,12 @@ def main(argv=None):
     del csr0
     csr = m.Csr.empty(w.n_atoms, E, device=dev)
     G0 = torch.as_tensor(C.features(args.workload, args.seed, E), dtype=dt, device=dev)
-    Gout = torch.empty_like(G0)
+    local = args.variant == "local"
+    # local attention writes one row per centre, from the centres' own features
+    Gout = torch.empty((w.n_atoms, w.channels), dtype=dt, device=dev) if local \
+        else torch.empty_like(G0)
+    Hc = torch.as_tensor(C.features(args.workload, args.seed + 1000, w.n_atoms), dtype=dt,
+                         device=dev) if local else None
     Wt = [torch.as_tensor(W[l][k], dtype=dt, device=dev) for l in range(w.n_layers)
           for k in range(3)]
     ws = m.workspace(m.mlg_forward_workspace_bytes(w.n_atoms, w.rcut, s["box"], s["pbc"], E,
@@ -401,9 +417,19 @@ def main(argv=None):
     def build_call():
         m.mlg_build_csr(sysd, w.rcut, w.r_on, w.nnei_max, csr, ws, stream=stream)
 
+    def attn_call(g_in, g_out):
+        if args.variant == "smooth":
+            m.mlg_attention_stack_smooth(csr, w.n_atoms, w.nnei_max, w.channels, w.heads,
+                                         w.n_layers, mdt, Wt, g_in, g_out, stack_ws, stream=stream)
+        elif local:
+            m.mlg_local_attention(csr, w.n_atoms, w.nnei_max, w.channels, w.heads, mdt, Hc, g_in,
+                                  g_out, Wt[0], Wt[1], Wt[2], stream=stream)
+        else:
+            m.mlg_attention_stack(csr, w.n_atoms, w.nnei_max, w.channels, w.heads, w.n_layers,
+                                  mdt, Wt, g_in, g_out, stack_ws, stream=stream)
+
     def stack_call():
-        m.mlg_attention_stack(csr, w.n_atoms, w.nnei_max, w.channels, w.heads, w.n_layers, mdt,
-                              Wt, G0, Gout, stack_ws, stream=stream)
+        attn_call(G0, Gout)
 
     def timed_steps(k):
         evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(k)]
@@ -460,17 +486,22 @@ def main(argv=None):
 
     attn_avg = statistics.mean(attn_ms_steps)
     build_avg = statistics.mean(build_ms_steps)
-    flops = attention_flops(row_ptr, w.channels) * w.n_layers
+    flops = local_attention_flops(row_ptr, w.channels, w.heads) if local else \
+        attention_flops(row_ptr, w.channels) * w.n_layers
     peak_fp = FP64_PEAK_TFLOPS if w.dtype == "f64" else FP32_PEAK_TFLOPS
     achieved_tf = flops / (attn_avg * 1e-3) / 1e12
     hbm_peak, hbm_src = load_peaks()
     bbytes = build_bytes(w.n_atoms, E)
     abytes = attention_bytes(w.n_atoms, E, w.channels, elem) + \
         (w.n_layers - 1) * 3.0 * w.channels * w.channels * elem
-    kname, traffic = ATTN_KERNEL.get(w.key, ("attention stack", None))
+    kernels = m.mlg_attention_kernels(w.nnei_max, w.channels, w.heads, w.n_layers, mdt)
+    kname = kernels if not local else "k_local_attn"
+    rec_k, traffic = ATTN_TRAFFIC.get(w.key, ("", None))
+    if rec_k != kname or args.variant != "block":
+        traffic = None
     if args.cells is not None:   # a resized system: the stored capture does not apply
         traffic = None
-    if tensor_core_path(w):
+    if tensor_core_path(kernels) and args.variant == "block":
         # products on the tensor cores: the exponentials bound the kernel
         # (special-function unit), ahead of HBM and of the tensor pipe
         exps = attention_exps(row_ptr, w.heads) * w.n_layers
@@ -520,8 +551,7 @@ def main(argv=None):
         x_d.copy_(x_h, non_blocking=True)
         m.mlg_build_csr(sys_e, w.rcut, w.r_on, w.nnei_max, csr, ws, stream=stream)
         stream.wait_event(ev_g)
-        m.mlg_attention_stack(csr, w.n_atoms, w.nnei_max, w.channels, w.heads, w.n_layers, mdt,
-                              Wt, g_d, Gout, stack_ws, stream=stream)
+        attn_call(g_d, Gout)
         out_h.copy_(Gout, non_blocking=True)
 
     timed_loop(e2e_step, 3)
@@ -566,8 +596,7 @@ def main(argv=None):
             if i >= 2:
                 stream.wait_event(ev_out[i - 2])
             m.mlg_build_csr(syss[b], w.rcut, w.r_on, w.nnei_max, csr, ws, stream=stream)
-            m.mlg_attention_stack(csr, w.n_atoms, w.nnei_max, w.channels, w.heads, w.n_layers,
-                                  mdt, Wt, gs[b], ys[b], stack_ws, stream=stream)
+            attn_call(gs[b], ys[b])
             ev_done[i].record(stream)
             s_out.wait_event(ev_done[i])
             with torch.cuda.stream(s_out):

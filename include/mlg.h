@@ -399,6 +399,11 @@ int mlg_build_csr_wait_test(const mlg_system* sys, double rcut, double r_on, int
                             const mlg_csr* csr, void* ws, size_t ws_bytes, int32_t polls,
                             mlg_stream_t stream);
 
+/* A static string naming the kernels mlg_attention_stack launches for this
+ * shape (for benchmark records); "" for invalid arguments. */
+const char* mlg_attention_kernels(int32_t nnei_max, int32_t channels, int32_t heads,
+                                  int32_t n_layers, mlg_dtype dtype);
+
 /* A static string naming a host status code. */
 const char* mlg_status_string(int status);
 

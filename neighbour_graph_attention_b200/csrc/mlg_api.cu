@@ -1177,6 +1177,37 @@ int mlg_forward_launch_count(int64_t n_atoms, double rcut, const double box[9],
          attn;
 }
 
+const char* mlg_attention_kernels(int32_t nnei_max, int32_t channels, int32_t heads,
+                                  int32_t n_layers, mlg_dtype dtype) {
+  if (channels < 1 || heads < 1 || channels % heads != 0 || n_layers < 1) return "";
+  const int D = channels / heads;
+  const int R = tile_rows(dtype, channels, D, nnei_max);
+  if (R > 0 && n_layers <= kMaxFusedLayers) {
+    if (dtype == MLG_F64) return nnei_max > R ? "k_attn_dmma + k_attn_generic" : "k_attn_dmma";
+    if (kTcAttn && channels == 32 && D == 8 && n_layers == 1) {
+#if MLG_TC_ATTN == 4
+#define MLG_TC_NAME "k_attn_tc4 (tcgen05 logits, rows <= 64)"
+#elif MLG_TC_ATTN == 3
+#define MLG_TC_NAME "k_attn_tc3 (tcgen05 logits, rows <= 64)"
+#else
+#define MLG_TC_NAME "k_attn_tc2 (tcgen05 logits and P.V, rows <= 64)"
+#endif
+      if (nnei_max > R) return MLG_TC_NAME " + k_attn_tc (rows <= 128) + k_attn_generic";
+      if (nnei_max > tc2::MAXN) return MLG_TC_NAME " + k_attn_tc (rows <= 128)";
+      return MLG_TC_NAME;
+#undef MLG_TC_NAME
+    }
+    return nnei_max > R ? "k_attn_tc + k_attn_generic" : "k_attn_tc";
+  }
+  const int Rg = hg_rows(dtype, channels, D);
+  if (Rg > 0) {
+    const char* k = dtype == MLG_F32 ? "k_attn_hgtc" : "k_attn_hg";
+    if (nnei_max <= Rg) return k;
+    return dtype == MLG_F32 ? "k_attn_hgtc + k_attn_generic" : "k_attn_hg + k_attn_generic";
+  }
+  return "k_attn_generic";
+}
+
 const char* mlg_status_string(int status) {
   switch (status) {
     case MLG_OK: return "MLG_OK";

@@ -125,6 +125,8 @@ _lib.mlg_verlet_step.argtypes = [ctypes.POINTER(mlg_system), _c_dbl, _c_dbl, _c_
 _lib.mlg_build_csr_wait_test.restype = ctypes.c_int
 _lib.mlg_build_csr_wait_test.argtypes = [ctypes.POINTER(mlg_system), _c_dbl, _c_dbl, _c_i32,
                                          ctypes.POINTER(mlg_csr), _p, _c_sz, _c_i32, _p]
+_lib.mlg_attention_kernels.restype = ctypes.c_char_p
+_lib.mlg_attention_kernels.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, ctypes.c_int]
 _lib.mlg_status_string.restype = ctypes.c_char_p
 _lib.mlg_status_string.argtypes = [ctypes.c_int]
 _lib.mlg_version.restype = ctypes.c_int
@@ -152,6 +154,13 @@ def mlg_exp2_neg(y, out, stream=None, check: bool = True) -> int:
     if check and rc != MLG_OK:
         raise MlgError(rc, "mlg_exp2_neg")
     return rc
+
+
+def mlg_attention_kernels(nnei_max: int, channels: int, heads: int, n_layers: int,
+                          dtype: int) -> str:
+    """The kernels mlg_attention_stack launches for this shape."""
+    return _lib.mlg_attention_kernels(int(nnei_max), int(channels), int(heads), int(n_layers),
+                                      int(dtype)).decode()
 
 
 def mlg_version() -> int:

@@ -19,6 +19,7 @@
 #include "mlg_attn_tc2.cuh"
 #include "mlg_attn_tc3.cuh"
 #include "mlg_attn_tc4.cuh"
+#include "mlg_attn_tc5.cuh"
 #include "mlg_attn_hgtc.cuh"
 #include "mlg_local.cuh"
 #include "mlg_verlet.cuh"
@@ -658,13 +659,18 @@ int launch_tc(TileArgs& ta, cudaStream_t stream) {
 // Which kernel takes fp32 rows of up to 64 edges at 32 channels, 4 heads,
 // one layer: 0 = the tile kernel of every fp32 row (logits and P V on the
 // FP32 pipe), 2 = every product on tcgen05, 3 = the logits on tcgen05 (two
-// groups of warps), 4 = the logits on tcgen05 (one group of warps per head).
+// groups of warps), 4 = the logits on tcgen05 (one group of warps per head),
+// 5 = as 4 with each group reading back its own head.
 #ifndef MLG_TC_ATTN
 #define MLG_TC_ATTN 0
 #endif
 constexpr bool kTcAttn = MLG_TC_ATTN != 0;
 int launch_tc2(TileArgs& ta, cudaStream_t stream) {
-#if MLG_TC_ATTN == 4
+#if MLG_TC_ATTN == 5
+  auto kern = k_attn_tc5;
+  const size_t smem = tc5::SMEM;
+  const int nt = tc5::NT;
+#elif MLG_TC_ATTN == 4
   auto kern = k_attn_tc4;
   const size_t smem = tc4::SMEM;
   const int nt = tc4::NT;
@@ -1185,7 +1191,9 @@ const char* mlg_attention_kernels(int32_t nnei_max, int32_t channels, int32_t he
   if (R > 0 && n_layers <= kMaxFusedLayers) {
     if (dtype == MLG_F64) return nnei_max > R ? "k_attn_dmma + k_attn_generic" : "k_attn_dmma";
     if (kTcAttn && channels == 32 && D == 8 && n_layers == 1) {
-#if MLG_TC_ATTN == 4
+#if MLG_TC_ATTN == 5
+#define MLG_TC_NAME "k_attn_tc5 (tcgen05 logits, rows <= 64)"
+#elif MLG_TC_ATTN == 4
 #define MLG_TC_NAME "k_attn_tc4 (tcgen05 logits, rows <= 64)"
 #elif MLG_TC_ATTN == 3
 #define MLG_TC_NAME "k_attn_tc3 (tcgen05 logits, rows <= 64)"

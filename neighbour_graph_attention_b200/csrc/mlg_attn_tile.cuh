@@ -69,11 +69,36 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait (about a second at most): false if the phase never completed.
+// One potentially blocking test: the hardware may hold the thread (without
+// issuing) until the phase completes or a system-dependent time limit passes.
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: false if the phase has not completed after about a second
+// (global timer) or 2^24 tests, whichever comes first.  A waiting warp is
+// held by try_wait rather than spinning, so it takes no issue slots from the
+// warps that work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (int it = 0; it < (1 << 22); ++it) {
-    if (mbar_test(bar, parity)) return true;
-    if (it > 64) __nanosleep(200);
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (int it = 0; it < (1 << 24); ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > 1000000000ull) return false;
   }
   return false;
 }

@@ -20,6 +20,7 @@
 #include "mlg_attn_tc3.cuh"
 #include "mlg_attn_tc4.cuh"
 #include "mlg_attn_tc5.cuh"
+#include "mlg_attn_tc6.cuh"
 #include "mlg_attn_hgtc.cuh"
 #include "mlg_local.cuh"
 #include "mlg_verlet.cuh"
@@ -654,19 +655,23 @@ int launch_tc(TileArgs& ta, cudaStream_t stream) {
   return launch_status();
 }
 
-// fp32, 32 channels, 4 heads, one layer: every product on tcgen05 (centres of
-// up to 64 edges); one CTA of 320 threads per SM holding all of its TMEM.
-// Which kernel takes fp32 rows of up to 64 edges at 32 channels, 4 heads,
+// fp32, 32 channels, 4 heads, one layer, centres of up to 64 edges: one CTA
+// per SM holding all of its TMEM.  Which kernel takes fp32 rows of up to 64 edges at 32 channels, 4 heads,
 // one layer: 0 = the tile kernel of every fp32 row (logits and P V on the
 // FP32 pipe), 2 = every product on tcgen05, 3 = the logits on tcgen05 (two
 // groups of warps), 4 = the logits on tcgen05 (one group of warps per head),
-// 5 = as 4 with each group reading back its own head.
+// 5 = as 4 with each group reading back its own head, 6 = as 5 with one
+// logits buffer of 64 columns per head (no buffer shared between heads).
 #ifndef MLG_TC_ATTN
-#define MLG_TC_ATTN 0
+#define MLG_TC_ATTN 6
 #endif
 constexpr bool kTcAttn = MLG_TC_ATTN != 0;
 int launch_tc2(TileArgs& ta, cudaStream_t stream) {
-#if MLG_TC_ATTN == 5
+#if MLG_TC_ATTN == 6
+  auto kern = k_attn_tc6;
+  const size_t smem = tc6::SMEM;
+  const int nt = tc6::NT;
+#elif MLG_TC_ATTN == 5
   auto kern = k_attn_tc5;
   const size_t smem = tc5::SMEM;
   const int nt = tc5::NT;
@@ -1191,7 +1196,9 @@ const char* mlg_attention_kernels(int32_t nnei_max, int32_t channels, int32_t he
   if (R > 0 && n_layers <= kMaxFusedLayers) {
     if (dtype == MLG_F64) return nnei_max > R ? "k_attn_dmma + k_attn_generic" : "k_attn_dmma";
     if (kTcAttn && channels == 32 && D == 8 && n_layers == 1) {
-#if MLG_TC_ATTN == 5
+#if MLG_TC_ATTN == 6
+#define MLG_TC_NAME "k_attn_tc6 (tcgen05 logits, rows <= 64)"
+#elif MLG_TC_ATTN == 5
 #define MLG_TC_NAME "k_attn_tc5 (tcgen05 logits, rows <= 64)"
 #elif MLG_TC_ATTN == 4
 #define MLG_TC_NAME "k_attn_tc4 (tcgen05 logits, rows <= 64)"

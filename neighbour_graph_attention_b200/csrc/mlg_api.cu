@@ -21,6 +21,7 @@
 #include "mlg_attn_tc4.cuh"
 #include "mlg_attn_tc5.cuh"
 #include "mlg_attn_tc6.cuh"
+#include "mlg_attn_tc7.cuh"
 #include "mlg_attn_hgtc.cuh"
 #include "mlg_local.cuh"
 #include "mlg_verlet.cuh"
@@ -661,13 +662,19 @@ int launch_tc(TileArgs& ta, cudaStream_t stream) {
 // FP32 pipe), 2 = every product on tcgen05, 3 = the logits on tcgen05 (two
 // groups of warps), 4 = the logits on tcgen05 (one group of warps per head),
 // 5 = as 4 with each group reading back its own head, 6 = as 5 with one
-// logits buffer of 64 columns per head (no buffer shared between heads).
+// logits buffer of 64 columns per head (no buffer shared between heads),
+// 7 = as 6 with P V on warp-level tensor-core MMAs and the slabs planned and
+// loaded two tiles ahead.
 #ifndef MLG_TC_ATTN
-#define MLG_TC_ATTN 6
+#define MLG_TC_ATTN 7
 #endif
 constexpr bool kTcAttn = MLG_TC_ATTN != 0;
 int launch_tc2(TileArgs& ta, cudaStream_t stream) {
-#if MLG_TC_ATTN == 6
+#if MLG_TC_ATTN == 7
+  auto kern = k_attn_tc7;
+  const size_t smem = tc7::SMEM;
+  const int nt = tc7::NT;
+#elif MLG_TC_ATTN == 6
   auto kern = k_attn_tc6;
   const size_t smem = tc6::SMEM;
   const int nt = tc6::NT;
@@ -1196,7 +1203,9 @@ const char* mlg_attention_kernels(int32_t nnei_max, int32_t channels, int32_t he
   if (R > 0 && n_layers <= kMaxFusedLayers) {
     if (dtype == MLG_F64) return nnei_max > R ? "k_attn_dmma + k_attn_generic" : "k_attn_dmma";
     if (kTcAttn && channels == 32 && D == 8 && n_layers == 1) {
-#if MLG_TC_ATTN == 6
+#if MLG_TC_ATTN == 7
+#define MLG_TC_NAME "k_attn_tc7 (tcgen05 logits, mma.sync P.V, rows <= 64)"
+#elif MLG_TC_ATTN == 6
 #define MLG_TC_NAME "k_attn_tc6 (tcgen05 logits, rows <= 64)"
 #elif MLG_TC_ATTN == 5
 #define MLG_TC_NAME "k_attn_tc5 (tcgen05 logits, rows <= 64)"

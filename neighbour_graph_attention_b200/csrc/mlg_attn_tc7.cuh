@@ -28,9 +28,10 @@
 //   projection  D[128 x 96] = X[128 x 32] . [Wq|Wk|Wv], 3xTF32 (12 MMAs)
 //   read-back   group h reads its head's q (scaled by s_a log2(e)/sqrt(d))
 //               and k (scaled by s_b) back and splits them into TF32 hi / lo
-//               K-major shared-memory operands: q into the operand of its
-//               row's centre (the other centre's operand gets a zero row), k
-//               into its centre's key operand at the key's slot; v as fp32
+//               operands: q into TMEM, the A operand of its row's centre
+//               (the other centre's operand gets a zero row), k into its
+//               centre's K-major shared-memory key operand at the key's
+//               slot; v as fp32
 //               rows with the two keys of a pair interleaved (two buffers
 //               per head, alternating between tiles)
 //   logits      per head, as soon as its group has read back: for each
@@ -90,6 +91,9 @@ using tc2::centre_of_group;
 using tc2::ex2;
 using tc2::idesc_tf32;
 using tc2::mbar_arrive;
+using tc2::tmem_st16;
+using tc2::tmem_wait_st;
+using tc2::umma_tf32_ts;
 
 constexpr int C = 32, D = 8, H = 4, N3 = 96, R = 128;
 constexpr int MAXN = 64;        // most edges of a centre handled here
@@ -101,26 +105,23 @@ constexpr int VS2 = 2 * C + 4;  // floats per key pair of V: [head][t][2 keys], 
 // TMEM columns (512 allocated)
 constexpr uint32_t T_PROJ = 0;    // projection D: q 0-31, k 32-63, v 64-95
 constexpr uint32_t T_S = 128;     // logits of head h: T_S + 64 h, [128 rows x 64 keys]
+constexpr uint32_t T_Q = 384;     // q operands of head h: T_Q + 32 h + 16 c + 8 m
+                                  // (centre c, m 0 hi / 1 lo), [128 rows x 8]
 
 // shared memory layout (bytes)
 constexpr size_t W_BYTES = (size_t)N3 * C * 4;          // one of W hi / lo (B operand)
 constexpr size_t A_BYTES = (size_t)R * C * 4;           // one of X hi / lo, the raw slab
-constexpr size_t Q_BYTES = (size_t)R * D * 4;           // one (head, centre) q operand, hi or lo
 constexpr size_t K_BYTES = (size_t)MAXN * D * 4;        // one (head, centre) k operand, hi or lo
 constexpr size_t V_BYTES = (size_t)(R / 2) * VS2 * 4;   // one V buffer
 constexpr size_t OFF_WHI = 0;
 constexpr size_t OFF_WLO = OFF_WHI + W_BYTES;
 constexpr size_t OFF_X = OFF_WLO + W_BYTES;             // 2 slabs (TMA targets, A hi)
 constexpr size_t OFF_ALO = OFF_X + 2 * A_BYTES;         // A lo of the next projection
-constexpr size_t OFF_Q = OFF_ALO + A_BYTES;             // [head][centre][hi, lo]
-constexpr size_t OFF_K = OFF_Q + 4 * H * Q_BYTES;       // [head][centre][hi, lo]
+constexpr size_t OFF_K = OFF_ALO + A_BYTES;             // [head][centre][hi, lo]
 constexpr size_t OFF_V = OFF_K + 4 * H * K_BYTES;       // 2 x [64 key pairs][VS2] fp32
 constexpr size_t OFF_META = OFF_V + 2 * V_BYTES;
 
 // operand of (head h, centre c, part m: 0 hi, 1 lo)
-__host__ __device__ constexpr size_t q_off(int h, int c, int m) {
-  return OFF_Q + (size_t)((h * 2 + c) * 2 + m) * Q_BYTES;
-}
 __host__ __device__ constexpr size_t k_off(int h, int c, int m) {
   return OFF_K + (size_t)((h * 2 + c) * 2 + m) * K_BYTES;
 }
@@ -180,6 +181,20 @@ __device__ __forceinline__ void mma_f16(float* d, const uint32_t* a, uint32_t b0
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// (p0, p1) in [0, 1] -> fp16x2 hi and lo, p = hi + lo: hi is p rounded to a
+// multiple of 2^-11 by adding and removing 2^12 (exact in fp16), lo the rest
+// (|lo| <= 2^-12, rounded to fp16: at most 2^-25 off)
+__device__ __forceinline__ void split_p_f16x2(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  const float2 c = make_float2(4096.f, 4096.f), nc = make_float2(-4096.f, -4096.f);
+  const float2 p = make_float2(p0, p1);
+  const float2 h = __fadd2_rn(__fadd2_rn(p, c), nc);
+  const float2 l = __fadd2_rn(p, make_float2(-h.x, -h.y));
+  const __half2 hh = __floats2half2_rn(h.x, h.y);
+  const __half2 ll = __floats2half2_rn(l.x, l.y);
+  hi = *reinterpret_cast<const uint32_t*>(&hh);
+  lo = *reinterpret_cast<const uint32_t*>(&ll);
 }
 
 // the TF32 part of x as the tensor core reads it: its leading 19 bits
@@ -357,13 +372,12 @@ __global__ void __launch_bounds__(tc7::NT, 1)
         const uint32_t id = idesc_tf32(R, (nmax + 15) & ~15);
         const uint32_t d = tmem + T_S + 64u * (uint32_t)h;
         for (int c = 0; c < p.ncent; ++c) {
-          const uint64_t dqh = umma_sdesc(smem_u32(sm + q_off(h, c, 0)), R * 16, 128);
-          const uint64_t dql = umma_sdesc(smem_u32(sm + q_off(h, c, 1)), R * 16, 128);
+          const uint32_t qh = tmem + T_Q + 32u * (uint32_t)h + 16u * (uint32_t)c, ql = qh + 8u;
           const uint64_t dkh = umma_sdesc(smem_u32(sm + k_off(h, c, 0)), MAXN * 16, 128);
           const uint64_t dkl = umma_sdesc(smem_u32(sm + k_off(h, c, 1)), MAXN * 16, 128);
-          umma_tf32(d, dql, dkh, id, c > 0 ? 1u : 0u);
-          umma_tf32(d, dqh, dkl, id, 1u);
-          umma_tf32(d, dqh, dkh, id, 1u);
+          umma_tf32_ts(d, ql, dkh, id, c > 0 ? 1u : 0u);
+          umma_tf32_ts(d, qh, dkl, id, 1u);
+          umma_tf32_ts(d, qh, dkh, id, 1u);
         }
         umma_commit(&mt.bar_s[h]);
       };
@@ -482,28 +496,30 @@ __global__ void __launch_bounds__(tc7::NT, 1)
         tmem_ld8(tmem + lane_addr + T_PROJ + 32u + 8u * h, v + 8);
         tmem_ld8(tmem + lane_addr + T_PROJ + 64u + 8u * h, v + 16);
         tmem_wait_ld();
-        // q (scaled by s_a log2(e)/sqrt(d)) into its centre's operand, a zero
-        // row into the other's
+        // q (scaled by s_a log2(e)/sqrt(d)), hi and lo, into its centre's
+        // TMEM operand (A of the logits), a zero row into the other's
         {
           const float fq = (float)ri.sw * qscale;
-          float4 xh[2], xl[2];
+          uint32_t qv[16], zv[16];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float x = __uint_as_float(v[j]) * fq;
             const float hi = tf32_rna(x);
-            reinterpret_cast<float*>(xh)[j] = hi;
-            reinterpret_cast<float*>(xl)[j] = tf32_rna(x - hi);
+            qv[j] = __float_as_uint(hi);
+            qv[8 + j] = __float_as_uint(tf32_rna(x - hi));
+            zv[j] = zv[8 + j] = 0u;
           }
-          const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const bool mine = c == ri.cw;
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-              const uint32_t off = kmajor_offset(row, 4 * ch, R);
-              *reinterpret_cast<float4*>(sm + q_off(h, c, 0) + off) = mine ? xh[ch] : z;
-              *reinterpret_cast<float4*>(sm + q_off(h, c, 1) + off) = mine ? xl[ch] : z;
-            }
+          // the warp's centre is the same for all its threads
+          const uint32_t qa = tmem + lane_addr + T_Q + 32u * (uint32_t)h;
+          if (ri.cw == 0) {
+            tmem_st16(qa, qv);
+            tmem_st16(qa + 16u, zv);
+          } else if (ri.cw == 1) {
+            tmem_st16(qa, zv);
+            tmem_st16(qa + 16u, qv);
+          } else {
+            tmem_st16(qa, zv);
+            tmem_st16(qa + 16u, zv);
           }
         }
         // k (scaled by s_b, kept finite) into its centre's key operand
@@ -537,6 +553,7 @@ __global__ void __launch_bounds__(tc7::NT, 1)
         const uint32_t vb = __reduce_max_sync(0xffffffffu, __float_as_uint(vm));
         if (lane == 0) mt.vmax[h][t & 1][quad] = vb;
         fence_proxy_async();
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&mt.bar_qk[h]);
       }
@@ -650,8 +667,8 @@ __global__ void __launch_bounds__(tc7::NT, 1)
               l0 = __fadd2_rn(l0, p0);
               l1 = __fadd2_rn(l1, p1);
               // a0a1 / a4a5: row g; a2a3 / a6a7: row g + 8
-              split_f16x2(p0.x, p0.y, ah[2 * hf], al[2 * hf]);
-              split_f16x2(p1.x, p1.y, ah[2 * hf + 1], al[2 * hf + 1]);
+              split_p_f16x2(p0.x, p0.y, ah[2 * hf], al[2 * hf]);
+              split_p_f16x2(p1.x, p1.y, ah[2 * hf + 1], al[2 * hf + 1]);
             }
             mma_f16(o, ah, bh[kb][0], bh[kb][1]);
             mma_f16(oc, ah, bl[kb][0], bl[kb][1]);
@@ -671,11 +688,11 @@ __global__ void __launch_bounds__(tc7::NT, 1)
           // rows g and g + 8: columns 2c, 2c + 1 of the head (8 bytes; a
           // quad writes the head's whole 32-byte sector of the row)
           if (ra - ri.key0 < nrow) {
-            const float r0 = vunscale / s0;
+            const float r0 = __fdividef(vunscale, s0);
             *reinterpret_cast<float2*>(dst + (ri.obase + ra) * C) = make_float2(o[0] * r0, o[1] * r0);
           }
           if (ra + 8 - ri.key0 < nrow) {
-            const float r1 = vunscale / s1;
+            const float r1 = __fdividef(vunscale, s1);
             *reinterpret_cast<float2*>(dst + (ri.obase + ra + 8) * C) = make_float2(o[2] * r1, o[3] * r1);
           }
         }

@@ -495,7 +495,8 @@ def main(argv=None):
     abytes = attention_bytes(w.n_atoms, E, w.channels, elem) + \
         (w.n_layers - 1) * 3.0 * w.channels * w.channels * elem
     kernels = m.mlg_attention_kernels(w.nnei_max, w.channels, w.heads, w.n_layers, mdt)
-    kname = kernels if not local else "k_local_attn"
+    kname = kernels if not local else (
+        "k_local_attn_w32" if w.channels == 32 and w.heads in (1, 2, 4, 8) else "k_local_attn")
     rec_k, traffic = ATTN_TRAFFIC.get(w.key, ("", None))
     if rec_k != kname or args.variant != "block":
         traffic = None

@@ -1099,6 +1099,31 @@ int mlg_local_attention(const mlg_csr* csr, int64_t n_centres, int32_t nnei_max,
     kern<<<grid, kLocalThreads, smem, st>>>(la);
     return launch_status();
   };
+  // 32 channels: one warp per centre
+  auto go_w32 = [&](auto kern, size_t smem) {
+    if (smem > 227 * 1024) return (int)MLG_ERR_UNSUPPORTED;
+    prefer_shared(kern, smem);
+    if (cudaGetLastError() != cudaSuccess) return (int)MLG_ERR_CUDA;
+    const int nt = kLocalW32Warps * 32;
+    const int64_t want = (int64_t)resident_blocks(kern, nt, smem) * sm_count();
+    const int64_t need = (n_centres + kLocalW32Warps - 1) / kLocalW32Warps;
+    const int grid = (int)(need < want ? need : want);
+    kern<<<grid < 1 ? 1 : grid, nt, smem, st>>>(la);
+    return launch_status();
+  };
+  if (channels == 32 && (heads == 1 || heads == 2 || heads == 4 || heads == 8)) {
+    const bool f64 = dtype == MLG_F64;
+    switch (heads) {
+      case 1: return f64 ? go_w32(k_local_attn_w32<double, 1>, local_w32_smem<double, 1>(nnei_max))
+                         : go_w32(k_local_attn_w32<float, 1>, local_w32_smem<float, 1>(nnei_max));
+      case 2: return f64 ? go_w32(k_local_attn_w32<double, 2>, local_w32_smem<double, 2>(nnei_max))
+                         : go_w32(k_local_attn_w32<float, 2>, local_w32_smem<float, 2>(nnei_max));
+      case 4: return f64 ? go_w32(k_local_attn_w32<double, 4>, local_w32_smem<double, 4>(nnei_max))
+                         : go_w32(k_local_attn_w32<float, 4>, local_w32_smem<float, 4>(nnei_max));
+      default: return f64 ? go_w32(k_local_attn_w32<double, 8>, local_w32_smem<double, 8>(nnei_max))
+                          : go_w32(k_local_attn_w32<float, 8>, local_w32_smem<float, 8>(nnei_max));
+    }
+  }
   if (dtype == MLG_F64)
     return go(k_local_attn<double>, local_smem<double>(channels, heads, nnei_max));
   return go(k_local_attn<float>, local_smem<float>(channels, heads, nnei_max));

@@ -199,7 +199,24 @@ __global__ void __launch_bounds__(NT) k_attn_tc(TileArgs a, const __grid_constan
   auto plan_and_load = [&](int b) {
       int c = meta.next_c, k = 0, rows = 0, tasks = 0;
       const int c_end = meta.c_end;
+      // skip to the next centre this kernel takes, 16 row starts per step so
+      // that their loads go out together (with a lower row bound most
+      // centres are left to another kernel)
       while (c < c_end) {
+        if (c + 16 <= c_end) {
+          long long rp[17];
+#pragma unroll
+          for (int u = 0; u <= 16; ++u) rp[u] = a.row_ptr[c + u];
+          int u = 0;
+          for (; u < 16; ++u) {
+            const int n = (int)(rp[u + 1] - rp[u]);
+            if (n > a.min_n && n <= R && n <= a.nnei_max) break;
+            if (n > a.nnei_max) atomicOr(a.status, (uint32_t)MLG_STATUS_ROW_TOO_LONG);
+          }
+          c += u;
+          if (u < 16) break;
+          continue;
+        }
         const int n = (int)(a.row_ptr[c + 1] - a.row_ptr[c]);
         if (n > a.min_n && n <= R && n <= a.nnei_max) break;
         if (n > a.nnei_max) atomicOr(a.status, (uint32_t)MLG_STATUS_ROW_TOO_LONG);

@@ -388,15 +388,29 @@ __global__ void __launch_bounds__(tc7::NT, 1)
         issue_proj(0);
       }
       for (int t = 0; ok && p.ncent > 0; ++t) {
-        // head h as soon as group h has read it back (the group's read-back
-        // follows its softmax of the previous tile, so the buffer is free)
+        // each head's logits as soon as its group has read it back (the
+        // group's read-back follows its softmax of the previous tile, so the
+        // buffer is free), in the order the groups get there
+        {
+          uint32_t done = 0;
+          const uint64_t t0 = globaltimer_ns();
+          while (done != (1u << H) - 1u) {
+            bool any = false;
 #pragma unroll
-        for (int h = 0; h < H; ++h) {
-          if (!ok) break;
-          ok = wqk[h].wait(&mt.bar_qk[h]);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(h, p);
+            for (int h = 0; h < H; ++h) {
+              if (!(done & (1u << h)) && mbar_test(&mt.bar_qk[h], wqk[h].par)) {
+                wqk[h].par ^= 1u;
+                tc_fence_after();
+                issue_s(h, p);
+                done |= 1u << h;
+                any = true;
+              }
+            }
+            if (!any) {
+              if (globaltimer_ns() - t0 > 1000000000ull) { ok = false; break; }
+              __nanosleep(32);
+            }
+          }
         }
         if (!ok) break;
         // the next tile's projection: every group has read this tile's back

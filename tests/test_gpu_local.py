@@ -76,7 +76,11 @@ def test_local_largest_system_sampled_centres():
     assert ok, err
 
 
-@pytest.mark.parametrize("dtype,channels,heads", [("f64", 32, 4), ("f32", 128, 8)])
+@pytest.mark.parametrize("dtype,channels,heads", [
+    ("f64", 32, 4), ("f32", 128, 8),
+    # the warp-per-centre kernel of 32 channels at every head count it takes
+    ("f32", 32, 1), ("f64", 32, 2), ("f32", 32, 8),
+])
 def test_local_empty_rows_and_ones(dtype, channels, heads):
     """A dilute random graph (many centres without edges: zero rows) and all
     value vectors equal to ones (every other row exactly a weighted mean of

@@ -140,7 +140,11 @@ typedef struct {
 
 /* Bytes of device workspace that mlg_build_csr needs for this system.  The
  * cell grid depends on N, rcut, the box and pbc (not on the coordinates).
- * Returns 0 for invalid arguments. */
+ * For systems built by the kernel chain (more than 4,096 atoms, or narrow
+ * boxes aside) the size includes 516 bytes per atom in which the count pass
+ * keeps the accepted keys of every row of at most 64 of them, so that the
+ * fill pass does not search the stencil again.  Returns 0 for invalid
+ * arguments. */
 size_t mlg_build_csr_workspace_bytes(int64_t n_atoms, double rcut, const double box[9],
                                      const uint8_t pbc[3]);
 
@@ -325,8 +329,9 @@ int mlg_verlet_step(const mlg_system* sys, double rcut, double r_on, double skin
  *   - Same arguments, results and device status as mlg_build_csr; the CSR
  *     output buffers are still the caller's.
  *   - Returns MLG_ERR_WORKSPACE, launching nothing, when the system needs more
- *     scratch than the array holds (mlg_build_csr_workspace_bytes() >
- *     MLG_NOALLOC_SCRATCH_BYTES; about 150,000 atoms for a periodic box).
+ *     scratch than the array holds (about 150,000 atoms for a periodic box).
+ *     The array build goes without the count-to-fill key stash that
+ *     mlg_build_csr_workspace_bytes() counts.
  *   - The first call on a device looks up the array's device address (with
  *     that device current) and caches it with the current context; make that
  *     first call before any stream capture begins.  A later call under a new

@@ -40,6 +40,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct BuildLayout {
   size_t grid, bbox, cell_count, cell_start, atom_cell, atom_rank, atom_w, recs, pos4, kept, raw,
       partial, sync, total;
+  size_t stash, stash_n, total_stash;  // the count-to-fill key stash after `total`
 };
 
 int64_t scan_tiles(int64_t n) { return (n + kScanTile - 1) / kScanTile; }
@@ -67,6 +68,9 @@ BuildLayout build_layout(int64_t n, int ncell_cap) {
   L.partial = take((size_t)(tiles + 2) * sizeof(long long));
   L.sync = take(sizeof(FusedSync));
   L.total = off;
+  L.stash = take((size_t)n * kStashSlots * sizeof(unsigned long long));
+  L.stash_n = take((size_t)n * sizeof(int));
+  L.total_stash = off;
   return L;
 }
 
@@ -315,6 +319,8 @@ BuildArgs make_build_args(const mlg_system* sys, double rcut, double r_on, int32
   a.kept = reinterpret_cast<int*>(w + L.kept);
   a.raw = reinterpret_cast<int*>(w + L.raw);
   a.partial = reinterpret_cast<long long*>(w + L.partial);
+  a.stash = nullptr;
+  a.stash_n = nullptr;
   return a;
 }
 
@@ -351,7 +357,13 @@ void launch_count_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
   launch_scan<int>(a.cell_count, plan.ncell_cap, a.cell_start, a.partial,
                    ScanTail{nullptr, nullptr, 0, a.gate}, stream);
   k_scatter<<<atom_blocks, tb, 0, stream>>>(a);
-  if (plan.max_reach <= 1) {
+  if (plan.max_reach <= 1 && a.stash != nullptr) {
+    // the count keeps each whole row's keys (its warps collect them)
+    const size_t sm_count_ = cellscan_smem(true);
+    prefer_shared(k_cellscan<false, true>, sm_count_);
+    k_cellscan<false, true><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kScanWarps * 32,
+                              sm_count_, stream>>>(a);
+  } else if (plan.max_reach <= 1) {
     const size_t sm_count_ = cellscan_smem(false);
     prefer_shared(k_cellscan<false>, sm_count_);
     k_cellscan<false><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kScanWarps * 32,
@@ -364,7 +376,12 @@ void launch_count_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
 // The fill, once row_ptr holds the row starts.
 void launch_fill_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
                        cudaStream_t stream) {
-  if (plan.max_reach <= 1) {
+  if (plan.max_reach <= 1 && a.stash != nullptr) {
+    const size_t sm_fill = cellscan_smem(true);
+    prefer_shared(k_cellscan<true, true>, sm_fill);
+    k_cellscan<true, true><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kScanWarps * 32,
+                             sm_fill, stream>>>(a);
+  } else if (plan.max_reach <= 1) {
     const size_t sm_fill = cellscan_smem(true);
     prefer_shared(k_cellscan<true>, sm_fill);
     k_cellscan<true><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kScanWarps * 32,
@@ -435,6 +452,11 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
     if (!use_fused_build(plan, n)) return MLG_ERR_UNSUPPORTED;
     a.spin_polls = opt.polls;
     a.hold_release = opt.hold_release;
+  }
+  // the key stash of the count-to-fill chain, when the workspace holds it
+  if (!use_fused_build(plan, n) && plan.max_reach <= 1 && ws_bytes >= L.total_stash) {
+    a.stash = reinterpret_cast<unsigned long long*>(w + L.stash);
+    a.stash_n = reinterpret_cast<int*>(w + L.stash_n);
   }
   if (use_fused_build(plan, n)) {
     // the whole build in one cooperative launch (small systems); systems of
@@ -1020,7 +1042,9 @@ size_t mlg_build_csr_workspace_bytes(int64_t n_atoms, double rcut, const double 
                                      const uint8_t pbc[3]) {
   BuildPlan plan;
   if (make_plan(n_atoms, rcut, box, pbc, &plan) != MLG_OK) return 0;
-  return build_layout(n_atoms, plan.ncell_cap).total;
+  const BuildLayout L = build_layout(n_atoms, plan.ncell_cap);
+  // the key stash only where the kernel chain with per-cell scans runs
+  return !use_fused_build(plan, n_atoms) && plan.max_reach <= 1 ? L.total_stash : L.total;
 }
 
 int mlg_build_csr(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max,
@@ -1383,7 +1407,14 @@ extern "C" int mlg_build_csr_noalloc(const mlg_system* sys, double rcut, double 
                                      int32_t nnei_max, const mlg_csr* csr,
                                      mlg_stream_t stream) {
   if (sys == nullptr) return MLG_ERR_INVALID_ARG;
-  const size_t need = mlg_build_csr_workspace_bytes(sys->n_atoms, rcut, sys->box, sys->pbc);
+  // what the build cannot do without (the array holds no key stash for
+  // systems this size; the fill then searches the stencil again)
+  size_t need = 0;
+  {
+    BuildPlan plan;
+    if (make_plan(sys->n_atoms, rcut, sys->box, sys->pbc, &plan) == MLG_OK)
+      need = build_layout(sys->n_atoms, plan.ncell_cap).total;
+  }
   if (need == 0)  // invalid arguments: let the regular checks name the error
     return build_impl(sys, rcut, r_on, nnei_max, csr, nullptr, 0, (cudaStream_t)stream);
   if (need > kNoAllocScratchBytes) return MLG_ERR_WORKSPACE;  // system too large for the array

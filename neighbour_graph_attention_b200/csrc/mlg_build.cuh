@@ -115,6 +115,9 @@ struct BuildArgs {
   int* kept;                 // [n]
   int* raw;                  // [n]
   long long* partial;        // scan partials
+  unsigned long long* stash; // [n][kStashSlots] accepted keys of each row the count
+                             // could keep whole (nullptr: none; the fill searches again)
+  int* stash_n;              // [n] keys in the row's stash, -1: not stashed
 };
 
 // False when the build is gated off by a device word (uniform for a launch:
@@ -124,6 +127,10 @@ __device__ __forceinline__ bool gated_off(const uint32_t* gate) {
 }
 
 constexpr int kFillMaxCand = 256;  // shared-memory candidates per destination
+// Rows of at most kStashSlots accepted candidates (and no truncation) keep
+// their keys from the count to the fill, which then sorts and writes them
+// without searching the stencil again.
+constexpr int kStashSlots = 64;
 constexpr int kCountWarps = 8;
 constexpr int kFillWarps = 4;
 
@@ -964,7 +971,8 @@ __host__ __device__ constexpr size_t cellscan_smem(bool fill, bool rec = false) 
 // the same cell from an earlier call are reused.  With STASH (and REC) the
 // count keeps each warp's accepted keys and distances in its key buffer, and
 // a fill of the same centre by the same warp starts from them.
-template <bool FILL, bool REC, bool STASH = false, int CAP = kCellCand, int NW = kCellWarps>
+template <bool FILL, bool REC, bool STASH = false, int CAP = kCellCand, int NW = kCellWarps,
+          bool GST = false>
 __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratch* sws,
                               unsigned char* s_dyn, int cell, int ys, int nsplit,
                               const int* row_off) {
@@ -979,6 +987,44 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
   const int c_hi = reuse ? cs.c_hi : a.cell_start[cell + 1];
   if (c_lo + ys * NW >= c_hi) return;
   const int cz = cell % sg.n[2], cy = (cell / sg.n[2]) % sg.n[1], cx = cell / (sg.n[2] * sg.n[1]);
+  // (GST fill) a row is stashed when the count kept all its accepted keys
+  auto stashed = [&](int i) { return a.stash_n[i] >= 0; };
+  if (GST && FILL) {
+    // the stashed rows of this split's centres, straight from the count's
+    // keys: sort and write; the stencil is staged only if a row is left
+    unsigned long long* wkeys =
+        reinterpret_cast<unsigned long long*>(s_dyn + CellSmem<CAP, NW>::keys_off) +
+        (size_t)warp * 2 * kFillMaxCand;
+    uint32_t st0 = 0;
+    int left = 0;
+    for (int ci = c_lo + ys * NW + warp; ci < c_hi; ci += nsplit * NW) {
+      const Rec rci = a.recs[ci];
+      const int i = rci.j;
+      if (!stashed(i)) {
+        left = 1;
+        continue;
+      }
+      const int n = a.stash_n[i];
+      if (n == 0) continue;
+      for (int q = lane; q < n; q += 32) wkeys[q] = a.stash[(int64_t)i * kStashSlots + q];
+      __syncwarp();
+      Centre cc;
+      cc.i = i;
+      cc.x[0] = rci.x;
+      cc.x[1] = rci.y;
+      cc.x[2] = rci.z;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) cc.w[k] = unpack_w(rci.w, k);
+      cc.c[0] = cx;
+      cc.c[1] = cy;
+      cc.c[2] = cz;
+      st0 |= finish_row(a, cc, wkeys, wkeys + kFillMaxCand, n, n, a.row_ptr[i], nullptr);
+      __syncwarp();
+    }
+    st0 = __reduce_or_sync(kFull, st0);
+    if (lane == 0 && st0) atomicOr(a.status, st0);
+    if (!__syncthreads_or(left)) return;
+  }
   if (!reuse) {
     __syncthreads();  // earlier readers of the staging arrays are done
     if (warp == 0) {
@@ -1113,6 +1159,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
           a.raw[i] = cnt;
           a.kept[i] = cnt < a.nnei_max ? cnt : a.nnei_max;
           if (cnt > a.nnei_max) atomicAdd(&cs.trunc, 1);
+          if (GST) a.stash_n[i] = -1;   // the fill searches again
         }
       } else {
         const int n = a.kept[i];
@@ -1128,6 +1175,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
       if (n > 0) st |= finish_row(a, cc, keys, keys + kFillMaxCand, n, raw, p0, s_rec);
       continue;
     }
+    if (GST && FILL && stashed(i)) continue;   // written from the stash above
     const int n = FILL ? a.kept[i] : 0;
     if (FILL && n == 0) continue;
     if (STASH) {
@@ -1136,7 +1184,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
     }
     const float4 pi = staged_self ? cs.cand[self_slot] : a.pos4[ci];
     const bool need_d2 = FILL && a.raw[i] > n;
-    constexpr bool kCollect = FILL || STASH;
+    constexpr bool kCollect = FILL || STASH || GST;
     int cnt = 0;
     // the candidates, two per lane per step (slots t0 and t0 + 32 of a block
     // of 64); the fp32 prefilter decides all but the few within its margin of
@@ -1206,6 +1254,16 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
           cs.stash_cnt[warp] = cnt;
         }
       }
+      if (GST) {
+        // the row's keys for the fill (any order: the fill sorts them)
+        const bool whole = cnt <= kStashSlots && cnt <= a.nnei_max;
+        if (whole) {
+          __syncwarp();
+          for (int q = lane; q < cnt; q += 32) a.stash[(int64_t)i * kStashSlots + q] = keys[q];
+          __syncwarp();   // the next centre's keys go to the same buffer
+        }
+        if (lane == 0) a.stash_n[i] = whole ? cnt : -1;
+      }
     } else {
       __syncwarp();
       if (cnt > kFillMaxCand) {
@@ -1226,7 +1284,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
   }
 }
 
-template <bool FILL>
+template <bool FILL, bool GST = false>
 __global__ void __launch_bounds__(kScanWarps * 32, FILL ? MLG_FILL_MINB : MLG_COUNT_MINB)
     k_cellscan(BuildArgs a) {
   if (gated_off(a.gate)) return;
@@ -1239,8 +1297,8 @@ __global__ void __launch_bounds__(kScanWarps * 32, FILL ? MLG_FILL_MINB : MLG_CO
   }
   __syncthreads();
   // blockIdx.y splits a cell's centres over several CTAs (small grids)
-  cellscan_item<FILL, false, false, kCellCand, kScanWarps>(a, sg, sws, s_dyn, blockIdx.x,
-                                                           blockIdx.y, gridDim.y, nullptr);
+  cellscan_item<FILL, false, false, kCellCand, kScanWarps, GST>(a, sg, sws, s_dyn, blockIdx.x,
+                                                                blockIdx.y, gridDim.y, nullptr);
 }
 
 // ------------------------------------------------------------------ scans

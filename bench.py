@@ -52,6 +52,10 @@ SFU_PEAK_TEXP = SM_COUNT * 16 * SM_MAX_GHZ / 1e3
 # entry.
 ATTN_TRAFFIC = {
     2: ("k_attn_dmma", 5.622e6),   # profiles/k_attn_dmma_f64_diamond512.md
+    # profiles/k_attn_tc7_fe_bcc_65536.md: 1,077 MB per launch at 65,536 atoms
+    # (4,194,304 edges), scaled by the edges to 33,554,436
+    5: ("k_attn_tc7 (tcgen05 logits, mma.sync P.V, rows <= 64) + k_attn_tc (rows <= 128)",
+        1.0769e9 * 33554436 / 4194304),
 }
 
 

@@ -17,9 +17,6 @@
 #include "mlg_attn_dmma.cuh"
 #include "mlg_attn_tc.cuh"
 #include "mlg_attn_tc2.cuh"
-#include "mlg_attn_tc3.cuh"
-#include "mlg_attn_tc4.cuh"
-#include "mlg_attn_tc5.cuh"
 #include "mlg_attn_tc6.cuh"
 #include "mlg_attn_tc7.cuh"
 #include "mlg_attn_hgtc.cuh"
@@ -679,14 +676,12 @@ int launch_tc(TileArgs& ta, cudaStream_t stream) {
 }
 
 // fp32, 32 channels, 4 heads, one layer, centres of up to 64 edges: one CTA
-// per SM holding all of its TMEM.  Which kernel takes fp32 rows of up to 64 edges at 32 channels, 4 heads,
-// one layer: 0 = the tile kernel of every fp32 row (logits and P V on the
-// FP32 pipe), 2 = every product on tcgen05, 3 = the logits on tcgen05 (two
-// groups of warps), 4 = the logits on tcgen05 (one group of warps per head),
-// 5 = as 4 with each group reading back its own head, 6 = as 5 with one
-// logits buffer of 64 columns per head (no buffer shared between heads),
-// 7 = as 6 with P V on warp-level tensor-core MMAs and the slabs planned and
-// loaded two tiles ahead.
+// per SM holding all of its TMEM.  Which kernel takes these rows (a build-time
+// choice for A/B runs): 0 = the tile kernel of every fp32 row (logits and P V
+// on the FP32 pipe), 2 = every product on tcgen05, 6 = the logits on tcgen05
+// with one 64-column TMEM buffer per head and P V on the FP32 pipe, 7 = as 6
+// with P V on warp-level tensor-core MMAs and the slabs planned and loaded two
+// tiles ahead.
 #ifndef MLG_TC_ATTN
 #define MLG_TC_ATTN 7
 #endif
@@ -700,18 +695,6 @@ int launch_tc2(TileArgs& ta, cudaStream_t stream) {
   auto kern = k_attn_tc6;
   const size_t smem = tc6::SMEM;
   const int nt = tc6::NT;
-#elif MLG_TC_ATTN == 5
-  auto kern = k_attn_tc5;
-  const size_t smem = tc5::SMEM;
-  const int nt = tc5::NT;
-#elif MLG_TC_ATTN == 4
-  auto kern = k_attn_tc4;
-  const size_t smem = tc4::SMEM;
-  const int nt = tc4::NT;
-#elif MLG_TC_ATTN == 3
-  auto kern = k_attn_tc3;
-  const size_t smem = tc3::SMEM;
-  const int nt = tc3::NT;
 #else
   auto kern = k_attn_tc2;
   const size_t smem = tc2::SMEM;
@@ -1256,12 +1239,6 @@ const char* mlg_attention_kernels(int32_t nnei_max, int32_t channels, int32_t he
 #define MLG_TC_NAME "k_attn_tc7 (tcgen05 logits, mma.sync P.V, rows <= 64)"
 #elif MLG_TC_ATTN == 6
 #define MLG_TC_NAME "k_attn_tc6 (tcgen05 logits, rows <= 64)"
-#elif MLG_TC_ATTN == 5
-#define MLG_TC_NAME "k_attn_tc5 (tcgen05 logits, rows <= 64)"
-#elif MLG_TC_ATTN == 4
-#define MLG_TC_NAME "k_attn_tc4 (tcgen05 logits, rows <= 64)"
-#elif MLG_TC_ATTN == 3
-#define MLG_TC_NAME "k_attn_tc3 (tcgen05 logits, rows <= 64)"
 #else
 #define MLG_TC_NAME "k_attn_tc2 (tcgen05 logits and P.V, rows <= 64)"
 #endif

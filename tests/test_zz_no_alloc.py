@@ -74,7 +74,7 @@ def test_noalloc_allocates_nothing_after_setup():
 
 def test_noalloc_rejects_systems_beyond_the_array():
     m = U.mlg()
-    w = C.workload(5)                       # 524,288 atoms: needs about 27 MB of scratch
+    w = C.workload(5)                       # 524,288 atoms: about 27 MB without the key stash
     s = C.system(5, 0)
     need = m.mlg_build_csr_workspace_bytes(w.n_atoms, w.rcut, s["box"], s["pbc"])
     assert need > m.MLG_NOALLOC_SCRATCH_BYTES

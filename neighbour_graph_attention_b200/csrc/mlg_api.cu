@@ -355,8 +355,8 @@ void launch_count_phase(const BuildArgs& a, const BuildPlan& plan, int nsplit,
                    ScanTail{nullptr, nullptr, 0, a.gate}, stream);
   k_scatter<<<atom_blocks, tb, 0, stream>>>(a);
   if (plan.max_reach <= 1 && a.stash != nullptr) {
-    // the count keeps each whole row's keys (its warps collect them)
-    const size_t sm_count_ = cellscan_smem(true);
+    // the count keeps each whole row's keys in the workspace stash
+    const size_t sm_count_ = cellscan_smem(false);
     prefer_shared(k_cellscan<false, true>, sm_count_);
     k_cellscan<false, true><<<dim3((unsigned)plan.ncell_cap, (unsigned)nsplit), kScanWarps * 32,
                               sm_count_, stream>>>(a);

@@ -1184,7 +1184,11 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
     }
     const float4 pi = staged_self ? cs.cand[self_slot] : a.pos4[ci];
     const bool need_d2 = FILL && a.raw[i] > n;
-    constexpr bool kCollect = FILL || STASH || GST;
+    constexpr bool kCollect = FILL || STASH;
+    // (GST count) each lane's accepted candidates as bits: bit 2 s + u for slot
+    // 64 s + lane + 32 u; the keys are formed once the row is known to fit
+    constexpr bool kMask = GST && !FILL;
+    uint32_t amask = 0;
     int cnt = 0;
     // the candidates, two per lane per step (slots t0 and t0 + 32 of a block
     // of 64); the fp32 prefilter decides all but the few within its margin of
@@ -1227,6 +1231,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
       }
       if (!kCollect) {
         cnt += (a0 ? 1 : 0) + (a1 ? 1 : 0);
+        if (kMask) amask |= ((a0 ? 1u : 0u) | (a1 ? 2u : 0u)) << (base >> 5);
       } else {
         collect(a0, t0, c0);
         collect(a1, t1, c1);
@@ -1244,6 +1249,7 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
       }
     }
     if (!FILL) {
+      const int lane_cnt = cnt;
       if (!kCollect) cnt = warp_sum(cnt);  // collecting lanes hold the warp total already
       if (lane == 0) {
         a.raw[i] = cnt;
@@ -1255,12 +1261,23 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
         }
       }
       if (GST) {
-        // the row's keys for the fill (any order: the fill sorts them)
+        // the row's keys for the fill (any order: the fill sorts them), each
+        // lane's after the lanes below it
         const bool whole = cnt <= kStashSlots && cnt <= a.nnei_max;
         if (whole) {
-          __syncwarp();
-          for (int q = lane; q < cnt; q += 32) a.stash[(int64_t)i * kStashSlots + q] = keys[q];
-          __syncwarp();   // the next centre's keys go to the same buffer
+          int q = lane_cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(kFull, q, o);
+            if (lane >= o) q += v;
+          }
+          q -= lane_cnt;   // exclusive
+          unsigned long long* dst = a.stash + (int64_t)i * kStashSlots;
+          for (uint32_t m = amask; m != 0; m &= m - 1) {
+            const int b = __ffs(m) - 1;
+            const int t = 32 * b + lane;   // slot 64 (b / 2) + 32 (b % 2) + lane
+            dst[q++] = edge_key(__float_as_int(cs.cand[t].w), cs.ct[t]);
+          }
         }
         if (lane == 0) a.stash_n[i] = whole ? cnt : -1;
       }

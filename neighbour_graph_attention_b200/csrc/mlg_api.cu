@@ -318,6 +318,7 @@ BuildArgs make_build_args(const mlg_system* sys, double rcut, double r_on, int32
   a.partial = reinterpret_cast<long long*>(w + L.partial);
   a.stash = nullptr;
   a.stash_n = nullptr;
+  a.stash_q = 0;
   return a;
 }
 
@@ -454,6 +455,7 @@ int build_impl(const mlg_system* sys, double rcut, double r_on, int32_t nnei_max
   if (!use_fused_build(plan, n) && plan.max_reach <= 1 && ws_bytes >= L.total_stash) {
     a.stash = reinterpret_cast<unsigned long long*>(w + L.stash);
     a.stash_n = reinterpret_cast<int*>(w + L.stash_n);
+    a.stash_q = n <= (int64_t(1) << 21) ? 1 : 0;
   }
   if (use_fused_build(plan, n)) {
     // the whole build in one cooperative launch (small systems); systems of

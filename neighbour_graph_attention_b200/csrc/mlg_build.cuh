@@ -118,6 +118,7 @@ struct BuildArgs {
   unsigned long long* stash; // [n][kStashSlots] accepted keys of each row the count
                              // could keep whole (nullptr: none; the fill searches again)
   int* stash_n;              // [n] keys in the row's stash, -1: not stashed
+  int stash_q;               // stash keys carry the source's cell-order record (n <= 2^21)
 };
 
 // False when the build is gated off by a device word (uniform for a launch:
@@ -680,6 +681,14 @@ __device__ __forceinline__ void warp_sort64_keys(unsigned long long& k0, unsigne
 
 // ------------------------------------------------------------------- fill
 
+// Stash key of a system of at most 2^21 atoms: source, packed image and the
+// source's cell-order record index (the order is that of edge_key: (j, image)
+// pairs are unique in a row, and the record follows from j).
+__device__ __forceinline__ unsigned long long stash_key(int j, int tpack, int q) {
+  return ((unsigned long long)j << 42) | ((unsigned long long)tpack << 21) |
+         (unsigned long long)q;
+}
+
 __device__ __forceinline__ unsigned long long edge_key(int j, int tpack) {
   return ((unsigned long long)(unsigned)j << 21) | (unsigned long long)tpack;
 }
@@ -766,10 +775,19 @@ __device__ int fill_overflow_select(const BuildArgs& a, const CellGrid& g, const
 // Writes edge p of centre cc for `key` (a staged_key() with srec, else an
 // edge_key()).
 __device__ __forceinline__ void write_edge(const BuildArgs& a, const Centre& cc,
-                                           unsigned long long key, int64_t p, const Rec* srec) {
+                                           unsigned long long key, int64_t p, const Rec* srec,
+                                           bool qkey = false) {
   int j, tp, wj;
   double xj[3];
-  if (srec != nullptr) {
+  if (qkey) {   // stash_key(): the source's record (one 32-byte sector)
+    j = (int)(key >> 42);
+    tp = (int)((key >> 21) & 0x1fffffull);
+    const Rec rc = a.recs[(int)(key & 0x1fffffull)];
+    wj = rc.w;
+    xj[0] = rc.x;
+    xj[1] = rc.y;
+    xj[2] = rc.z;
+  } else if (srec != nullptr) {
     j = staged_src(key);
     tp = staged_image(key);
     const Rec& rc = srec[staged_slot(key)];
@@ -815,7 +833,7 @@ __device__ __forceinline__ void write_edge(const BuildArgs& a, const Centre& cc,
 // registers.  Returns status bits.
 __device__ uint32_t finish_row(const BuildArgs& a, const Centre& cc, unsigned long long* keys,
                                unsigned long long* d2, int n, int m, int64_t p0,
-                               const Rec* srec = nullptr) {
+                               const Rec* srec = nullptr, bool qkey = false) {
   const int lane = lane_id();
   uint32_t st = 0;
   if (m > kFillMaxCand) m = kFillMaxCand;
@@ -832,13 +850,13 @@ __device__ uint32_t finish_row(const BuildArgs& a, const Centre& cc, unsigned lo
       if (lane + 32 >= nv) k1 = ~0ull;
     }
     warp_sort64_keys(k0, k1);
-    if (lane < nv) write_edge(a, cc, k0, p0 + lane, srec);
-    if (lane + 32 < nv) write_edge(a, cc, k1, p0 + lane + 32, srec);
+    if (lane < nv) write_edge(a, cc, k0, p0 + lane, srec, qkey);
+    if (lane + 32 < nv) write_edge(a, cc, k1, p0 + lane + 32, srec, qkey);
     return st;
   }
   if (m > n) warp_sort_pairs(d2, keys, m);
   warp_sort_keys(keys, nv);
-  for (int e = lane; e < nv; e += 32) write_edge(a, cc, keys[e], p0 + e, srec);
+  for (int e = lane; e < nv; e += 32) write_edge(a, cc, keys[e], p0 + e, srec, qkey);
   return st;
 }
 
@@ -1018,7 +1036,8 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
       cc.c[0] = cx;
       cc.c[1] = cy;
       cc.c[2] = cz;
-      st0 |= finish_row(a, cc, wkeys, wkeys + kFillMaxCand, n, n, a.row_ptr[i], nullptr);
+      st0 |= finish_row(a, cc, wkeys, wkeys + kFillMaxCand, n, n, a.row_ptr[i], nullptr,
+                        a.stash_q != 0);
       __syncwarp();
     }
     st0 = __reduce_or_sync(kFull, st0);
@@ -1276,7 +1295,8 @@ __device__ void cellscan_item(const BuildArgs& a, const CellGrid& sg, WarpScratc
           for (uint32_t m = amask; m != 0; m &= m - 1) {
             const int b = __ffs(m) - 1;
             const int t = 32 * b + lane;   // slot 64 (b / 2) + 32 (b % 2) + lane
-            dst[q++] = edge_key(__float_as_int(cs.cand[t].w), cs.ct[t]);
+            const int j = __float_as_int(cs.cand[t].w);
+            dst[q++] = a.stash_q ? stash_key(j, cs.ct[t], cs.cq[t]) : edge_key(j, cs.ct[t]);
           }
         }
         if (lane == 0) a.stash_n[i] = whole ? cnt : -1;

@@ -304,3 +304,22 @@ def test_forward_launch_counts(mlg):
         got = mlg.mlg_forward_launch_count(w.n_atoms, w.rcut, box, pbc, w.nnei_max, w.channels,
                                            w.heads, w.n_layers, dt)
         assert got == n, (w.name, got, n)
+
+
+def test_recorded_attention_traffic_names_the_launched_kernels(mlg):
+    """bench.py reports a stored DRAM capture as roofline.traffic only while
+    the library still launches the kernels it was taken on: each record must
+    name exactly what mlg_attention_kernels() returns for its workload, so that
+    a kernel change makes the stale figure drop out (and this test fail)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from neighbour_graph_attention_b200 import configs as C
+
+    assert bench.ATTN_TRAFFIC
+    for key, (name, traffic) in bench.ATTN_TRAFFIC.items():
+        w = C.workload(key)
+        dt = mlg.MLG_F64 if w.dtype == "f64" else mlg.MLG_F32
+        launched = mlg.mlg_attention_kernels(w.nnei_max, w.channels, w.heads, w.n_layers, dt)
+        assert launched == name, (key, launched, name)
+        assert traffic > 0

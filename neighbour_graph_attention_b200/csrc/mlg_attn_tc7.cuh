@@ -25,16 +25,18 @@
 //
 // Tiles of 128 rows hold up to two centres, each starting at a multiple of
 // 32 rows, so that every warp's TMEM lane quadrant belongs to one centre.
-//   projection  D[128 x 96] = X[128 x 32] . [Wq|Wk|Wv], 3xTF32 (12 MMAs)
+//   projection  D[128 x 96] = X[128 x 32] . [Wq|Wk|Wv], 3xTF32 (12 MMAs):
+//               A hi is the slab as TMA landed it (the tensor core reads the
+//               leading 19 bits of each fp32 value), A lo = x - those bits
+//               (formed by the groups, two float4 per thread)
 //   read-back   group h reads its head's q (scaled by s_a log2(e)/sqrt(d))
 //               and k (scaled by s_b) back and splits them into TF32 hi / lo
 //               operands: q into TMEM, the A operand of its row's centre
 //               (the other centre's operand gets a zero row), k into its
 //               centre's K-major shared-memory key operand at the key's
-//               slot; v as fp32
-//               rows with the two keys of a pair interleaved (two buffers
-//               per head, alternating between tiles)
-//   logits      per head, as soon as its group has read back: for each
+//               slot; v as fp32 rows with the two keys of a pair
+//               interleaved (two buffers per head, alternating between tiles)
+//   logits      per head, in the order the groups finish reading back: for each
 //               centre c, S[128 x N] += Q_h^c . (K_h^c)^T, 3 MMAs (lo.hi,
 //               hi.lo, hi.hi) with N the tile's longest row in 16s.  The zero
 //               rows make each centre's MMAs add exactly 0 to the other
@@ -48,7 +50,7 @@
 //               maxima over the four threads of a quad, 2^(S - max) on the
 //               special-function unit, the sums, then per 16 keys
 //               O += P_hi V_hi + P_hi V_lo + P_lo V_hi (three m16n8k16 MMAs):
-//               P = P_hi + P_lo with P_hi = P rounded to 11 significant bits
+//               P = P_hi + P_lo with P_hi = P rounded to a multiple of 2^-11
 //               and both halves fp16; v scaled by a power of two (the tile's
 //               largest |v| of the head below 2^14, so that no fp16 value
 //               overflows) and split the same way.  The rounding left is
@@ -62,15 +64,15 @@
 //
 // Warp roles (576 threads, one CTA per SM):
 //   warp 0      issues every MMA (one elected thread)
-//   warp 1      plans tiles two ahead (a window of row starts in the lanes),
-//               loads each slab with 2-D TMA boxes of {4 channels x 32 rows}
-//               straight into the K-major operand layout (two slab slots), and
-//               splits it into the TF32 hi / lo A operands of the projection
-//   warps 2-17  four groups of four warps, group h: the read-back of head h
-//               and the softmax and P V of head h
+//   warp 1      plans tiles two ahead (a window of row starts in the lanes)
+//               and loads each slab with 2-D TMA boxes of {4 channels x 32
+//               rows}, one per lane, straight into the K-major operand
+//               layout (two slab slots)
+//   warps 2-17  four groups of four warps, group h: the read-back of head h,
+//               a share of the next tile's A lo, the softmax and P V of head h
 // Every wait is bounded; on expiry the kernel records MLG_STATUS_TIMEOUT,
 // every role leaves its loop, the MMA thread waits for its own MMAs and the
-// producer for its last copy before TMEM is freed.
+// producer for the slab copies in flight before TMEM is freed.
 #pragma once
 
 #include <cuda.h>
@@ -256,8 +258,8 @@ __global__ void __launch_bounds__(tc7::NT, 1)
     // ------------------------------------------------------------ producer
     // The whole warp plans in step: lanes hold a window of 32 row starts
     // (the next window already loading), so a tile's plan costs shuffles, not
-    // a chain of global loads; slab t lands in slot t % 2 once the slab
-    // before it there is split, one copy per lane.
+    // a chain of global loads; slab t lands in slot t % 2, one copy per lane,
+    // once the projection of tile t - 2 (which read that slot) is done.
     const unsigned kFull = 0xffffffffu;
     int64_t c = 0, c_end = 0;
     if (lane == 0) {
@@ -718,7 +720,7 @@ __global__ void __launch_bounds__(tc7::NT, 1)
     }
     if (!ok) mt.fail = 1;
   }
-  // ---- teardown: report, let a slab copy in flight land, free TMEM
+  // ---- teardown: report, let the slab copies in flight land, free TMEM
   __syncthreads();
   if (tid == 0 && mt.fail) atomicOr(a.status, kStatusTimeout);
   if (warp == 1 && lane < 2 && mt.fail && mt.nissued[lane] > 0)   // a slab copy may still land

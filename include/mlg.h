@@ -65,7 +65,7 @@ typedef enum {
     MLG_ERR_WORKSPACE = 2,    /* ws_bytes smaller than the matching *_workspace_bytes() */
     MLG_ERR_CAPACITY = 3,     /* capacity < 0 */
     MLG_ERR_INPUT_DATA = 4,   /* reserved for host-visible data errors */
-    MLG_ERR_UNSUPPORTED = 5,  /* a shape this build does not handle (see each call) */
+    MLG_ERR_UNSUPPORTED = 5,  /* a shape the library does not handle (see each call) */
     MLG_ERR_CUDA = 6          /* a CUDA launch error (cudaGetLastError) */
 } mlg_status;
 
@@ -178,7 +178,7 @@ int mlg_build_csr_batch(const mlg_system* systems, int32_t n_systems, double rcu
                         int32_t nnei_max, const mlg_csr* csr, void* ws, size_t ws_bytes,
                         mlg_stream_t stream);
 
-/* Bytes of device workspace that mlg_block_attention needs (0 in this build). */
+/* Bytes of device workspace that mlg_block_attention needs (0: it needs none). */
 size_t mlg_attention_workspace_bytes(int64_t n_centres, int32_t nnei_max, int32_t channels,
                                      int32_t heads, mlg_dtype dtype);
 

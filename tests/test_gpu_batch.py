@@ -3,7 +3,7 @@ oracle's per-system graphs joined with atom and edge offsets -- bit for bit.
 
 The source pages batch many structures per GPU call (NValchemi batching) and
 report neighbour-cache defects after same-size refills, gradual cell
-changes and partition changes.  This build keeps no cache, so each of those
+changes and partition changes.  The library keeps no cache, so each of those
 cases must give the fresh graph; the tests run them in sequence on one
 workspace and one CSR.
 """

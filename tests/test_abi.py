@@ -323,3 +323,14 @@ def test_recorded_attention_traffic_names_the_launched_kernels(mlg):
         launched = mlg.mlg_attention_kernels(w.nnei_max, w.channels, w.heads, w.n_layers, dt)
         assert launched == name, (key, launched, name)
         assert traffic > 0
+
+
+def test_workspace_holds_the_key_stash_only_for_the_kernel_chain(mlg):
+    """Systems past the one-launch build get 516 bytes per atom more (the
+    count-to-fill key stash: 64 keys of 8 bytes and a count); the one-launch
+    build needs none."""
+    L64 = 2.855 * 32
+    chain = mlg.mlg_build_csr_workspace_bytes(65536, 6.0, np.diag([L64] * 3), [1, 1, 1])
+    assert chain > 65536 * 516
+    small = mlg.mlg_build_csr_workspace_bytes(512, 2.4, np.diag([3.567 * 4] * 3), [1, 1, 1])
+    assert 0 < small < 512 * 516

@@ -167,8 +167,8 @@ def _random_graph(n_atoms, density, rcut, nnei_max, seed):
     ("f64", 32, 4, 2, 0.2, 96),    # ~62 edges: fused tile (<= 64) + generic for larger rows
     ("f32", 64, 4, 1, 0.41, 181),  # ~128 edges: fused tile (<= 128) + generic for larger
     ("f32", 32, 4, 2, 0.004, 128), # dilute: many centres without edges between full ones
-    ("f32", 32, 4, 1, 0.13, 64),   # one layer, ragged rows <= 64: every product on tcgen05
-    ("f32", 32, 4, 1, 0.2, 128),   # ~62 edges: tcgen05 tiles (<= 64) + FP32-pipe tile (<= 128)
+    ("f32", 32, 4, 1, 0.13, 64),   # one layer, ragged rows <= 64: tcgen05 logits, mma.sync P.V
+    ("f32", 32, 4, 1, 0.2, 128),   # ~62 edges: tcgen05-logits tiles (<= 64) + FP32-pipe tile (<= 128)
     ("f32", 32, 4, 1, 0.41, 181),  # ~128 edges: both tile kernels + generic for larger rows
     ("f32", 32, 4, 1, 0.004, 64),  # dilute, one layer: centres without edges between
     ("f64", 128, 4, 2, 0.3, 96),   # head-group kernel, two layers (ping-pong)
@@ -213,8 +213,8 @@ def test_stack_mixed_row_sizes(dtype, channels, heads, n_layers, density, nnei):
 
 
 @pytest.mark.parametrize("dtype,channels,heads,n_layers,density,nnei", [
-    ("f32", 32, 4, 1, 0.13, 64),   # every product on tcgen05
-    ("f32", 32, 4, 1, 0.2, 128),   # tcgen05 tiles (<= 64) + FP32-pipe tile (<= 128)
+    ("f32", 32, 4, 1, 0.13, 64),   # tcgen05 logits, mma.sync P.V (rows <= 64)
+    ("f32", 32, 4, 1, 0.2, 128),   # tcgen05-logits tiles (<= 64) + FP32-pipe tile (<= 128)
     ("f32", 32, 4, 2, 0.2, 96),    # two fused layers on the FP32-pipe tile
     ("f32", 64, 4, 1, 0.41, 181),  # fused tile (<= 128) + generic for larger rows
     ("f32", 128, 8, 2, 0.31, 181), # head-group kernel (<= 96) + generic, two layers
@@ -358,7 +358,7 @@ def test_nan_feature_confined_to_its_centre():
 
 
 def test_nan_feature_confined_to_its_centre_f32_tensor_core_tiles():
-    """fp32, 32 channels, one layer (every product on tcgen05, two centres per
+    """fp32, 32 channels, one layer (tcgen05 logits, mma.sync P.V, two centres per
     tile): a NaN in one edge feature reaches every row of its centre and no
     row of any other centre, including the other centre of its tile."""
     import oracle

@@ -385,6 +385,28 @@ def test_nan_feature_confined_to_its_centre_f32_tensor_core_tiles():
     assert ok, err
 
 
+@pytest.mark.parametrize("scale", [1e-3, 1e-6])
+def test_f32_small_features_keep_fp32_precision(scale):
+    """fp32, 32 channels, one layer with features of scale 1e-3 and 1e-6: the
+    v values that P.V splits into fp16 halves are scaled up per tile, so the
+    lo halves of small values do not fall into fp16 subnormals."""
+    import oracle
+    from neighbour_graph_attention_b200.configs import Workload
+
+    gpu, csr_t = _random_graph(3000, 0.13, 4.2, 64, 17)
+    rp = gpu["row_ptr"]
+    e = gpu["n_edges"]
+    w = Workload(0, "random", "random", 0, 0, 0, 3000, 4.2, 3.7, 64, 32, 4, 1, "f32")
+    rng = np.random.default_rng(41)
+    W = [rng.normal(0, 1 / np.sqrt(32), (32, 32)).astype(np.float32) for _ in range(3)]
+    G = (rng.normal(size=(e, 32)) * scale).astype(np.float32)
+    out = U.gpu_attention(csr_t, 3000, w, G, *W)
+    sw = gpu["sw"].astype(np.float32).astype(np.float64)
+    ref = oracle.attention(rp, sw, G, *W, 4)
+    ok, err = U.attn_tolerance_ok(w, out, ref)
+    assert ok, err
+
+
 @pytest.mark.parametrize("case", ["f64-ragged", "f32-protein", "f64-full"])
 def test_smooth_attention_matches_oracle(case):
     """The slot-occupancy softmax (phantom slots of logit 0 up to nnei_max) on
